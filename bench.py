@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the DeepSeekMoE layer forward on B200: routed tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3p] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of T tokens:
+route (gate GEMM + sigmoid + biased top-K + gates + counts) -> permute ->
+routed expert FFN (up-projection + SwiGLU, down-projection) -> shared expert
+FFN -> combine with the residual -> bias update. With N > 1 (torchrun, one
+rank per GPU) every rank runs its own batch of T tokens (data parallel, weak
+scaling) and the per-expert counts are summed over ranks with one NCCL
+all-reduce before the bias update, so the bias stays identical everywhere.
+
+Rank 0 prints one JSON line. `value` is the whole-job throughput (all ranks'
+tokens / max-over-ranks device time) with inputs resident in HBM; `e2e` is the
+same metric through the public API with the batch copied from pinned host
+memory and the output copied back inside the timed region; `roofline` is the
+routed expert up-projection kernel (the dominant launch) against the measured
+bf16 tensor peak; `cpu_baseline` is the fp64 oracle on a bounded sample.
+`--impl reference` times that oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/sec per DeepSeekMoE layer on 1 B200; % of tensor/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("ptx.cuh", "gemm.cuh"):
+        h.update(open(os.path.join(ROOT, "mixture_experts_layer_58_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the up-projection kernel from the committed ncu
+    summary, or None if absent or taken on different kernel source."""
+    p = os.path.join(ROOT, "profiles", "expert_up_swiglu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_sha") != kernel_source_sha() or d.get("workload") != workload:
+        return None
+    return d.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is None:
+            return
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(cfg, u_host, e_host, b_host, expert_fn, shared_list, n_tokens):
+    """The oracle's full layer (route, routed + shared FFN, combine) on the
+    first n_tokens of the batch. Returns seconds."""
+    from oracle import moe_oracle as om
+    t0 = time.perf_counter()
+    u = u_host[:n_tokens]
+    out, _ = om.layer(u, e_host, b_host if cfg.gate_kind == "sigmoid" else None, expert_fn,
+                      shared_list, cfg.top_k, cfg.routed_scale, cfg.gate_kind)
+    assert out.shape[0] == n_tokens
+    return time.perf_counter() - t0
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def make_expert_fn(cfg, W_host=None):
+    from mixture_experts_layer_58_b200 import synth
+    cache = {}
+
+    def fn(i):
+        if i not in cache:
+            if W_host is not None:
+                ws = (W_host[0][i], W_host[1][i], W_host[2][i])
+            else:
+                ws = synth.expert_weights(cfg, i, "cuda" if cfg.weights_on_gpu else "cpu")
+            cache.clear()
+            cache[i] = tuple(w.float().cpu().numpy() for w in ws)
+        return cache[i]
+    return fn
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, cfg, rank):
+    """The fp64 oracle on the host cores as the reference arm, on this arm's
+    workload and metric: each step is the oracle's full layer over a bounded
+    sample of the batch's tokens."""
+    import torch
+    from mixture_experts_layer_58_b200 import synth
+    if rank != 0:
+        return
+    u, e, b = synth.tokens(cfg), synth.centroids(cfg), synth.bias(cfg)
+    shared = synth.shared_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
+    shared_list = [tuple(w.float().cpu().numpy() for w in shared)] if shared is not None else []
+    expert_fn = make_expert_fn(cfg)
+    # size the per-step sample so the whole run stays within ~2 minutes
+    probe = oracle_sample(cfg, u, e, b, expert_fn, shared_list, 1)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(cfg.T, budget / max(probe, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, u, e, b, expert_fn, shared_list, n)
+    times = [oracle_sample(cfg, u, e, b, expert_fn, shared_list, n) for _ in range(args.steps)]
+    sec = sum(times) / len(times)
+    tps = n / sec
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "n_routed": cfg.n_routed,
+                   "top_k": cfg.top_k, "n_shared": cfg.n_shared, "inter": cfg.inter,
+                   "routed_scale": cfg.routed_scale, "gate": cfg.gate_kind,
+                   "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"oracle full layer on the first {n} of {cfg.T} tokens per "
+                                   f"step (expert weights copied from the GPU on demand)"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    del torch
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="v3p")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from mixture_experts_layer_58_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from mixture_experts_layer_58_b200 import _lib as L
+    from mixture_experts_layer_58_b200 import build, dp
+    from mixture_experts_layer_58_b200.layer import MoELayer
+    build.build()
+    L.load()
+
+    # ---- inputs: same workload on every rank, each rank its own batch (seed + rank)
+    rcfg = cfg.replace(seed=cfg.seed + rank) if world > 1 else cfg
+    u_host = synth.tokens(rcfg)
+    e_host, b_host = synth.centroids(cfg), synth.bias(cfg)
+    W1, W3, W2 = synth.all_expert_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
+    shared = synth.shared_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
+    lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
+                   routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
+                   device=dev)
+    W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
+    del W1, W3, W2
+    torch.cuda.empty_cache()
+    T, K, d, I = cfg.T, cfg.top_k, cfg.d, cfg.inter
+    u = u_host.to(dev)
+    lay.allocate(T)
+    stream = torch.cuda.current_stream()
+    up_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+
+    def step(i=None):
+        lay.route(u)
+        lay.permute(u)
+        if i is not None:
+            up_ev[i][0].record(stream)
+        L.moe_expert_up_swiglu(lay.x_perm, lay.offsets, cfg.n_routed, T * K, d, I, lay.w13,
+                               lay.ffn_ws)
+        if i is not None:
+            up_ev[i][1].record(stream)
+        L.moe_expert_down(lay.ffn_ws, lay.offsets, cfg.n_routed, T * K, I, d, lay.w2, lay.y_perm)
+        lay.shared_ffn(u)
+        lay.combine(u)
+        if cfg.gate_kind == "sigmoid":
+            if world > 1:
+                lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
+            else:
+                lay.update_bias()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if L.moe_get_device_status() != 0:
+        raise SystemExit("device timeout during warm-up")
+
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = t_start.elapsed_time(t_end)
+    up_ms = sum(a.elapsed_time(b) for a, b in up_ev) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    if L.moe_get_device_status() != 0:
+        raise SystemExit("device timeout during the timed region")
+    ms_step = ms / args.steps
+    value = T * world / (ms_step * 1e-3)
+    counts = lay.counts.cpu()
+
+    # ---- e2e: host batch in pinned memory -> device, forward, output back
+    u_pin = u_host.pin_memory()
+    out_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    u_dev2 = torch.empty_like(u)
+
+    def e2e_step():
+        u_dev2.copy_(u_pin, non_blocking=True)
+        out = lay.forward(u_dev2)
+        if cfg.gate_kind == "sigmoid":
+            if world > 1:
+                lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
+            else:
+                lay.update_bias()
+        out_pin.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = T * world / (e2e_ms / args.steps * 1e-3)
+
+    # ---- roofline of the dominant kernel (routed up-projection + SwiGLU)
+    pk = peaks()
+    up_flops = 2.0 * T * K * d * 2 * I
+    achieved = up_flops / (up_ms * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
+                "kernel": "grouped_gemm_bf16_kernel<256,SwiGLU> (moe_expert_up_swiglu)",
+                "kernel_ms": up_ms,
+                "peak_source": f"{pk['_source']} bf16_tflops_sustained"}
+    layer_flops = T * cfg.flops_per_token()
+    layer_tflops = layer_flops / (ms_step * 1e-3) / 1e12
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights of the V3 layer shape)",
+        "config": {"workload": cfg.name, "T": T, "d": d, "n_routed": cfg.n_routed, "top_k": K,
+                   "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
+                   "gate": cfg.gate_kind, "global_batch_tokens": T * world,
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (22.6 GB of expert weights streamed per step)"
+                   if cfg.weights_on_gpu else "L2 not flushed: small workload",
+                   "max_expert_load": int(counts.max()), "mean_expert_load": T * K / cfg.n_routed},
+        "layer_tflops": layer_tflops,
+        "layer_frac_of_bf16_peak": layer_tflops / pk["bf16_tflops"],
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+                "d2h_bytes_per_step": T * d * 2},
+        "gpu_launches": args.steps * lay.launches_per_step(),
+        "clocks": clk.summary(),
+    }
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        expert_fn = make_expert_fn(cfg, W_host)
+        shared_list = ([tuple(w.float().cpu().numpy() for w in shared)]
+                       if shared is not None else [])
+        probe = oracle_sample(cfg, u_host, e_host, b_host, expert_fn, shared_list, 1)
+        n = int(max(1, min(T, args.cpu_seconds / max(probe, 1e-3))))
+        sec = oracle_sample(cfg, u_host, e_host, b_host, expert_fn, shared_list, n)
+        result["cpu_baseline"] = {
+            "value": n / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"oracle full layer (fp64) on the first {n} of {T} tokens, {sec:.1f} s; "
+                      f"host has {os.cpu_count()} cores"}
+
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

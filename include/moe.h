@@ -1,0 +1,217 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * The layer (DeepSeek-V3 technical report summary, xyznot.com, arXiv
+ * 2412.19437, Method §2 "DeepSeekMoE with auxiliary-loss-free balancing"):
+ *
+ *   h'_t = u_t + sum_{i<=N_s} FFN_i^(s)(u_t) + sum_{i<=N_r} g_{i,t} FFN_i^(r)(u_t)
+ *   s_{i,t} = Sigmoid(u_t . e_i)
+ *   g'_{i,t} = s_{i,t} if s_{i,t} + b_i is among the K_r largest of {s_{j,t} + b_j}, else 0
+ *   g_{i,t}  = S * g'_{i,t} / sum_j g'_{j,t}            (S: routed scale)
+ *   end of step: b_i -= gamma if expert i is overloaded, += gamma if underloaded
+ *
+ * A forward pass is five calls on one stream:
+ *   moe_route -> moe_permute -> moe_grouped_ffn (routed experts, then the
+ *   shared expert as one more group) -> moe_combine, then moe_bias_update.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned and allocated by the
+ *     caller; the library allocates no device memory. Scratch memory is passed
+ *     in as `workspace` (size from the matching *_workspace_size call).
+ *   - Tensors are dense row-major. bf16 tensors are raw 16-bit bfloat16.
+ *     Buffers read or written in 16-byte vectors or by TMA must be 16-byte
+ *     aligned (stated per argument); a misaligned pointer is rejected.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls
+ *     are asynchronous: they enqueue kernels and return; nothing is
+ *     synchronised and no device->host copy happens.
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code. Arguments are
+ *     validated on the host before anything is enqueued; on error nothing is
+ *     launched and outputs are untouched. MOE_ERR_CUDA keeps the CUDA error
+ *     for moe_last_cuda_error(). A kernel whose internal bounded wait gives
+ *     up (a broken pipeline, never a normal run) records a code that
+ *     moe_get_device_status() reports after the stream has drained.
+ *   - Tokens with index >= T, experts with no tokens and T = 0 are all valid:
+ *     an empty batch produces zero counts and enqueues no expert work.
+ *
+ * Supported shapes (others return MOE_ERR_UNSUPPORTED_SHAPE):
+ *   d % 256 == 0, inter % 128 == 0, 1 <= top_k <= 8, top_k <= n_routed <= 256,
+ *   1 <= G <= 1024 groups per grouped-FFN call.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* Status codes. */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)       /* null/misaligned pointer, negative size, bad enum */
+#define MOE_ERR_UNSUPPORTED_SHAPE (-2) /* shape outside the supported set above */
+#define MOE_ERR_CUDA (-3)              /* a CUDA runtime/driver call failed */
+#define MOE_ERR_DEVICE_TIMEOUT (-4)    /* a kernel's bounded wait ran out */
+#define MOE_ERR_WORKSPACE (-5)         /* workspace NULL or smaller than required */
+
+/* Gate form. SIGMOID_BIAS is the technical report's form (above).
+ * SOFTMAX_TOPK is the form of the DeepSeekMoE forward listing on "DeepSeek
+ * model architecture explained" (deepseekmodel.com): top-k over the raw
+ * logits z = u.e (no sigmoid, no bias), then softmax over the k selected
+ * logits, times the routed scale. */
+typedef enum { MOE_GATE_SIGMOID_BIAS = 0, MOE_GATE_SOFTMAX_TOPK = 1 } moe_gate_kind;
+
+/* Arithmetic type of the expert GEMM operands. MOE_FP8_E4M3 is reserved for
+ * the FP8 variant and currently returns MOE_ERR_UNSUPPORTED_SHAPE. */
+typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1 } moe_dtype;
+
+typedef void* moe_stream_t; /* cudaStream_t */
+
+/* ------------------------------------------------------------------ route
+ * Gate GEMM + affinity + bias-adjusted top-K + gate normalisation + load
+ * histogram (technical report summary, Method §2: s_{i,t}, the g'_{i,t}
+ * selection equation, the normalisation of g'; softmax form per the
+ * deepseekmodel.com DeepSeekMoE forward listing).
+ *
+ *   u          [T, d] bf16, 16-B aligned. Token hidden states.
+ *   centroids  [n_routed, d] bf16, 16-B aligned. e_i, one row per routed expert.
+ *   bias       [n_routed] fp32 or NULL (= all zero). b_i; used for SELECTION
+ *              only (the gate uses the unbiased s). Ignored for SOFTMAX_TOPK.
+ *   routed_scale  S, multiplies every normalised gate.
+ *   topk_idx   [T, top_k] int32 out. Selected experts in descending key
+ *              order; equal keys: lower expert index first.
+ *   topk_gate  [T, top_k] fp32 out. g of each selected expert (sums to S).
+ *   expert_counts [n_routed] int32 out, OVERWRITTEN (not accumulated):
+ *              number of (token, slot) pairs routed to each expert.
+ * Logits are accumulated in fp32 on the tensor cores from the bf16 inputs;
+ * sigmoid, keys and gates are fp32.
+ */
+MOE_API int moe_route(const void* u, const void* centroids, const float* bias, int T, int d,
+                      int n_routed, int top_k, moe_gate_kind kind, float routed_scale,
+                      int32_t* topk_idx, float* topk_gate, int32_t* expert_counts,
+                      moe_stream_t stream);
+
+/* ------------------------------------------------------------------ permute
+ * Dispatch: copy each token's row into an expert-contiguous buffer, once per
+ * selected expert (the per-expert grouping of tokens that the deepseekmodel.com
+ * DeepSeekMoE listing does with a mask, written as explicit row numbers).
+ * Rows of expert i occupy [expert_offsets[i], expert_offsets[i+1]); inside an
+ * expert, rows are in ascending token order (stable).
+ *
+ *   u              [T, d] bf16, 16-B aligned.
+ *   topk_idx       [T, top_k] int32 from moe_route (entries outside
+ *                  [0, n_routed) are skipped and get pos = -1).
+ *   expert_counts  [n_routed] int32 from moe_route.
+ *   x_perm         [T*top_k, d] bf16 out, 16-B aligned.
+ *   expert_offsets [n_routed + 1] int32 out: exclusive scan of the counts.
+ *   pos            [T, top_k] int32 out: row of x_perm holding (t, slot k).
+ *   src_token      [T*top_k] int32 out: token of each x_perm row.
+ *   workspace      >= moe_permute_workspace_size(T, n_routed) bytes, 16-B aligned.
+ */
+MOE_API int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* expert_counts,
+                        int T, int d, int n_routed, int top_k, void* x_perm,
+                        int32_t* expert_offsets, int32_t* pos, int32_t* src_token,
+                        void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+MOE_API size_t moe_permute_workspace_size(int T, int n_routed);
+
+/* ------------------------------------------------------------------ expert FFN
+ * Grouped SwiGLU expert FFN (FFN_i^(r) and FFN_i^(s) of the technical report's
+ * output equation; the pages do not define the FFN's inside — SwiGLU without
+ * biases, FFN(x) = W2 (silu(W1 x) * (W3 x)), is this library's reading).
+ *
+ * Group g owns rows [group_offsets[g], group_offsets[g+1]) of x and its own
+ * weights. group_offsets is a DEVICE array of G+1 non-decreasing int32 with
+ * group_offsets[G] <= rows (rows outside every group are not written).
+ *
+ *   x      [rows, d] bf16, 16-B aligned.
+ *   w13    [G, 2*inter, d] bf16, 16-B aligned: W1 and W3 of each group,
+ *          row-interleaved in 128-row chunks ([W1 rows 0..127; W3 rows
+ *          0..127; W1 rows 128..255; ...]); moe_pack_w13 builds it.
+ *   w2     [G, d, inter] bf16, 16-B aligned.
+ *   y      [rows, d] bf16 out, 16-B aligned.
+ *   workspace >= moe_grouped_ffn_workspace_size(rows, inter, dtype): holds
+ *          h = silu(x W1^T) * (x W3^T) as bf16 [rows, inter].
+ * The shared expert(s) run as G = 1 with group_offsets = {0, T}, x = u and
+ * the N_s shared experts' weights concatenated along inter.
+ * x_scales / w13_scales / w2_scales are for the FP8 variant; pass NULL.
+ */
+MOE_API int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_offsets,
+                            int G, int rows, int d, int inter, const void* w13,
+                            const float* w13_scales, const void* w2, const float* w2_scales,
+                            moe_dtype dtype, void* y, void* workspace, size_t ws_bytes,
+                            moe_stream_t stream);
+
+MOE_API size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dtype);
+
+/* The two halves of moe_grouped_ffn, for callers that keep h themselves.
+ * moe_expert_up_swiglu:  h[rows, inter] = silu(x W1^T) * (x W3^T) per group.
+ * moe_expert_down:       y[rows, d]     = h W2^T per group.
+ * Same argument rules as moe_grouped_ffn; h is bf16, 16-B aligned. */
+MOE_API int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, int G, int rows,
+                                 int d, int inter, const void* w13, void* h,
+                                 moe_stream_t stream);
+MOE_API int moe_expert_down(const void* h, const int32_t* group_offsets, int G, int rows,
+                            int inter, int d, const void* w2, void* y, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ combine
+ * out_t = residual_t + shared_t + sum_k topk_gate[t,k] * y_perm[pos[t,k]]
+ * (the technical report's output equation h'_t). Sums in fp32, one rounding
+ * to bf16; a gather per token, no atomics, deterministic.
+ *
+ *   y_perm     [T*top_k, d] bf16, 16-B aligned (moe_grouped_ffn output).
+ *   pos        [T, top_k] int32 (moe_permute output; negative = skip).
+ *   topk_gate  [T, top_k] fp32 (moe_route output).
+ *   shared_out [T, d] bf16 or NULL (no shared expert).
+ *   residual   [T, d] bf16 or NULL (the listing form without residual).
+ *   out        [T, d] bf16 out, 16-B aligned. May alias residual.
+ */
+MOE_API int moe_combine(const void* y_perm, const int32_t* pos, const float* topk_gate,
+                        const void* shared_out, const void* residual, int T, int d, int top_k,
+                        void* out, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ bias update
+ * Auxiliary-loss-free balancing (technical report summary, Method §2): at the
+ * end of a step, b_i <- b_i - gamma if expert i is overloaded and
+ * b_i <- b_i + gamma if it is underloaded. Load is compared with the mean
+ * T*top_k/n_routed exactly in integers (n_routed*c_i vs T*top_k); an expert
+ * exactly at the mean is unchanged. bias is fp32 state, updated in place.
+ * For data-parallel use, pass counts already summed over all ranks and the
+ * global T.
+ */
+MOE_API int moe_bias_update(const int32_t* expert_counts, float* bias, int n_routed,
+                            long long T, int top_k, float gamma, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ helpers
+ * moe_pack_w13: build the interleaved w13 [G, 2*inter, d] from w1 and w3
+ * [G, inter, d] (all bf16, 16-B aligned; layout described at moe_grouped_ffn).
+ */
+MOE_API int moe_pack_w13(const void* w1, const void* w3, int G, int inter, int d, void* w13,
+                         moe_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+MOE_API const char* moe_strerror(int status);
+
+/* The CUDA error code behind the calling thread's last MOE_ERR_CUDA (0 if none). */
+MOE_API int moe_last_cuda_error(void);
+
+/* Synchronises the current device, then writes the device status word of the
+ * current device (0 = no kernel timed out) to *status; clears it if `clear`.
+ * Returns MOE_ERR_DEVICE_TIMEOUT if the word was non-zero. */
+MOE_API int moe_get_device_status(unsigned int* status, int clear);
+
+/* Library version, major*10000 + minor*100 + patch. */
+MOE_API int moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,177 @@
+"""ctypes binding of libmoe.so: the C-ABI entry points under the same names.
+
+Argument marshalling only: tensors become device pointers (data_ptr()),
+None becomes NULL, the stream defaults to torch's current CUDA stream. Every
+non-zero status raises MoEError. There is no fallback: if the library is
+missing, loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED_SHAPE = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_DEVICE_TIMEOUT = -4
+MOE_ERR_WORKSPACE = -5
+
+MOE_GATE_SIGMOID_BIAS = 0
+MOE_GATE_SOFTMAX_TOPK = 1
+MOE_BF16 = 0
+MOE_FP8_E4M3 = 1
+
+GATE_KINDS = {"sigmoid": MOE_GATE_SIGMOID_BIAS, "softmax": MOE_GATE_SOFTMAX_TOPK}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: status {status}"
+        try:
+            msg += f" ({_L().moe_strerror(status).decode()})"
+            if status == MOE_ERR_CUDA:
+                msg += f", cuda error {_L().moe_last_cuda_error()}"
+        except Exception:  # noqa: BLE001 - the message is best effort
+            pass
+        super().__init__(msg)
+
+
+_vp, _i, _ll, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+
+_SIGS = {
+    "moe_route": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp]),
+    "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_workspace_size": (_sz, [_i, _i]),
+    "moe_grouped_ffn": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp,
+                             _sz, _vp]),
+    "moe_grouped_ffn_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_expert_up_swiglu": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_expert_down": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_combine": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_bias_update": (_i, [_vp, _vp, _i, _ll, _i, _f, _vp]),
+    "moe_pack_w13": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_strerror": (ctypes.c_char_p, [_i]),
+    "moe_last_cuda_error": (_i, []),
+    "moe_get_device_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i]),
+    "moe_version": (_i, []),
+}
+
+_LIB = None
+
+
+def _L():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built: run "
+                              "`python -m mixture_experts_layer_58_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def load():
+    """Load libmoe.so (raises if absent) and return the ctypes handle."""
+    return _L()
+
+
+def _p(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != MOE_OK:
+        raise MoEError(rc, where)
+
+
+def moe_route(u, centroids, bias, T, d, n_routed, top_k, kind, routed_scale, topk_idx,
+              topk_gate, expert_counts, stream=None):
+    k = GATE_KINDS.get(kind, kind)
+    _check(_L().moe_route(_p(u), _p(centroids), _p(bias), T, d, n_routed, top_k, k,
+                          float(routed_scale), _p(topk_idx), _p(topk_gate), _p(expert_counts),
+                          _stream(stream)), "moe_route")
+
+
+def moe_permute(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm, expert_offsets, pos,
+                src_token, workspace, ws_bytes, stream=None):
+    _check(_L().moe_permute(_p(u), _p(topk_idx), _p(expert_counts), T, d, n_routed, top_k,
+                            _p(x_perm), _p(expert_offsets), _p(pos), _p(src_token),
+                            _p(workspace), ws_bytes, _stream(stream)), "moe_permute")
+
+
+def moe_permute_workspace_size(T, n_routed) -> int:
+    return _L().moe_permute_workspace_size(T, n_routed)
+
+
+def moe_grouped_ffn(x, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales, w2,
+                    w2_scales, dtype, y, workspace, ws_bytes, stream=None):
+    _check(_L().moe_grouped_ffn(_p(x), _p(x_scales), _p(group_offsets), G, rows, d, inter,
+                                _p(w13), _p(w13_scales), _p(w2), _p(w2_scales), dtype, _p(y),
+                                _p(workspace), ws_bytes, _stream(stream)), "moe_grouped_ffn")
+
+
+def moe_grouped_ffn_workspace_size(rows, inter, dtype=MOE_BF16) -> int:
+    return _L().moe_grouped_ffn_workspace_size(rows, inter, dtype)
+
+
+def moe_expert_up_swiglu(x, group_offsets, G, rows, d, inter, w13, h, stream=None):
+    _check(_L().moe_expert_up_swiglu(_p(x), _p(group_offsets), G, rows, d, inter, _p(w13), _p(h),
+                                     _stream(stream)), "moe_expert_up_swiglu")
+
+
+def moe_expert_down(h, group_offsets, G, rows, inter, d, w2, y, stream=None):
+    _check(_L().moe_expert_down(_p(h), _p(group_offsets), G, rows, inter, d, _p(w2), _p(y),
+                                _stream(stream)), "moe_expert_down")
+
+
+def moe_combine(y_perm, pos, topk_gate, shared_out, residual, T, d, top_k, out, stream=None):
+    _check(_L().moe_combine(_p(y_perm), _p(pos), _p(topk_gate), _p(shared_out), _p(residual), T,
+                            d, top_k, _p(out), _stream(stream)), "moe_combine")
+
+
+def moe_bias_update(expert_counts, bias, n_routed, T, top_k, gamma, stream=None):
+    _check(_L().moe_bias_update(_p(expert_counts), _p(bias), n_routed, int(T), top_k,
+                                float(gamma), _stream(stream)), "moe_bias_update")
+
+
+def moe_pack_w13(w1, w3, G, inter, d, w13, stream=None):
+    _check(_L().moe_pack_w13(_p(w1), _p(w3), G, inter, d, _p(w13), _stream(stream)),
+           "moe_pack_w13")
+
+
+def moe_get_device_status(clear: bool = True) -> int:
+    v = ctypes.c_uint(0)
+    rc = _L().moe_get_device_status(ctypes.byref(v), 1 if clear else 0)
+    if rc not in (MOE_OK, MOE_ERR_DEVICE_TIMEOUT):
+        raise MoEError(rc, "moe_get_device_status")
+    return int(v.value)
+
+
+def moe_strerror(status: int) -> str:
+    return _L().moe_strerror(status).decode()
+
+
+def moe_version() -> int:
+    return _L().moe_version()

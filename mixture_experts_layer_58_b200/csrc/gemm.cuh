@@ -1,0 +1,285 @@
+// Grouped bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA)
+// for the expert FFNs: per group g, D_g = A[rows of g] * B_g^T, both operands
+// K-major. Epilogues: plain bf16 store, or SwiGLU over interleaved W1/W3 column
+// pairs (h = silu(a) * b).
+//
+// One persistent CTA per SM, 6 warps:
+//   warp 0      TMA producer (one elected lane): A and B tiles into a
+//               4-stage shared-memory ring (128B-swizzled, K block 64).
+//   warp 1      MMA issuer (one elected lane): tcgen05.mma M=128, N=BN, K=16
+//               into one of two TMEM accumulators (2 x BN fp32 columns).
+//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator (one TMEM
+//               lane = one output row per thread), convert, store to global;
+//               runs while the MMA warp fills the other accumulator.
+// Tiles are (group, m-block of 128 rows, n-block of BN columns); within a
+// group the m-blocks of one n-block are consecutive so the CTAs running at
+// the same time share the weight tile through L2. The tile list is rebuilt
+// on the device from group_offsets: no host round trip for the group sizes.
+#pragma once
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128;        // rows per tile (UMMA M)
+constexpr int kBK = 64;         // bf16 K elements per stage = one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
+constexpr int kGemmThreads = 192;
+constexpr int kMaxGroups = 1024;
+
+enum { EPI_STORE = 0, EPI_SWIGLU = 1 };
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;   // double-buffered accumulator
+  static constexpr int kBarBytes = 256;
+  static size_t smem_bytes(int G) {
+    return 1024 + static_cast<size_t>(kStages) * kStageBytes + kBarBytes +
+           2 * static_cast<size_t>(G + 1) * sizeof(int);
+  }
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// tile index -> (group, m block, n block); m blocks fastest inside a group.
+__device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const int* s_off, int G,
+                                            int& g, int& m_blk, int& n_blk) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_tstart[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  const int local = t - s_tstart[g];
+  const int mt = (s_off[g + 1] - s_off[g] + kBM - 1) / kBM;
+  n_blk = local / mt;
+  m_blk = local - n_blk * mt;
+}
+
+__device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + __expf(-a)); }
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB,
+                         const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
+                         int rows, __nv_bfloat16* __restrict__ out, int ldo,
+                         unsigned int* status) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * C::kBBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
+  int* s_tstart = s_off + (G + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_blocks_n = n_per_group / BN;
+  const int num_kb = K / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(&full[s], 1);
+        mbar_init(&empty[s], 1);
+      }
+      for (int a = 0; a < 2; ++a) {
+        mbar_init(&tfull[a], 1);
+        mbar_init(&tempty[a], 128);
+      }
+      mbar_init(mma_done, 1);
+      fence_mbar_init();
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+    }
+    __syncwarp();
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  } else if (warp == 1) {
+    // Group table: row offsets and the first tile of every group (warp scan).
+    int carry = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int nt = 0;
+      if (g < G) {
+        const int o0 = offsets[g];
+        const int o1 = offsets[g + 1];
+        s_off[g] = o0;
+        nt = (o1 > o0 ? (o1 - o0 + kBM - 1) / kBM : 0) * n_blocks_n;
+      }
+      int v = nt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+      }
+      if (g < G) s_tstart[g] = carry + v - nt;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) {
+      s_tstart[G] = carry;
+      s_off[G] = offsets[G];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = s_tstart[G];
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, issued_par = 0;   // per stage: ever filled / parity of last fill
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      int g, m_blk, n_blk;
+      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      const int a_row = s_off[g] + m_blk * kBM;
+      const int b_row = g * n_per_group + n_blk * BN;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, status, kStatusTimeoutProducer)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+        tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * kBK, a_row);
+        tma_load_2d(sB + stage * C::kBBytes, &tmB, &full[stage], kb * kBK, b_row);
+        issued |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Never leave with a TMA write into shared memory still in flight.
+    for (int s = 0; s < kStages; ++s)
+      if (issued & (1u << s))
+        mbar_wait(&full[s], (issued_par >> s) & 1u, status, kStatusTimeoutProducer);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int local = 0;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      if (!mbar_wait(&tempty[acc], acc_par ^ 1u, status, kStatusTimeoutMma)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&full[stage], phase, status, kStatusTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * C::kABytes));
+        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * C::kBBytes));
+#pragma unroll
+        for (int k = 0; k < kBK / kUmmaK; ++k) {
+          // advance 16 bf16 = 32 bytes along K inside the swizzle row
+          umma_bf16(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+        }
+        umma_commit(&empty[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) umma_commit(&tfull[acc]);
+    }
+    // Every issued MMA has finished before TMEM is released.
+    umma_commit(mma_done);
+    mbar_wait(mma_done, 0, status, kStatusTimeoutMma);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;               // TMEM lanes this warp may read
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    int local = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+      int g, m_blk, n_blk;
+      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      const int acc = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_par, status, kStatusTimeoutEpilogue)) break;
+      tc_fence_after();
+      const int grow = s_off[g] + m_blk * kBM + row_in_tile;
+      const int row_end = min(s_off[g + 1], rows);
+      const bool valid = grow < row_end;
+      const uint32_t taddr = tmem_base + acc * BN + lane_addr;
+      if constexpr (EPI == EPI_SWIGLU) {
+        // accumulator columns [0,128) = x.W1 rows, [128,256) = x.W3 rows of the
+        // same 128 h columns
+        static_assert(BN == 256, "SwiGLU epilogue pairs 128 gate with 128 up columns");
+        __nv_bfloat16* dst_row = out + static_cast<size_t>(grow) * ldo + n_blk * 128;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t ga[32], up[32];
+          tmem_ld_32cols(taddr + c, ga);
+          tmem_ld_32cols(taddr + 128 + c, up);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f32(__uint_as_float(ga[2 * i])) * __uint_as_float(up[2 * i]);
+              const float h1 =
+                  silu_f32(__uint_as_float(ga[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      } else {
+        __nv_bfloat16* dst_row = out + static_cast<size_t>(grow) * ldo + n_blk * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32cols(taddr + c, r);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace moe

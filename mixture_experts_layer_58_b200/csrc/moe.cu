@@ -1,0 +1,391 @@
+// C-ABI entry points of libmoe.so (declared in include/moe.h): host-side
+// validation, TMA tensor-map construction and kernel launches. Every entry
+// point checks its arguments before touching the GPU and returns a status
+// code; nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "moe.h"
+#include "dispatch.cuh"
+#include "gemm.cuh"
+#include "route.cuh"
+
+namespace {
+
+using namespace moe;
+
+__device__ unsigned int g_status;   // per-device status word (see moe_get_device_status)
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+inline int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_CUDA(call)                        \
+  do {                                        \
+    cudaError_t _e = (call);                  \
+    if (_e != cudaSuccess) return cuda_fail(_e); \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device constants, looked up once.
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_INVALID_ARG;
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!di.ready) {
+      MOE_CUDA(cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev));
+      void* p = nullptr;
+      MOE_CUDA(cudaGetSymbolAddress(&p, g_status));
+      di.status = static_cast<unsigned int*>(p);
+      di.ready = true;
+    }
+  }
+  *out = &di;
+  return MOE_OK;
+}
+
+int get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) {
+    t_last_cuda_error = static_cast<int>(cudaErrorNotSupported);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix, box
+// [box_rows, 64 columns], 128-byte swizzle, zero fill out of bounds.
+int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                   uint32_t box_rows) {
+  int rc = get_encoder();
+  if (rc != MOE_OK) return rc;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+template <typename K>
+int set_smem(K kernel, size_t bytes) {
+  MOE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(bytes)));
+  return MOE_OK;
+}
+
+inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ------------------------------------------------------------------ GEMM launch
+template <int BN, int EPI>
+int launch_grouped_gemm(const void* A, int rows, int K, const void* B, int G, int n_per_group,
+                        const int32_t* offsets, void* out, int ldo, cudaStream_t st) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  CUtensorMap tmA, tmB;
+  if ((rc = make_tmap_bf16(&tmA, A, K, rows, kBM)) != MOE_OK) return rc;
+  if ((rc = make_tmap_bf16(&tmB, B, K, static_cast<uint64_t>(G) * n_per_group, BN)) != MOE_OK)
+    return rc;
+  const size_t smem = GemmCfg<BN>::smem_bytes(G);
+  auto kern = grouped_gemm_bf16_kernel<BN, EPI>;
+  if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
+  const long long max_tiles =
+      (static_cast<long long>(rows) / kBM + G) * static_cast<long long>(n_per_group / BN);
+  const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
+  kern<<<grid, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
+                                         static_cast<__nv_bfloat16*>(out), ldo, di->status);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int check_ffn_shape(int G, int rows, int d, int inter) {
+  if (G < 1 || rows < 0 || d <= 0 || inter <= 0) return MOE_ERR_INVALID_ARG;
+  if (G > kMaxGroups || d % 256 != 0 || inter % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(G) * 2 * inter > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+template <int TOPK>
+int launch_route_k(int kind, const CUtensorMap& tmU, const CUtensorMap& tmE, const float* bias,
+                   int T, int d, int n_routed, int n_pad, uint32_t tcols, float scale,
+                   int32_t* idx, float* gate, int32_t* counts, unsigned int* status,
+                   cudaStream_t st) {
+  const size_t smem = RouteSmem::bytes(n_pad);
+  const int grid = (T + kBM - 1) / kBM;
+  int rc;
+  if (kind == MOE_GATE_SIGMOID_BIAS) {
+    auto k = route_kernel<TOPK, 0>;
+    if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
+    k<<<grid, kGemmThreads, smem, st>>>(tmU, tmE, bias, T, d, n_routed, n_pad, tcols, scale, idx,
+                                        gate, counts, status);
+  } else {
+    auto k = route_kernel<TOPK, 1>;
+    if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
+    k<<<grid, kGemmThreads, smem, st>>>(tmU, tmE, bias, T, d, n_routed, n_pad, tcols, scale, idx,
+                                        gate, counts, status);
+  }
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_version(void) { return 100; }
+
+const char* moe_strerror(int s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer, bad size or enum)";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA error (see moe_last_cuda_error)";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int moe_last_cuda_error(void) { return t_last_cuda_error; }
+
+int moe_get_device_status(unsigned int* status, int clear) {
+  if (!status) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  MOE_CUDA(cudaDeviceSynchronize());
+  unsigned int v = 0;
+  MOE_CUDA(cudaMemcpyFromSymbol(&v, g_status, sizeof(v)));
+  if (clear && v) {
+    const unsigned int zero = 0;
+    MOE_CUDA(cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)));
+  }
+  *status = v;
+  return v ? MOE_ERR_DEVICE_TIMEOUT : MOE_OK;
+}
+
+// ------------------------------------------------------------------ route
+int moe_route(const void* u, const void* centroids, const float* bias, int T, int d, int n_routed,
+              int top_k, moe_gate_kind kind, float routed_scale, int32_t* topk_idx,
+              float* topk_gate, int32_t* expert_counts, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (kind != MOE_GATE_SIGMOID_BIAS && kind != MOE_GATE_SOFTMAX_TOPK) return MOE_ERR_INVALID_ARG;
+  if (!expert_counts || !centroids || !aligned16(centroids)) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!u || !topk_idx || !topk_gate || !aligned16(u))) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 256 != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!(routed_scale == routed_scale)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  MOE_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * n_routed, st));
+  if (T == 0) return MOE_OK;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int n_pad = std::max(16, (n_routed + 15) / 16 * 16);
+  uint32_t tcols = 32;
+  while (tcols < static_cast<uint32_t>(n_pad)) tcols <<= 1;
+  CUtensorMap tmU, tmE;
+  if ((rc = make_tmap_bf16(&tmU, u, d, T, kBM)) != MOE_OK) return rc;
+  if ((rc = make_tmap_bf16(&tmE, centroids, d, n_routed, n_pad)) != MOE_OK) return rc;
+  const float* b = (kind == MOE_GATE_SIGMOID_BIAS) ? bias : nullptr;
+#define MOE_ROUTE_CASE(KK)                                                                   \
+  case KK:                                                                                   \
+    return launch_route_k<KK>(kind, tmU, tmE, b, T, d, n_routed, n_pad, tcols, routed_scale, \
+                              topk_idx, topk_gate, expert_counts, di->status, st);
+  switch (top_k) {
+    MOE_ROUTE_CASE(1)
+    MOE_ROUTE_CASE(2)
+    MOE_ROUTE_CASE(3)
+    MOE_ROUTE_CASE(4)
+    MOE_ROUTE_CASE(5)
+    MOE_ROUTE_CASE(6)
+    MOE_ROUTE_CASE(7)
+    MOE_ROUTE_CASE(8)
+    default: return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+#undef MOE_ROUTE_CASE
+}
+
+// ------------------------------------------------------------------ permute
+size_t moe_permute_workspace_size(int T, int n_routed) {
+  if (T <= 0 || n_routed <= 0) return 16;
+  const size_t chunks = (static_cast<size_t>(T) + kPermChunk - 1) / kPermChunk;
+  return (chunks * n_routed * sizeof(int32_t) + 255) / 256 * 256;
+}
+
+int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* expert_counts, int T, int d,
+                int n_routed, int top_k, void* x_perm, int32_t* expert_offsets, int32_t* pos,
+                int32_t* src_token, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 256 != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = as_stream(stream);
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (n_routed + 1), st));
+    return MOE_OK;
+  }
+  if (!u || !topk_idx || !x_perm || !pos || !src_token || !aligned16(u) || !aligned16(x_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < moe_permute_workspace_size(T, n_routed) || !aligned16(workspace))
+    return MOE_ERR_WORKSPACE;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int chunks = (T + kPermChunk - 1) / kPermChunk;
+  int32_t* hist = static_cast<int32_t*>(workspace);
+  permute_hist_kernel<<<chunks, 256, 0, st>>>(topk_idx, T, top_k, n_routed, hist);
+  MOE_CUDA(cudaGetLastError());
+  permute_index_kernel<<<chunks, 256, 0, st>>>(topk_idx, expert_counts, hist, T, top_k, n_routed,
+                                               expert_offsets, pos, src_token);
+  MOE_CUDA(cudaGetLastError());
+  const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
+  permute_copy_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(u), pos, T, d,
+                                              top_k, static_cast<__nv_bfloat16*>(x_perm));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ expert FFN
+size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dtype) {
+  (void)dtype;
+  if (rows <= 0 || inter <= 0) return 256;
+  return (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
+}
+
+int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, int G, int rows, int d,
+                         int inter, const void* w13, void* h, moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!x || !group_offsets || !w13 || !h || !aligned16(x) || !aligned16(w13) || !aligned16(h))
+    return MOE_ERR_INVALID_ARG;
+  return launch_grouped_gemm<256, EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
+                                              inter, as_stream(stream));
+}
+
+int moe_expert_down(const void* h, const int32_t* group_offsets, int G, int rows, int inter, int d,
+                    const void* w2, void* y, moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!h || !group_offsets || !w2 || !y || !aligned16(h) || !aligned16(w2) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  return launch_grouped_gemm<256, EPI_STORE>(h, rows, inter, w2, G, d, group_offsets, y, d,
+                                             as_stream(stream));
+}
+
+int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_offsets, int G,
+                    int rows, int d, int inter, const void* w13, const float* w13_scales,
+                    const void* w2, const float* w2_scales, moe_dtype dtype, void* y,
+                    void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (dtype != MOE_BF16 && dtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_FP8_E4M3) return MOE_ERR_UNSUPPORTED_SHAPE;
+  (void)x_scales;
+  (void)w13_scales;
+  (void)w2_scales;
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!workspace || ws_bytes < moe_grouped_ffn_workspace_size(rows, inter, dtype) ||
+      !aligned16(workspace))
+    return MOE_ERR_WORKSPACE;
+  rc = moe_expert_up_swiglu(x, group_offsets, G, rows, d, inter, w13, workspace, stream);
+  if (rc != MOE_OK) return rc;
+  return moe_expert_down(workspace, group_offsets, G, rows, inter, d, w2, y, stream);
+}
+
+// ------------------------------------------------------------------ combine
+int moe_combine(const void* y_perm, const int32_t* pos, const float* topk_gate,
+                const void* shared_out, const void* residual, int T, int d, int top_k, void* out,
+                moe_stream_t stream) {
+  if (T < 0 || d <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!y_perm || !pos || !topk_gate || !out || !aligned16(y_perm) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if ((shared_out && !aligned16(shared_out)) || (residual && !aligned16(residual)))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
+  combine_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(y_perm), pos, topk_gate,
+      static_cast<const __nv_bfloat16*>(shared_out), static_cast<const __nv_bfloat16*>(residual),
+      T, d, top_k, static_cast<__nv_bfloat16*>(out));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ bias update
+int moe_bias_update(const int32_t* expert_counts, float* bias, int n_routed, long long T,
+                    int top_k, float gamma, moe_stream_t stream) {
+  if (!expert_counts || !bias || n_routed <= 0 || T < 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (!(gamma == gamma)) return MOE_ERR_INVALID_ARG;
+  bias_update_kernel<<<(n_routed + 255) / 256, 256, 0, as_stream(stream)>>>(
+      expert_counts, bias, n_routed, T * top_k, gamma);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ helpers
+int moe_pack_w13(const void* w1, const void* w3, int G, int inter, int d, void* w13,
+                 moe_stream_t stream) {
+  if (G <= 0 || inter <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (inter % 128 != 0 || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!w1 || !w3 || !w13 || !aligned16(w1) || !aligned16(w3) || !aligned16(w13))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  pack_w13_kernel<<<di->num_sms * 4, 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(w1), static_cast<const __nv_bfloat16*>(w3), G, inter, d,
+      static_cast<__nv_bfloat16*>(w13));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+}  // extern "C"

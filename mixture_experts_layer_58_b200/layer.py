@@ -1,0 +1,156 @@
+"""MoELayer: device buffers plus the sequence of C-ABI calls of one forward.
+
+PyTorch supplies device memory and the stream; every step of the layer runs
+in libmoe.so's kernels:
+
+    moe_route        gate GEMM + sigmoid + biased top-K + gates + counts
+    moe_permute      expert-contiguous copy of the token rows
+    moe_grouped_ffn  routed experts (G = N_r) then the shared expert (G = 1)
+    moe_combine      h' = u + shared + sum_k g * y
+    moe_bias_update  b -= / += gamma from the loads (end of the step)
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+class MoELayer:
+    """One DeepSeekMoE layer resident on a CUDA device.
+
+    Weights are given in the natural layout: w1, w3 [N_r, I, d], w2 [N_r, d, I]
+    (bf16) for the routed experts; ws1, ws3 [N_s*I, d], ws2 [d, N_s*I] for the
+    shared experts concatenated along I (or None); centroids [N_r, d] bf16;
+    bias [N_r] fp32 (the layer keeps its own device copy, updated in place).
+    """
+
+    def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
+                 routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
+                 device="cuda"):
+        L.load()
+        dev = torch.device(device)
+        self.device = dev
+        self.n_routed, self.d = centroids.shape
+        self.inter = w1.shape[1]
+        self.top_k = int(top_k)
+        self.routed_scale = float(routed_scale)
+        self.gate_kind = gate_kind
+        self.gamma = float(gamma)
+        bf = torch.bfloat16
+        self.centroids = centroids.to(dev, bf).contiguous()
+        self.bias = (bias.to(dev, torch.float32).contiguous() if bias is not None
+                     else torch.zeros(self.n_routed, dtype=torch.float32, device=dev))
+        self.w13 = self.pack_w13(w1.to(dev, bf).contiguous(), w3.to(dev, bf).contiguous())
+        self.w2 = w2.to(dev, bf).contiguous()
+        if shared is not None:
+            ws1, ws3, ws2 = shared
+            self.shared_inter = ws1.shape[0]
+            self.ws13 = self.pack_w13(ws1.to(dev, bf).contiguous()[None],
+                                      ws3.to(dev, bf).contiguous()[None])
+            self.ws2 = ws2.to(dev, bf).contiguous()
+        else:
+            self.shared_inter = 0
+            self.ws13 = self.ws2 = None
+        self._T = -1
+
+    # ------------------------------------------------------------------ setup
+    def pack_w13(self, w1, w3):
+        G, inter, d = w1.shape
+        w13 = torch.empty((G, 2 * inter, d), dtype=torch.bfloat16, device=self.device)
+        L.moe_pack_w13(w1, w3, G, inter, d, w13)
+        return w13
+
+    def allocate(self, T: int) -> None:
+        """(Re)allocate the activation buffers for a batch of T tokens."""
+        if T == self._T:
+            return
+        dev, K, d = self.device, self.top_k, self.d
+        rows = T * K
+        i32 = torch.int32
+        self.topk_idx = torch.empty((T, K), dtype=i32, device=dev)
+        self.topk_gate = torch.empty((T, K), dtype=torch.float32, device=dev)
+        self.counts = torch.empty(self.n_routed, dtype=i32, device=dev)
+        self.offsets = torch.empty(self.n_routed + 1, dtype=i32, device=dev)
+        self.pos = torch.empty((T, K), dtype=i32, device=dev)
+        self.src = torch.empty(rows, dtype=i32, device=dev)
+        self.x_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
+        self.y_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
+        self.perm_ws_bytes = L.moe_permute_workspace_size(T, self.n_routed)
+        self.perm_ws = torch.empty(self.perm_ws_bytes, dtype=torch.uint8, device=dev)
+        ffn_ws = max(L.moe_grouped_ffn_workspace_size(rows, self.inter),
+                     L.moe_grouped_ffn_workspace_size(T, max(self.shared_inter, 128)))
+        self.ffn_ws_bytes = ffn_ws
+        self.ffn_ws = torch.empty(ffn_ws, dtype=torch.uint8, device=dev)
+        self.shared_out = (torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+                           if self.ws13 is not None else None)
+        self.shared_offsets = torch.tensor([0, T], dtype=i32, device=dev)
+        self.out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+        self._T = T
+
+    # ------------------------------------------------------------------ steps
+    def route(self, u):
+        T = u.shape[0]
+        L.moe_route(u, self.centroids, self.bias if self.gate_kind == "sigmoid" else None, T,
+                    self.d, self.n_routed, self.top_k, self.gate_kind, self.routed_scale,
+                    self.topk_idx, self.topk_gate, self.counts)
+
+    def permute(self, u):
+        T = u.shape[0]
+        L.moe_permute(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
+                      self.x_perm, self.offsets, self.pos, self.src, self.perm_ws,
+                      self.perm_ws_bytes)
+
+    def routed_ffn(self, T):
+        L.moe_grouped_ffn(self.x_perm, None, self.offsets, self.n_routed, T * self.top_k, self.d,
+                          self.inter, self.w13, None, self.w2, None, L.MOE_BF16, self.y_perm,
+                          self.ffn_ws, self.ffn_ws_bytes)
+
+    def shared_ffn(self, u):
+        if self.ws13 is None:
+            return
+        T = u.shape[0]
+        L.moe_grouped_ffn(u, None, self.shared_offsets, 1, T, self.d, self.shared_inter, self.ws13,
+                          None, self.ws2, None, L.MOE_BF16, self.shared_out, self.ffn_ws,
+                          self.ffn_ws_bytes)
+
+    def combine(self, u, residual: bool = True):
+        T = u.shape[0]
+        L.moe_combine(self.y_perm, self.pos, self.topk_gate, self.shared_out,
+                      u if residual else None, T, self.d, self.top_k, self.out)
+
+    def forward(self, u, residual: bool = True):
+        """h' for the bf16 batch u [T, d] (device). Returns self.out (reused)."""
+        assert u.dtype == torch.bfloat16 and u.is_contiguous() and u.device.type == "cuda"
+        T = u.shape[0]
+        self.allocate(T)
+        self.route(u)
+        if T > 0:
+            self.permute(u)
+            self.routed_ffn(T)
+            self.shared_ffn(u)
+            self.combine(u, residual)
+        return self.out
+
+    def update_bias(self, counts=None, T=None):
+        """End-of-step bias update from this batch's loads (or from counts
+        summed over data-parallel ranks with the global T)."""
+        c = self.counts if counts is None else counts
+        L.moe_bias_update(c, self.bias, self.n_routed, self._T if T is None else T, self.top_k,
+                          self.gamma)
+
+    def step(self, u):
+        out = self.forward(u)
+        if self.gate_kind == "sigmoid":
+            self.update_bias()
+        return out
+
+    # kernels launched by one step(): route (1 + a memset), permute (3),
+    # routed FFN (2), shared FFN (2), combine (1), bias update (1)
+    def launches_per_step(self) -> int:
+        n = 1 + 3 + 2 + 1
+        if self.ws13 is not None:
+            n += 2
+        if self.gate_kind == "sigmoid":
+            n += 1
+        return n

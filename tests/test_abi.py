@@ -1,0 +1,146 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any launch.
+
+Every call below fails validation before the library touches CUDA, so the
+fake (never dereferenced) pointers are safe on a machine with or without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_58_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+A = 0x10000      # fake 16-byte aligned address (never dereferenced)
+MIS = 0x10002    # fake misaligned address
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixture_experts_layer_58_b200 import build
+    build.build()
+    return L.load()
+
+
+def test_header_declares_the_five_calls():
+    names = declared_symbols()
+    for n in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_bias_update"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(L.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(raw, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_symbol():
+    assert set(declared_symbols()) <= set(L._SIGS)
+
+
+def test_version_and_strerror(lib):
+    assert L.moe_version() >= 100
+    for code in (0, -1, -2, -3, -4, -5):
+        assert L.moe_strerror(code) and L.moe_strerror(code) != "unknown status"
+    assert L.moe_strerror(-99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    assert L.moe_permute_workspace_size(16384, 256) == 128 * 256 * 4
+    assert L.moe_permute_workspace_size(200, 16) == 256          # 2 chunks * 16 * 4 = 128 -> 256
+    assert L.moe_grouped_ffn_workspace_size(131072, 2048) == 131072 * 2048 * 2
+    assert L.moe_grouped_ffn_workspace_size(0, 2048) == 256
+
+
+def rc_route(lib, **kw):
+    a = dict(u=A, c=A, b=None, T=64, d=256, n=16, k=4, kind=0, s=1.0, idx=A, gate=A, cnt=A)
+    a.update(kw)
+    return lib.moe_route(a["u"], a["c"], a["b"], a["T"], a["d"], a["n"], a["k"], a["kind"],
+                         a["s"], a["idx"], a["gate"], a["cnt"], None)
+
+
+def test_route_rejects_bad_arguments(lib):
+    assert rc_route(lib, T=-1) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, d=0) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, k=0) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, kind=7) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, u=None) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, u=MIS) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, c=MIS) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, cnt=None) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, idx=None) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, s=float("nan")) == L.MOE_ERR_INVALID_ARG
+    assert rc_route(lib, k=9, n=16) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_route(lib, k=8, n=4) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_route(lib, n=300) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_route(lib, d=200) == L.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+def rc_permute(lib, **kw):
+    a = dict(u=A, idx=A, cnt=A, T=64, d=256, n=16, k=4, x=A, off=A, pos=A, src=A, ws=A, wsb=4096)
+    a.update(kw)
+    return lib.moe_permute(a["u"], a["idx"], a["cnt"], a["T"], a["d"], a["n"], a["k"], a["x"],
+                           a["off"], a["pos"], a["src"], a["ws"], a["wsb"], None)
+
+
+def test_permute_rejects_bad_arguments(lib):
+    assert rc_permute(lib, T=-5) == L.MOE_ERR_INVALID_ARG
+    assert rc_permute(lib, off=None) == L.MOE_ERR_INVALID_ARG
+    assert rc_permute(lib, x=MIS) == L.MOE_ERR_INVALID_ARG
+    assert rc_permute(lib, pos=None) == L.MOE_ERR_INVALID_ARG
+    assert rc_permute(lib, k=9) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_permute(lib, ws=None) == L.MOE_ERR_WORKSPACE
+    assert rc_permute(lib, wsb=16) == L.MOE_ERR_WORKSPACE
+    assert rc_permute(lib, ws=MIS) == L.MOE_ERR_WORKSPACE
+
+
+def rc_ffn(lib, **kw):
+    a = dict(x=A, off=A, G=16, rows=256, d=256, inter=128, w13=A, w2=A, dt=0, y=A, ws=A,
+             wsb=1 << 20)
+    a.update(kw)
+    return lib.moe_grouped_ffn(a["x"], None, a["off"], a["G"], a["rows"], a["d"], a["inter"],
+                               a["w13"], None, a["w2"], None, a["dt"], a["y"], a["ws"], a["wsb"],
+                               None)
+
+
+def test_grouped_ffn_rejects_bad_arguments(lib):
+    assert rc_ffn(lib, G=0) == L.MOE_ERR_INVALID_ARG
+    assert rc_ffn(lib, rows=-1) == L.MOE_ERR_INVALID_ARG
+    assert rc_ffn(lib, dt=5) == L.MOE_ERR_INVALID_ARG
+    assert rc_ffn(lib, dt=L.MOE_FP8_E4M3) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_ffn(lib, inter=100) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_ffn(lib, d=384) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_ffn(lib, G=5000) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rc_ffn(lib, ws=None) == L.MOE_ERR_WORKSPACE
+    assert rc_ffn(lib, wsb=1024) == L.MOE_ERR_WORKSPACE
+    # the halves: misaligned / null operands
+    assert lib.moe_expert_up_swiglu(MIS, A, 16, 256, 256, 128, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_down(A, None, 16, 256, 128, 256, A, A, None) == L.MOE_ERR_INVALID_ARG
+
+
+def test_combine_bias_pack_reject_bad_arguments(lib):
+    assert lib.moe_combine(A, A, A, None, None, 4, 256, 9, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_combine(None, A, A, None, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(A, A, A, MIS, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(A, A, A, None, None, -1, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(None, A, 16, 64, 4, 0.001, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(A, A, 0, 64, 4, 0.001, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(A, A, 16, 64, 4, float("nan"), None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_pack_w13(A, A, 2, 100, 256, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_pack_w13(A, None, 2, 128, 256, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_get_device_status(None, 0) == L.MOE_ERR_INVALID_ARG
+
+
+def test_binding_raises_moe_error(lib):
+    with pytest.raises(L.MoEError) as ei:
+        L.moe_combine(A, A, A, None, None, 4, 256, 9, A, stream=0)
+    assert ei.value.status == L.MOE_ERR_UNSUPPORTED_SHAPE

@@ -1,0 +1,226 @@
+"""Parity of every C-ABI call with the fp64 oracle on the Tiny and Mid
+workloads and on edge cases (ragged, empty, degenerate). Needs a B200."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_58_b200 import _lib as L
+from mixture_experts_layer_58_b200 import synth
+from mixture_experts_layer_58_b200.layer import MoELayer
+from oracle import moe_oracle as om
+
+from gpu_support import Inputs, check_close, check_route, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built(cuda_ok):
+    from mixture_experts_layer_58_b200 import build
+    build.build()
+    L.load()
+
+
+def _run_forward(inp: Inputs, residual=True):
+    out = inp.layer.forward(inp.u_dev, residual=residual)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    return out
+
+
+def _full_check(inp: Inputs, residual=True):
+    cfg = inp.cfg
+    out = _run_forward(inp, residual)
+    lay = inp.layer
+    r = inp.oracle_route()
+    gidx = lay.topk_idx.cpu().numpy()
+    near = check_route(gidx, lay.topk_gate.cpu().numpy(), lay.counts.cpu().numpy(), r,
+                       cfg.routed_scale, inp.u, inp.e, cfg.gate_kind)
+    # output on the GPU's own selection (gates recomputed by the oracle in fp64)
+    g = om.gates_for_indices(inp.u, inp.e, gidx, cfg.routed_scale, cfg.gate_kind)
+    ref = om.layer_output(inp.u, gidx, g, inp.expert, inp.shared_list(), residual=residual)
+    mx, mean = check_close(f64(out), ref)
+    return near, mx, mean
+
+
+def test_tiny_layer_forward_matches_oracle():
+    inp = Inputs(synth.CONFIGS["tiny"])
+    _full_check(inp)
+
+
+def test_tiny_every_call_matches_oracle():
+    cfg = synth.CONFIGS["tiny"]
+    inp = Inputs(cfg)
+    lay = inp.layer
+    _run_forward(inp)
+    T, K, d = cfg.T, cfg.top_k, cfg.d
+    gidx = lay.topk_idx.cpu().numpy()
+    # permute: bit-exact against the oracle's dispatch order of the same indices
+    disp = om.dispatch(gidx, cfg.n_routed)
+    assert np.array_equal(lay.offsets.cpu().numpy(), disp.offsets)
+    assert np.array_equal(lay.pos.cpu().numpy(), disp.pos)
+    assert np.array_equal(lay.src.cpu().numpy(), disp.src)
+    xp = lay.x_perm.cpu()
+    assert torch.equal(xp, inp.u[torch.from_numpy(disp.src)])
+    # routed FFN: each expert's rows against the fp64 FFN of the same rows
+    y = f64(lay.y_perm)
+    ref = np.zeros_like(y)
+    for i in range(cfg.n_routed):
+        a, b = disp.offsets[i], disp.offsets[i + 1]
+        if b > a:
+            ref[a:b] = om.ffn(xp[a:b].float().numpy(), *inp.expert(i))
+    check_close(y, ref, what="routed FFN")
+    # shared FFN
+    sh = om.shared_output(inp.u, inp.shared_list())
+    check_close(f64(lay.shared_out), sh, what="shared FFN")
+    # combine: fp64 sum of the GPU's own operands -> only the bf16 rounding differs
+    g = lay.topk_gate.cpu().numpy().astype(np.float64)
+    want = f64(inp.u) + f64(lay.shared_out)
+    for k in range(K):
+        want += g[:, k:k + 1] * y[disp.pos[:, k]]
+    got = f64(lay.out)
+    assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -8 + 1e-6)
+
+
+def test_tiny_bias_update_bit_exact():
+    cfg = synth.CONFIGS["tiny"]
+    inp = Inputs(cfg)
+    lay = inp.layer
+    b0 = lay.bias.cpu().numpy().copy()
+    lay.step(inp.u_dev)
+    torch.cuda.synchronize()
+    want = om.bias_update(lay.counts.cpu().numpy(), b0, cfg.T, cfg.top_k, cfg.gamma)
+    assert np.array_equal(lay.bias.cpu().numpy(), want)
+
+
+def test_mid_layer_forward_matches_oracle():
+    inp = Inputs(synth.CONFIGS["mid"])
+    near, mx, mean = _full_check(inp)
+    assert near < 0.05 * inp.T
+
+
+def test_mid_sixteen_bias_steps():
+    """16 route -> update steps on the same batch (b starts at 0). Each step's
+    routing is checked against the oracle under the GPU's current bias, and
+    each update is bit-exact against the oracle's update of the GPU's counts."""
+    cfg = synth.CONFIGS["mid"]
+    inp = Inputs(cfg)
+    lay = inp.layer
+    lay.allocate(cfg.T)
+    first_max = None
+    for step in range(cfg.bias_steps):
+        b_before = lay.bias.cpu().numpy().copy()
+        lay.route(inp.u_dev)
+        lay.update_bias()
+        torch.cuda.synchronize()
+        counts = lay.counts.cpu().numpy()
+        r = inp.oracle_route(bias=torch.from_numpy(b_before))
+        check_route(lay.topk_idx.cpu().numpy(), lay.topk_gate.cpu().numpy(), counts, r,
+                    cfg.routed_scale, inp.u, inp.e, cfg.gate_kind)
+        want = om.bias_update(counts, b_before, cfg.T, cfg.top_k, cfg.gamma)
+        assert np.array_equal(lay.bias.cpu().numpy(), want), f"step {step}"
+        if first_max is None:
+            first_max = counts.max()
+    assert L.moe_get_device_status() == 0
+
+
+@pytest.mark.parametrize("T", [1, 127, 129, 200, 383])
+def test_ragged_token_counts(T):
+    inp = Inputs(synth.CONFIGS["tiny"].replace(T=512), T=T)
+    _full_check(inp)
+
+
+def test_softmax_gate_variant():
+    inp = Inputs(synth.CONFIGS["tiny"].replace(gate_kind="softmax", bias_lo=0.0, bias_hi=0.0))
+    _full_check(inp)
+
+
+def test_no_residual_listing_form():
+    inp = Inputs(synth.CONFIGS["tiny"])
+    _full_check(inp, residual=False)
+
+
+def test_experts_not_multiple_of_16_and_empty_experts():
+    # 20 experts (padded to 32 MMA columns), top-2: several experts get no token
+    cfg = synth.CONFIGS["tiny"].replace(n_routed=20, top_k=2, T=48)
+    inp = Inputs(cfg)
+    _full_check(inp)
+
+
+def test_all_tokens_on_one_expert():
+    cfg = synth.CONFIGS["tiny"].replace(T=300)
+    inp = Inputs(cfg)
+    inp.layer.bias[7] = 5.0
+    b = inp.b.clone()
+    b[7] = 5.0
+    inp.b = b
+    near, _, _ = _full_check(inp)
+    assert int(inp.layer.counts[7]) == cfg.T
+
+
+def test_dense_reduction_one_expert_top1():
+    # N_r = 1, K = 1, S = 1, no shared expert: h' = u + FFN(u)
+    cfg = synth.CONFIGS["tiny"].replace(n_routed=1, top_k=1, n_shared=0, T=130)
+    inp = Inputs(cfg)
+    out = _run_forward(inp)
+    w1, w3, w2 = inp.expert(0)
+    ref = f64(inp.u) + om.ffn(inp.u.float().numpy(), w1, w3, w2)
+    check_close(f64(out), ref)
+    assert np.all(inp.layer.topk_gate.cpu().numpy() == 1.0)
+
+
+def test_all_experts_selected():
+    # K = N_r = 8: selection covers every expert whatever the bias
+    cfg = synth.CONFIGS["tiny"].replace(n_routed=8, top_k=8)
+    inp = Inputs(cfg)
+    _full_check(inp)
+    assert np.all(inp.layer.counts.cpu().numpy() == cfg.T)
+
+
+def test_empty_batch():
+    cfg = synth.CONFIGS["tiny"]
+    inp = Inputs(cfg, T=64)
+    lay = inp.layer
+    u0 = torch.empty((0, cfg.d), dtype=torch.bfloat16, device="cuda")
+    lay.allocate(0)
+    lay.counts.fill_(7)
+    out = lay.forward(u0)
+    lay.update_bias()
+    torch.cuda.synchronize()
+    assert out.shape == (0, cfg.d)
+    assert int(lay.counts.abs().sum()) == 0
+    assert np.array_equal(lay.bias.cpu().numpy(), inp.b.numpy())   # mean 0, loads 0: no change
+
+
+def test_run_to_run_bit_identical():
+    inp = Inputs(synth.CONFIGS["mid"])
+    a = _run_forward(inp).clone()
+    b = _run_forward(inp).clone()
+    assert torch.equal(a, b)
+
+
+def test_grouped_ffn_single_group_vs_torch_matmul():
+    """moe_grouped_ffn with G = 1 against fp32 torch matmuls of the same bf16
+    operands (h rounded to bf16 between the two GEMMs as the kernel does)."""
+    g = torch.Generator(device="cuda").manual_seed(11)
+    rows, d, inter = 333, 512, 384
+    x = torch.randn(rows, d, generator=g, device="cuda").bfloat16()
+    w1 = (0.05 * torch.randn(inter, d, generator=g, device="cuda")).bfloat16()
+    w3 = (0.05 * torch.randn(inter, d, generator=g, device="cuda")).bfloat16()
+    w2 = (0.05 * torch.randn(d, inter, generator=g, device="cuda")).bfloat16()
+    w13 = torch.empty(1, 2 * inter, d, dtype=torch.bfloat16, device="cuda")
+    L.moe_pack_w13(w1[None].contiguous(), w3[None].contiguous(), 1, inter, d, w13)
+    off = torch.tensor([0, rows], dtype=torch.int32, device="cuda")
+    y = torch.empty(rows, d, dtype=torch.bfloat16, device="cuda")
+    wsb = L.moe_grouped_ffn_workspace_size(rows, inter)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    L.moe_grouped_ffn(x, None, off, 1, rows, d, inter, w13, None, w2, None, L.MOE_BF16, y, ws, wsb)
+    torch.cuda.synchronize()
+    a = x.float() @ w1.float().T
+    b = x.float() @ w3.float().T
+    h = (torch.nn.functional.silu(a) * b).bfloat16()
+    ref = h.float() @ w2.float().T
+    check_close(y.float().cpu().numpy(), ref.cpu().numpy(), max_tol=1e-2, mean_tol=3e-3)
+    hk = ws[: rows * inter * 2].view(torch.bfloat16).view(rows, inter)
+    check_close(hk.float().cpu().numpy(), h.float().cpu().numpy(), max_tol=1e-2, mean_tol=3e-3,
+                what="h")
