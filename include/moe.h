@@ -122,6 +122,31 @@ MOE_API int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* e
 
 MOE_API size_t moe_permute_workspace_size(int T, int n_routed);
 
+/* moe_permute_noalloc: moe_permute without a workspace argument. The pages
+ * have no counterpart: this entry point exists for callers that cannot
+ * allocate device memory where they call the library — for example a plugin
+ * whose host framework owns the whole device-memory budget and hands it no
+ * allocator, or a latency-critical loop that must not call cudaMalloc (which
+ * can synchronise the device). It allocates nothing and calls no allocating
+ * routine; its scratch is a 256 KiB array in the library's own device memory,
+ * reserved on every GPU that loads the library until the process exits.
+ *
+ * Same arguments, outputs and errors as moe_permute. Limit: ceil(T/128) *
+ * n_routed <= 65536 (e.g. T <= 32768 with 256 experts); larger sizes return
+ * MOE_ERR_UNSUPPORTED_SHAPE before anything is enqueued.
+ * The first call on a device looks up the array's device address (one
+ * cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. Every call on a device shares the one array and
+ * leaves its contents behind (nothing in it needs clearing: each call
+ * overwrites every entry it reads), so calls that can overlap on the GPU —
+ * concurrent streams, or several host threads on one device — race on it and
+ * must be serialised by the caller.
+ */
+MOE_API int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
+                                const int32_t* expert_counts, int T, int d, int n_routed,
+                                int top_k, void* x_perm, int32_t* expert_offsets, int32_t* pos,
+                                int32_t* src_token, moe_stream_t stream);
+
 /* ------------------------------------------------------------------ expert FFN
  * Grouped SwiGLU expert FFN (FFN_i^(r) and FFN_i^(s) of the technical report's
  * output equation; the pages do not define the FFN's inside — SwiGLU without

@@ -47,6 +47,7 @@ _SIGS = {
     "moe_route": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp]),
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i]),
+    "moe_permute_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
     "moe_grouped_ffn": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp,
                              _sz, _vp]),
     "moe_grouped_ffn_workspace_size": (_sz, [_i, _i, _i]),
@@ -119,6 +120,16 @@ def moe_permute(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm, exper
     _check(_L().moe_permute(_p(u), _p(topk_idx), _p(expert_counts), T, d, n_routed, top_k,
                             _p(x_perm), _p(expert_offsets), _p(pos), _p(src_token),
                             _p(workspace), ws_bytes, _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm,
+                        expert_offsets, pos, src_token, stream=None):
+    """moe_permute for callers that cannot allocate device memory: no workspace
+    argument; the library's own 256 KiB device array serves as scratch (shared
+    by every call on the device, so calls must not overlap on the GPU)."""
+    _check(_L().moe_permute_noalloc(_p(u), _p(topk_idx), _p(expert_counts), T, d, n_routed,
+                                    top_k, _p(x_perm), _p(expert_offsets), _p(pos),
+                                    _p(src_token), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_permute_workspace_size(T, n_routed) -> int:

@@ -389,3 +389,77 @@ int moe_pack_w13(const void* w1, const void* w3, int G, int inter, int d, void* 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ permute, allocation-free
+// moe_permute without a workspace argument, for callers that cannot allocate
+// device memory at the call site. Its scratch (the per-chunk expert
+// histograms of the dispatch's first pass) lives in this file-scope device
+// array instead: every GPU that loads the library holds it until the process
+// exits, and every call shares it.
+namespace {
+
+constexpr int kNoAllocScratchInts = 65536;   // 256 KiB: ceil(T/128) * n_routed <= 65536
+__device__ __align__(256) int32_t g_permute_scratch[kNoAllocScratchInts];
+
+int32_t* g_scratch_ptr[kMaxDevices];          // device address of the array, per device
+std::mutex g_scratch_mu;
+
+// Device address of g_permute_scratch on the current device. In host code the
+// array's name is only a stand-in for the symbol, never a device address: the
+// address is looked up once per device with that device current.
+int scratch_address(int32_t** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_INVALID_ARG;
+  if (!g_scratch_ptr[dev]) {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+      void* p = nullptr;
+      MOE_CUDA(cudaGetSymbolAddress(&p, g_permute_scratch));
+      g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    }
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
+                                   const int32_t* expert_counts, int T, int d, int n_routed,
+                                   int top_k, void* x_perm, int32_t* expert_offsets,
+                                   int32_t* pos, int32_t* src_token, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 256 != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const long long chunks = (static_cast<long long>(T) + kPermChunk - 1) / kPermChunk;
+  if (chunks * n_routed > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T > 0 && (!u || !topk_idx || !x_perm || !pos || !src_token || !aligned16(u) ||
+                !aligned16(x_perm)))
+    return MOE_ERR_INVALID_ARG;
+  int32_t* hist = nullptr;
+  int rc = scratch_address(&hist);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t st = as_stream(stream);
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (n_routed + 1), st));
+    return MOE_OK;
+  }
+  DeviceInfo* di;
+  if ((rc = device_info(&di)) != MOE_OK) return rc;
+  // Pass 1 overwrites every histogram entry pass 2 reads, so the array needs
+  // no clearing between calls.
+  const int nch = static_cast<int>(chunks);
+  permute_hist_kernel<<<nch, 256, 0, st>>>(topk_idx, T, top_k, n_routed, hist);
+  MOE_CUDA(cudaGetLastError());
+  permute_index_kernel<<<nch, 256, 0, st>>>(topk_idx, expert_counts, hist, T, top_k, n_routed,
+                                            expert_offsets, pos, src_token);
+  MOE_CUDA(cudaGetLastError());
+  const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
+  permute_copy_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(u), pos, T, d,
+                                              top_k, static_cast<__nv_bfloat16*>(x_perm));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
