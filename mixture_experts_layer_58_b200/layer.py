@@ -114,23 +114,27 @@ class MoELayer:
                           None, self.ws2, None, L.MOE_BF16, self.shared_out, self.ffn_ws,
                           self.ffn_ws_bytes)
 
-    def combine(self, u, residual: bool = True):
+    def combine(self, u, residual: bool = True, out=None):
         T = u.shape[0]
         L.moe_combine(self.y_perm, self.pos, self.topk_gate, self.shared_out,
-                      u if residual else None, T, self.d, self.top_k, self.out)
+                      u if residual else None, T, self.d, self.top_k,
+                      self.out if out is None else out)
 
-    def forward(self, u, residual: bool = True):
-        """h' for the bf16 batch u [T, d] (device). Returns self.out (reused)."""
+    def forward(self, u, residual: bool = True, out=None):
+        """h' for the bf16 batch u [T, d] (device), written to `out` ([T, d]
+        bf16, device) or to the layer's own output buffer, which is returned."""
         assert u.dtype == torch.bfloat16 and u.is_contiguous() and u.device.type == "cuda"
         T = u.shape[0]
         self.allocate(T)
+        dst = self.out if out is None else out
+        assert dst.shape == (T, self.d) and dst.dtype == torch.bfloat16 and dst.is_contiguous()
         self.route(u)
         if T > 0:
             self.permute(u)
             self.routed_ffn(T)
             self.shared_ffn(u)
-            self.combine(u, residual)
-        return self.out
+            self.combine(u, residual, dst)
+        return dst
 
     def update_bias(self, counts=None, T=None):
         """End-of-step bias update from this batch's loads (or from counts

@@ -224,3 +224,37 @@ def test_grouped_ffn_single_group_vs_torch_matmul():
     hk = ws[: rows * inter * 2].view(torch.bfloat16).view(rows, inter)
     check_close(hk.float().cpu().numpy(), h.float().cpu().numpy(), max_tol=1e-2, mean_tol=3e-3,
                 what="h")
+
+
+def test_grouped_ffn_tile_paths_by_group_size():
+    """Group sizes that hit every tile path of the grouped GEMM: empty groups,
+    swapped tiles of 1..127 rows (N rounded up to 16), full 128-row tiles and
+    full + ragged combinations. Each group against fp32 torch matmuls of the
+    same bf16 operands, h rounded to bf16 as the kernel does."""
+    sizes = [1, 15, 0, 16, 17, 31, 32, 33, 100, 127, 128, 129, 255, 256, 0, 300]
+    G, d, inter = len(sizes), 256, 256
+    rows = sum(sizes)
+    g = torch.Generator(device="cuda").manual_seed(12)
+    x = torch.randn(rows, d, generator=g, device="cuda").bfloat16()
+    w1 = (0.05 * torch.randn(G, inter, d, generator=g, device="cuda")).bfloat16()
+    w3 = (0.05 * torch.randn(G, inter, d, generator=g, device="cuda")).bfloat16()
+    w2 = (0.05 * torch.randn(G, d, inter, generator=g, device="cuda")).bfloat16()
+    w13 = torch.empty(G, 2 * inter, d, dtype=torch.bfloat16, device="cuda")
+    L.moe_pack_w13(w1, w3, G, inter, d, w13)
+    off = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32, device="cuda")
+    y = torch.full((rows, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    wsb = L.moe_grouped_ffn_workspace_size(rows, inter)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    L.moe_grouped_ffn(x, None, off, G, rows, d, inter, w13, None, w2, None, L.MOE_BF16, y, ws, wsb)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    o = off.cpu().tolist()
+    for i in range(G):
+        a, b = o[i], o[i + 1]
+        if a == b:
+            continue
+        xa = x[a:b].float()
+        h = (torch.nn.functional.silu(xa @ w1[i].float().T) * (xa @ w3[i].float().T)).bfloat16()
+        ref = h.float() @ w2[i].float().T
+        check_close(y[a:b].float().cpu().numpy(), ref.cpu().numpy(), max_tol=1e-2,
+                    mean_tol=3e-3, what=f"group {i} ({b - a} rows)")
