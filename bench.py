@@ -248,7 +248,7 @@ def main():
     shared = synth.shared_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
     lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
                    routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
-                   device=dev)
+                   fp8=cfg.fp8, device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
     torch.cuda.empty_cache()
@@ -264,11 +264,22 @@ def main():
         lay.permute(u)
         if i is not None:
             up_ev[i][0].record(stream)
-        L.moe_expert_up_swiglu(lay.x_perm, lay.offsets, cfg.n_routed, T * K, d, I, lay.w13,
-                               lay.ffn_ws)
+        if cfg.fp8:
+            h8 = lay.ffn_ws
+            hs = lay.ffn_ws[(T * K * I + 255) // 256 * 256:]
+            L.moe_expert_up_swiglu_fp8(lay.x8, lay.x_s, lay.offsets, cfg.n_routed, T * K, d, I,
+                                       lay.w13, lay.w13_s, h8, hs)
+        else:
+            L.moe_expert_up_swiglu(lay.x_perm, lay.offsets, cfg.n_routed, T * K, d, I, lay.w13,
+                                   lay.ffn_ws)
         if i is not None:
             up_ev[i][1].record(stream)
-        L.moe_expert_down(lay.ffn_ws, lay.offsets, cfg.n_routed, T * K, I, d, lay.w2, lay.y_perm)
+        if cfg.fp8:
+            L.moe_expert_down_fp8(h8, hs, lay.offsets, cfg.n_routed, T * K, I, d, lay.w2,
+                                  lay.w2_s, lay.y_perm)
+        else:
+            L.moe_expert_down(lay.ffn_ws, lay.offsets, cfg.n_routed, T * K, I, d, lay.w2,
+                              lay.y_perm)
         lay.shared_ffn(u)
         lay.combine(u)
         if cfg.gate_kind == "sigmoid":
@@ -373,19 +384,23 @@ def main():
     pk = peaks()
     up_flops = 2.0 * T * K * d * 2 * I
     achieved = up_flops / (up_ms * 1e-3) / 1e12
-    peak = pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]
+    # an FP8 contraction takes the measured bf16 peak x the nominal fp8/bf16 ratio (2)
+    ratio = 2.0 if cfg.fp8 else 1.0
+    peak = (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * ratio
+    kname = ("grouped_gemm_fp8_kernel<SwiGLU+quant> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
+             "grouped_gemm_bf16_kernel<256,SwiGLU> (moe_expert_up_swiglu)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
-                "kernel": "grouped_gemm_bf16_kernel<256,SwiGLU> (moe_expert_up_swiglu)",
-                "kernel_ms": up_ms,
-                "peak_source": f"{pk['_source']} bf16_tflops_sustained"}
+                "kernel": kname, "kernel_ms": up_ms,
+                "peak_source": f"{pk['_source']} bf16_tflops_sustained"
+                               + (" x 2 (nominal fp8/bf16)" if cfg.fp8 else "")}
     layer_flops = T * cfg.flops_per_token()
     layer_tflops = layer_flops / (ms_step * 1e-3) / 1e12
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 promotion)" if cfg.fp8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the V3 layer shape)",
         "config": {"workload": cfg.name, "T": T, "d": d, "n_routed": cfg.n_routed, "top_k": K,
                    "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
@@ -396,6 +411,7 @@ def main():
                    "max_expert_load": int(counts.max()), "mean_expert_load": T * K / cfg.n_routed},
         "layer_tflops": layer_tflops,
         "layer_frac_of_bf16_peak": layer_tflops / pk["bf16_tflops"],
+        "layer_frac_of_tensor_peak": layer_tflops / (pk["bf16_tflops"] * ratio),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2, "api": "MoELayer.forward",

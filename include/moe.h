@@ -68,8 +68,7 @@ extern "C" {
  * logits, times the routed scale. */
 typedef enum { MOE_GATE_SIGMOID_BIAS = 0, MOE_GATE_SOFTMAX_TOPK = 1 } moe_gate_kind;
 
-/* Arithmetic type of the expert GEMM operands. MOE_FP8_E4M3 is reserved for
- * the FP8 variant and currently returns MOE_ERR_UNSUPPORTED_SHAPE. */
+/* Arithmetic type of the expert GEMM operands (see the FP8 section below). */
 typedef enum { MOE_BF16 = 0, MOE_FP8_E4M3 = 1 } moe_dtype;
 
 typedef void* moe_stream_t; /* cudaStream_t */
@@ -166,7 +165,12 @@ MOE_API int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
  *          h = silu(x W1^T) * (x W3^T) as bf16 [rows, inter].
  * The shared expert(s) run as G = 1 with group_offsets = {0, T}, x = u and
  * the N_s shared experts' weights concatenated along inter.
- * x_scales / w13_scales / w2_scales are for the FP8 variant; pass NULL.
+ * dtype MOE_BF16: x, w13, w2 bf16; x_scales / w13_scales / w2_scales unused
+ *   (pass NULL); workspace holds h as bf16 [rows, inter].
+ * dtype MOE_FP8_E4M3: x, w13, w2 are E4M3 codes (1 byte) with fp32 scales
+ *   x_scales [rows, d/128], w13_scales [G, 2*inter/128, d/128],
+ *   w2_scales [G, d/128, inter/128] (see the FP8 section); y stays bf16;
+ *   workspace holds h as E4M3 [rows, inter] + its scales [rows, inter/128].
  */
 MOE_API int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_offsets,
                             int G, int rows, int d, int inter, const void* w13,
@@ -185,6 +189,51 @@ MOE_API int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, in
                                  moe_stream_t stream);
 MOE_API int moe_expert_down(const void* h, const int32_t* group_offsets, int G, int rows,
                             int inter, int d, const void* w2, void* y, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ FP8 variant
+ * FP8 mixed precision of the technical report summary ("Main ideas", FP8
+ * bullet): E4M3 operands, tile-wise 1x128 activation scaling, block-wise
+ * 128x128 weight scaling, accumulation promoted to FP32 on the CUDA cores
+ * every 128 elements of K; the scale of a tile or block is max|x| / 448
+ * (block-quantisation pseudocode of "DeepSeek model architecture explained",
+ * 448 = largest E4M3 value). Codes are decided in fp32: scale = amax / 448
+ * (an all-zero tile gets 1) and x / scale are IEEE fp32 divisions, the
+ * quotient is rounded to E4M3 to nearest-even, saturating at +-448.
+ * E4M3 tensors are 1 byte per element, 16-B aligned; scales fp32, 4-B aligned.
+ * The routing (moe_route) stays bf16: the expert indices must be exact.
+ *
+ * moe_quant_act_fp8: x [rows, cols] bf16 -> q [rows, cols] E4M3 and
+ *   scales [rows, cols/128] (one per 1x128 tile). cols % 128 == 0.
+ * moe_quant_weights_fp8: w [G, R, C] bf16 -> q [G, R, C] E4M3 and
+ *   scales [G, R/128, C/128] (one per 128x128 block). R, C % 128 == 0.
+ *   For w13 quantise the packed (interleaved) [G, 2*inter, d] tensor: its
+ *   128-row chunks are whole W1 or W3 blocks.
+ * moe_permute_fp8: moe_permute for E4M3 rows: u8 [T, d] codes + u_scales
+ *   [T, d/128] (from moe_quant_act_fp8, quantised once per token) are copied
+ *   to x8 [T*top_k, d] + x_scales [T*top_k, d/128]; other arguments as
+ *   moe_permute.
+ * moe_expert_up_swiglu_fp8 / moe_expert_down_fp8: the two halves of
+ *   moe_grouped_ffn in FP8; the first writes h as E4M3 h8 [rows, inter] with
+ *   h_scales [rows, inter/128] (h = silu(a) * b is quantised per 1x128 tile
+ *   in the GEMM's epilogue), the second reads them and writes bf16 y.
+ */
+MOE_API int moe_quant_act_fp8(const void* x, int rows, int cols, void* q, float* scales,
+                              moe_stream_t stream);
+MOE_API int moe_quant_weights_fp8(const void* w, int G, int R, int C, void* q, float* scales,
+                                  moe_stream_t stream);
+MOE_API int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_idx,
+                            const int32_t* expert_counts, int T, int d, int n_routed, int top_k,
+                            void* x8, float* x_scales, int32_t* expert_offsets, int32_t* pos,
+                            int32_t* src_token, void* workspace, size_t ws_bytes,
+                            moe_stream_t stream);
+MOE_API int moe_expert_up_swiglu_fp8(const void* x8, const float* x_scales,
+                                     const int32_t* group_offsets, int G, int rows, int d,
+                                     int inter, const void* w13, const float* w13_scales, void* h8,
+                                     float* h_scales, moe_stream_t stream);
+MOE_API int moe_expert_down_fp8(const void* h8, const float* h_scales,
+                                const int32_t* group_offsets, int G, int rows, int inter, int d,
+                                const void* w2, const float* w2_scales, void* y,
+                                moe_stream_t stream);
 
 /* ------------------------------------------------------------------ combine
  * out_t = residual_t + shared_t + sum_k topk_gate[t,k] * y_perm[pos[t,k]]

@@ -53,6 +53,12 @@ _SIGS = {
     "moe_grouped_ffn_workspace_size": (_sz, [_i, _i, _i]),
     "moe_expert_up_swiglu": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "moe_expert_down": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_quant_act_fp8": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "moe_quant_weights_fp8": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_permute_fp8": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                             _sz, _vp]),
+    "moe_expert_up_swiglu_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "moe_expert_down_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_bias_update": (_i, [_vp, _vp, _i, _ll, _i, _f, _vp]),
     "moe_pack_w13": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
@@ -155,6 +161,38 @@ def moe_expert_up_swiglu(x, group_offsets, G, rows, d, inter, w13, h, stream=Non
 def moe_expert_down(h, group_offsets, G, rows, inter, d, w2, y, stream=None):
     _check(_L().moe_expert_down(_p(h), _p(group_offsets), G, rows, inter, d, _p(w2), _p(y),
                                 _stream(stream)), "moe_expert_down")
+
+
+def moe_quant_act_fp8(x, rows, cols, q, scales, stream=None):
+    _check(_L().moe_quant_act_fp8(_p(x), rows, cols, _p(q), _p(scales), _stream(stream)),
+           "moe_quant_act_fp8")
+
+
+def moe_quant_weights_fp8(w, G, R, C, q, scales, stream=None):
+    _check(_L().moe_quant_weights_fp8(_p(w), G, R, C, _p(q), _p(scales), _stream(stream)),
+           "moe_quant_weights_fp8")
+
+
+def moe_permute_fp8(u8, u_scales, topk_idx, expert_counts, T, d, n_routed, top_k, x8, x_scales,
+                    expert_offsets, pos, src_token, workspace, ws_bytes, stream=None):
+    _check(_L().moe_permute_fp8(_p(u8), _p(u_scales), _p(topk_idx), _p(expert_counts), T, d,
+                                n_routed, top_k, _p(x8), _p(x_scales), _p(expert_offsets), _p(pos),
+                                _p(src_token), _p(workspace), ws_bytes, _stream(stream)),
+           "moe_permute_fp8")
+
+
+def moe_expert_up_swiglu_fp8(x8, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales, h8,
+                             h_scales, stream=None):
+    _check(_L().moe_expert_up_swiglu_fp8(_p(x8), _p(x_scales), _p(group_offsets), G, rows, d,
+                                         inter, _p(w13), _p(w13_scales), _p(h8), _p(h_scales),
+                                         _stream(stream)), "moe_expert_up_swiglu_fp8")
+
+
+def moe_expert_down_fp8(h8, h_scales, group_offsets, G, rows, inter, d, w2, w2_scales, y,
+                        stream=None):
+    _check(_L().moe_expert_down_fp8(_p(h8), _p(h_scales), _p(group_offsets), G, rows, inter, d,
+                                    _p(w2), _p(w2_scales), _p(y), _stream(stream)),
+           "moe_expert_down_fp8")
 
 
 def moe_combine(y_perm, pos, topk_gate, shared_out, residual, T, d, top_k, out, stream=None):

@@ -1,0 +1,334 @@
+// Grouped FP8 (E4M3) GEMM with FP32 promotion every 128 K, on tcgen05.
+//
+// DeepSeek-V3 technical report summary (xyznot.com), "Main ideas", FP8 bullet:
+// E4M3 operands with 1x128 activation tiles and 128x128 weight blocks, and the
+// accumulation moved to FP32 on CUDA cores every N_c = 128 steps of K
+// ("Problem setting": FP8 tensor cores accumulate with limited precision).
+//
+// For every 128-wide K block kb the tensor cores form the block's product
+//   P_kb[m, n] = sum_{k in kb} qa[m, k] * qw[n, k]
+// from a fresh start (tcgen05.mma kind::f8f6f4, 4 x K=32) into one of two
+// 256-column TMEM buffers, and the epilogue warps fold it into fp32 registers:
+//   acc[m, n] += P_kb[m, n] * s_a[m, kb] * s_w[n / 128, kb].
+// The scales are the pages' arbitrary fp32 values (max|x| / 448), which the
+// hardware's block-scaled MMA (power-of-two, 32-element scale blocks) cannot
+// express; promotion on the CUDA cores keeps them exact.
+//
+// 10 warps, one persistent CTA per SM:
+//   warp 0      TMA producer: A [128 rows x 128 B] + B [256 rows x 128 B] per stage.
+//   warp 1      MMA issuer: one K block per P buffer, alternating buffers.
+//   warps 2-9   promotion + epilogue. Warp w reads TMEM lane quarter w % 4;
+//               half = (w - 2) / 4 picks its columns [64*half, +64) and
+//               [128 + 64*half, +64): the gate and up columns of the same 64 h
+//               columns when B is an interleaved W1/W3 tile. 128 fp32
+//               accumulators per thread.
+// Epilogues: EPI8_SWIGLU_Q — h = silu(a) * b, then h is quantised to E4M3 with
+// one 1x128 scale per row per tile (the two halves of a row trade their amax
+// through shared memory); EPI8_STORE — bf16 output.
+#pragma once
+#include "fp8.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+
+constexpr int kF8BK = 128;        // K elements (= bytes) per stage = one scale block
+constexpr int kF8UmmaK = 32;      // K of one tcgen05.mma kind::f8f6f4
+constexpr int kF8BN = 256;
+constexpr int kF8Threads = 320;
+constexpr int kF8EpiThreads = 256;
+
+enum { EPI8_STORE = 0, EPI8_SWIGLU_Q = 1 };
+
+struct GemmF8Cfg {
+  static constexpr int kABytes = kBM * kF8BK;
+  static constexpr int kBBytes = kF8BN * kF8BK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * kF8BN;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kXchgBytes = 2 * 2 * kBM * static_cast<int>(sizeof(float));
+  static size_t smem_bytes(int G) {
+    return 1024 + static_cast<size_t>(kStages) * kStageBytes + kBarBytes + kXchgBytes +
+           2 * static_cast<size_t>(G + 1) * sizeof(int);
+  }
+};
+
+// Instruction descriptor of tcgen05.mma kind::f8f6f4: E4M3 A and B (format
+// code 0, K-major), fp32 accumulator, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kF8Threads, 1)
+grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const float* __restrict__ a_scales, const float* __restrict__ b_scales,
+                        const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
+                        int rows, void* __restrict__ out, int ldo, float* __restrict__ out_scales,
+                        unsigned int* status) {
+  using C = GemmF8Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * C::kBBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* pfull = empty + kStages;
+  uint64_t* pempty = pfull + 2;
+  uint64_t* mma_done = pempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  float* xchg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
+  int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(xchg) + C::kXchgBytes);
+  int* s_tstart = s_off + (G + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_blocks_n = n_per_group / kF8BN;
+  const int num_kb = K / kF8BK;
+  const int nsb = n_per_group / kQBlock;   // weight scale blocks along N, per group
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(&full[s], 1);
+        mbar_init(&empty[s], 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&pfull[b], 1);
+        mbar_init(&pempty[b], kF8EpiThreads);
+      }
+      mbar_init(mma_done, 1);
+      fence_mbar_init();
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+    }
+    __syncwarp();
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  } else if (warp == 1) {
+    int carry = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int nt = 0;
+      if (g < G) {
+        const int o0 = offsets[g];
+        const int o1 = offsets[g + 1];
+        s_off[g] = o0;
+        nt = (o1 > o0 ? (o1 - o0 + kBM - 1) / kBM : 0) * n_blocks_n;
+      }
+      int v = nt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+      }
+      if (g < G) s_tstart[g] = carry + v - nt;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) {
+      s_tstart[G] = carry;
+      s_off[G] = offsets[G];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = s_tstart[G];
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, issued_par = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      int g, m_blk, n_blk;
+      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      const int a_row = s_off[g] + m_blk * kBM;
+      const int b_row = g * n_per_group + n_blk * kF8BN;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, status, kStatusTimeoutProducer)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+        tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * kF8BK, a_row);
+        tma_load_2d(sB + stage * C::kBBytes, &tmB, &full[stage], kb * kF8BK, b_row);
+        issued |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    for (int s = 0; s < kStages; ++s)
+      if (issued & (1u << s))
+        mbar_wait(&full[s], (issued_par >> s) & 1u, status, kStatusTimeoutProducer);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_e4m3_f32(kBM, kF8BN);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t kcount = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int kb = 0; kb < num_kb; ++kb, ++kcount) {
+        const uint32_t pb = kcount & 1u;
+        const uint32_t ppar = (kcount >> 1) & 1u;
+        if (!mbar_wait(&pempty[pb], ppar ^ 1u, status, kStatusTimeoutMma) ||
+            !mbar_wait(&full[stage], phase, status, kStatusTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * C::kABytes));
+        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * C::kBBytes));
+        const uint32_t d_tmem = tmem_base + pb * kF8BN;
+#pragma unroll
+        for (int k = 0; k < kF8BK / kF8UmmaK; ++k)   // 32 bytes of K per MMA
+          umma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, k != 0);
+        umma_commit(&empty[stage]);
+        umma_commit(&pfull[pb]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    umma_commit(mma_done);
+    mbar_wait(mma_done, 0, status, kStatusTimeoutMma);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ promotion + epilogue
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const int col0 = half * 64;            // gate (or first-half) columns
+    const int col1 = 128 + half * 64;      // up (or second-half) columns
+    uint32_t kcount = 0;
+    bool broken = false;
+    int local = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+      int g, m_blk, n_blk;
+      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      const int row0 = s_off[g] + m_blk * kBM;
+      const int row_end = min(s_off[g + 1], rows);
+      const int grow = row0 + row_in_tile;
+      const bool valid = grow >= 0 && grow < row_end;
+      const float* sa_row = a_scales + static_cast<size_t>(valid ? grow : 0) * num_kb;
+      const float* sw0 = b_scales + (static_cast<size_t>(g) * nsb + 2 * n_blk) * num_kb;
+      const float* sw1 = sw0 + num_kb;
+      float acc0[64], acc1[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        acc0[j] = 0.0f;
+        acc1[j] = 0.0f;
+      }
+      float sa_n = valid ? __ldg(sa_row) : 0.0f;
+      float w0_n = __ldg(sw0), w1_n = __ldg(sw1);
+      for (int kb = 0; kb < num_kb; ++kb, ++kcount) {
+        const float s0 = sa_n * w0_n;
+        const float s1 = sa_n * w1_n;
+        if (kb + 1 < num_kb) {
+          sa_n = valid ? __ldg(sa_row + kb + 1) : 0.0f;
+          w0_n = __ldg(sw0 + kb + 1);
+          w1_n = __ldg(sw1 + kb + 1);
+        }
+        const uint32_t pb = kcount & 1u;
+        const uint32_t ppar = (kcount >> 1) & 1u;
+        if (!broken && !mbar_wait(&pfull[pb], ppar, status, kStatusTimeoutEpilogue)) broken = true;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + pb * kF8BN + lane_addr;
+        uint32_t r[32];
+        tmem_ld_32cols(taddr + col0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc0[i] = fmaf(__uint_as_float(r[i]), s0, acc0[i]);
+        tmem_ld_32cols(taddr + col0 + 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc0[32 + i] = fmaf(__uint_as_float(r[i]), s0, acc0[32 + i]);
+        tmem_ld_32cols(taddr + col1, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc1[i] = fmaf(__uint_as_float(r[i]), s1, acc1[i]);
+        tmem_ld_32cols(taddr + col1 + 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc1[32 + i] = fmaf(__uint_as_float(r[i]), s1, acc1[32 + i]);
+        tc_fence_before();
+        mbar_arrive(&pempty[pb]);
+      }
+      if constexpr (EPI == EPI8_SWIGLU_Q) {
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          acc0[j] = silu_f32(acc0[j]) * acc1[j];
+          amax = fmaxf(amax, fabsf(acc0[j]));
+        }
+        float* xc = xchg + (local & 1) * (2 * kBM);
+        xc[half * kBM + row_in_tile] = amax;
+        named_bar_sync(1, kF8EpiThreads);
+        amax = fmaxf(amax, xc[(1 - half) * kBM + row_in_tile]);
+        const float s = fp8_scale_of(amax);
+        if (valid) {
+          uint8_t* dst = static_cast<uint8_t*>(out) + static_cast<size_t>(grow) * ldo +
+                         n_blk * 128 + half * 64;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 o;
+            o.x = to_e4m3x4(__fdiv_rn(acc0[16 * v + 0], s), __fdiv_rn(acc0[16 * v + 1], s),
+                            __fdiv_rn(acc0[16 * v + 2], s), __fdiv_rn(acc0[16 * v + 3], s));
+            o.y = to_e4m3x4(__fdiv_rn(acc0[16 * v + 4], s), __fdiv_rn(acc0[16 * v + 5], s),
+                            __fdiv_rn(acc0[16 * v + 6], s), __fdiv_rn(acc0[16 * v + 7], s));
+            o.z = to_e4m3x4(__fdiv_rn(acc0[16 * v + 8], s), __fdiv_rn(acc0[16 * v + 9], s),
+                            __fdiv_rn(acc0[16 * v + 10], s), __fdiv_rn(acc0[16 * v + 11], s));
+            o.w = to_e4m3x4(__fdiv_rn(acc0[16 * v + 12], s), __fdiv_rn(acc0[16 * v + 13], s),
+                            __fdiv_rn(acc0[16 * v + 14], s), __fdiv_rn(acc0[16 * v + 15], s));
+            reinterpret_cast<uint4*>(dst)[v] = o;
+          }
+          if (half == 0) out_scales[static_cast<size_t>(grow) * (ldo / kQBlock) + n_blk] = s;
+        }
+      } else {
+        if (valid) {
+          __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(out) + static_cast<size_t>(grow) * ldo +
+                                n_blk * kF8BN;
+          uint4* d0 = reinterpret_cast<uint4*>(yrow + col0);
+          uint4* d1 = reinterpret_cast<uint4*>(yrow + col1);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            d0[v] = make_uint4(pack_bf16x2(acc0[8 * v], acc0[8 * v + 1]),
+                               pack_bf16x2(acc0[8 * v + 2], acc0[8 * v + 3]),
+                               pack_bf16x2(acc0[8 * v + 4], acc0[8 * v + 5]),
+                               pack_bf16x2(acc0[8 * v + 6], acc0[8 * v + 7]));
+            d1[v] = make_uint4(pack_bf16x2(acc1[8 * v], acc1[8 * v + 1]),
+                               pack_bf16x2(acc1[8 * v + 2], acc1[8 * v + 3]),
+                               pack_bf16x2(acc1[8 * v + 4], acc1[8 * v + 5]),
+                               pack_bf16x2(acc1[8 * v + 6], acc1[8 * v + 7]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -13,7 +13,9 @@
 
 #include "moe.h"
 #include "dispatch.cuh"
+#include "fp8.cuh"
 #include "gemm.cuh"
+#include "gemm_fp8.cuh"
 #include "route.cuh"
 
 namespace {
@@ -138,6 +140,53 @@ int launch_grouped_gemm(const void* A, int rows, int K, const void* B, int G, in
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
+
+// 2-D E4M3 (byte) tensor map over a row-major [rows, cols] matrix, box
+// [box_rows, 128 columns], 128-byte swizzle, zero fill out of bounds.
+int make_tmap_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                 uint32_t box_rows) {
+  int rc = get_encoder();
+  if (rc != MOE_OK) return rc;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kF8BK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+template <int EPI>
+int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int K, const void* B,
+                            const float* b_scales, int G, int n_per_group,
+                            const int32_t* offsets, void* out, int ldo, float* out_scales,
+                            cudaStream_t st) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  CUtensorMap tmA, tmB;
+  if ((rc = make_tmap_u8(&tmA, A, K, rows, kBM)) != MOE_OK) return rc;
+  if ((rc = make_tmap_u8(&tmB, B, K, static_cast<uint64_t>(G) * n_per_group, kF8BN)) != MOE_OK)
+    return rc;
+  const size_t smem = GemmF8Cfg::smem_bytes(G);
+  auto kern = grouped_gemm_fp8_kernel<EPI>;
+  if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
+  const long long max_tiles =
+      (static_cast<long long>(rows) / kBM + G) * static_cast<long long>(n_per_group / kF8BN);
+  const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
+  kern<<<grid, kF8Threads, smem, st>>>(tmA, tmB, a_scales, b_scales, offsets, G, K, n_per_group,
+                                       rows, out, ldo, out_scales, di->status);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 int check_ffn_shape(int G, int rows, int d, int inter) {
   if (G < 1 || rows < 0 || d <= 0 || inter <= 0) return MOE_ERR_INVALID_ARG;
@@ -290,8 +339,12 @@ int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* expert_co
 
 // ------------------------------------------------------------------ expert FFN
 size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dtype) {
-  (void)dtype;
   if (rows <= 0 || inter <= 0) return 256;
+  if (dtype == MOE_FP8_E4M3) {
+    const size_t codes = (static_cast<size_t>(rows) * inter + 255) / 256 * 256;
+    const size_t scales = (static_cast<size_t>(rows) * (inter / 128) * 4 + 255) / 256 * 256;
+    return codes + scales;
+  }
   return (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
 }
 
@@ -322,19 +375,119 @@ int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_o
                     const void* w2, const float* w2_scales, moe_dtype dtype, void* y,
                     void* workspace, size_t ws_bytes, moe_stream_t stream) {
   if (dtype != MOE_BF16 && dtype != MOE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
-  if (dtype == MOE_FP8_E4M3) return MOE_ERR_UNSUPPORTED_SHAPE;
-  (void)x_scales;
-  (void)w13_scales;
-  (void)w2_scales;
   int rc = check_ffn_shape(G, rows, d, inter);
   if (rc != MOE_OK) return rc;
   if (rows == 0) return MOE_OK;
   if (!workspace || ws_bytes < moe_grouped_ffn_workspace_size(rows, inter, dtype) ||
       !aligned16(workspace))
     return MOE_ERR_WORKSPACE;
+  if (dtype == MOE_FP8_E4M3) {
+    uint8_t* h8 = static_cast<uint8_t*>(workspace);
+    float* hs = reinterpret_cast<float*>(h8 + (static_cast<size_t>(rows) * inter + 255) / 256 * 256);
+    rc = moe_expert_up_swiglu_fp8(x, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales,
+                                  h8, hs, stream);
+    if (rc != MOE_OK) return rc;
+    return moe_expert_down_fp8(h8, hs, group_offsets, G, rows, inter, d, w2, w2_scales, y, stream);
+  }
   rc = moe_expert_up_swiglu(x, group_offsets, G, rows, d, inter, w13, workspace, stream);
   if (rc != MOE_OK) return rc;
   return moe_expert_down(workspace, group_offsets, G, rows, inter, d, w2, y, stream);
+}
+
+// ------------------------------------------------------------------ FP8 variant
+int moe_quant_act_fp8(const void* x, int rows, int cols, void* q, float* scales,
+                      moe_stream_t stream) {
+  if (rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  if (cols % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || !aligned4(scales))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int blocks = std::max(1, std::min((rows + 7) / 8, di->num_sms * 8));
+  quant_act_fp8_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, cols, static_cast<uint8_t*>(q), scales);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_quant_weights_fp8(const void* w, int G, int R, int C, void* q, float* scales,
+                          moe_stream_t stream) {
+  if (G <= 0 || R <= 0 || C <= 0) return MOE_ERR_INVALID_ARG;
+  if (R % 128 != 0 || C % 128 != 0 || G > 65535 || R / 128 > 65535)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!w || !q || !scales || !aligned16(w) || !aligned16(q) || !aligned4(scales))
+    return MOE_ERR_INVALID_ARG;
+  quant_weight_fp8_kernel<<<dim3(C / 128, R / 128, G), 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(w), R, C, static_cast<uint8_t*>(q), scales);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_idx,
+                    const int32_t* expert_counts, int T, int d, int n_routed, int top_k, void* x8,
+                    float* x_scales, int32_t* expert_offsets, int32_t* pos, int32_t* src_token,
+                    void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 256 != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = as_stream(stream);
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (n_routed + 1), st));
+    return MOE_OK;
+  }
+  if (!u8 || !u_scales || !topk_idx || !x8 || !x_scales || !pos || !src_token ||
+      !aligned16(u8) || !aligned16(x8) || !aligned4(u_scales) || !aligned4(x_scales))
+    return MOE_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < moe_permute_workspace_size(T, n_routed) || !aligned16(workspace))
+    return MOE_ERR_WORKSPACE;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int chunks = (T + kPermChunk - 1) / kPermChunk;
+  int32_t* hist = static_cast<int32_t*>(workspace);
+  permute_hist_kernel<<<chunks, 256, 0, st>>>(topk_idx, T, top_k, n_routed, hist);
+  MOE_CUDA(cudaGetLastError());
+  permute_index_kernel<<<chunks, 256, 0, st>>>(topk_idx, expert_counts, hist, T, top_k, n_routed,
+                                               expert_offsets, pos, src_token);
+  MOE_CUDA(cudaGetLastError());
+  const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
+  permute_copy_fp8_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint8_t*>(u8), u_scales, pos,
+                                                  T, d, top_k, static_cast<uint8_t*>(x8), x_scales);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_expert_up_swiglu_fp8(const void* x8, const float* x_scales, const int32_t* group_offsets,
+                             int G, int rows, int d, int inter, const void* w13,
+                             const float* w13_scales, void* h8, float* h_scales,
+                             moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!x8 || !x_scales || !group_offsets || !w13 || !w13_scales || !h8 || !h_scales ||
+      !aligned16(x8) || !aligned16(w13) || !aligned16(h8) || !aligned4(x_scales) ||
+      !aligned4(w13_scales) || !aligned4(h_scales))
+    return MOE_ERR_INVALID_ARG;
+  return launch_grouped_gemm_fp8<EPI8_SWIGLU_Q>(x8, x_scales, rows, d, w13, w13_scales, G,
+                                                2 * inter, group_offsets, h8, inter, h_scales,
+                                                as_stream(stream));
+}
+
+int moe_expert_down_fp8(const void* h8, const float* h_scales, const int32_t* group_offsets, int G,
+                        int rows, int inter, int d, const void* w2, const float* w2_scales, void* y,
+                        moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!h8 || !h_scales || !group_offsets || !w2 || !w2_scales || !y || !aligned16(h8) ||
+      !aligned16(w2) || !aligned16(y) || !aligned4(h_scales) || !aligned4(w2_scales))
+    return MOE_ERR_INVALID_ARG;
+  return launch_grouped_gemm_fp8<EPI8_STORE>(h8, h_scales, rows, inter, w2, w2_scales, G, d,
+                                             group_offsets, y, d, nullptr, as_stream(stream));
 }
 
 // ------------------------------------------------------------------ combine

@@ -27,7 +27,7 @@ class MoELayer:
 
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
-                 device="cuda"):
+                 fp8: bool = False, device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -52,6 +52,15 @@ class MoELayer:
         else:
             self.shared_inter = 0
             self.ws13 = self.ws2 = None
+        self.fp8 = bool(fp8)
+        if self.fp8:
+            # E4M3 weights with one fp32 scale per 128x128 block (the bf16
+            # copies are dropped)
+            self.w13, self.w13_s = self.quant_weights(self.w13)
+            self.w2, self.w2_s = self.quant_weights(self.w2)
+            if self.ws13 is not None:
+                self.ws13, self.ws13_s = self.quant_weights(self.ws13)
+                self.ws2, self.ws2_s = self.quant_weights(self.ws2[None])
         self._T = -1
 
     # ------------------------------------------------------------------ setup
@@ -60,6 +69,16 @@ class MoELayer:
         w13 = torch.empty((G, 2 * inter, d), dtype=torch.bfloat16, device=self.device)
         L.moe_pack_w13(w1, w3, G, inter, d, w13)
         return w13
+
+    def quant_weights(self, w):
+        """E4M3 codes [G, R, C] and fp32 scales [G, R/128, C/128] of bf16 w."""
+        if w.dim() == 2:
+            w = w[None]
+        G, R, C = w.shape
+        q = torch.empty((G, R, C), dtype=torch.uint8, device=self.device)
+        s = torch.empty((G, R // 128, C // 128), dtype=torch.float32, device=self.device)
+        L.moe_quant_weights_fp8(w.contiguous(), G, R, C, q, s)
+        return q, s
 
     def allocate(self, T: int) -> None:
         """(Re)allocate the activation buffers for a batch of T tokens."""
@@ -74,12 +93,20 @@ class MoELayer:
         self.offsets = torch.empty(self.n_routed + 1, dtype=i32, device=dev)
         self.pos = torch.empty((T, K), dtype=i32, device=dev)
         self.src = torch.empty(rows, dtype=i32, device=dev)
-        self.x_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
+        self.x_perm = (None if self.fp8 else
+                       torch.empty((rows, d), dtype=torch.bfloat16, device=dev))
         self.y_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
         self.perm_ws_bytes = L.moe_permute_workspace_size(T, self.n_routed)
         self.perm_ws = torch.empty(self.perm_ws_bytes, dtype=torch.uint8, device=dev)
-        ffn_ws = max(L.moe_grouped_ffn_workspace_size(rows, self.inter),
-                     L.moe_grouped_ffn_workspace_size(T, max(self.shared_inter, 128)))
+        dt = L.MOE_FP8_E4M3 if self.fp8 else L.MOE_BF16
+        ffn_ws = max(L.moe_grouped_ffn_workspace_size(rows, self.inter, dt),
+                     L.moe_grouped_ffn_workspace_size(T, max(self.shared_inter, 128), dt))
+        if self.fp8:
+            u8 = torch.uint8
+            self.u8 = torch.empty((T, d), dtype=u8, device=dev)
+            self.u_s = torch.empty((T, d // 128), dtype=torch.float32, device=dev)
+            self.x8 = torch.empty((rows, d), dtype=u8, device=dev)
+            self.x_s = torch.empty((rows, d // 128), dtype=torch.float32, device=dev)
         self.ffn_ws_bytes = ffn_ws
         self.ffn_ws = torch.empty(ffn_ws, dtype=torch.uint8, device=dev)
         self.shared_out = (torch.empty((T, d), dtype=torch.bfloat16, device=dev)
@@ -97,11 +124,23 @@ class MoELayer:
 
     def permute(self, u):
         T = u.shape[0]
+        if self.fp8:
+            # quantise each token once (1x128 tiles), then copy its codes K times
+            L.moe_quant_act_fp8(u, T, self.d, self.u8, self.u_s)
+            L.moe_permute_fp8(self.u8, self.u_s, self.topk_idx, self.counts, T, self.d,
+                              self.n_routed, self.top_k, self.x8, self.x_s, self.offsets,
+                              self.pos, self.src, self.perm_ws, self.perm_ws_bytes)
+            return
         L.moe_permute(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
                       self.x_perm, self.offsets, self.pos, self.src, self.perm_ws,
                       self.perm_ws_bytes)
 
     def routed_ffn(self, T):
+        if self.fp8:
+            L.moe_grouped_ffn(self.x8, self.x_s, self.offsets, self.n_routed, T * self.top_k,
+                              self.d, self.inter, self.w13, self.w13_s, self.w2, self.w2_s,
+                              L.MOE_FP8_E4M3, self.y_perm, self.ffn_ws, self.ffn_ws_bytes)
+            return
         L.moe_grouped_ffn(self.x_perm, None, self.offsets, self.n_routed, T * self.top_k, self.d,
                           self.inter, self.w13, None, self.w2, None, L.MOE_BF16, self.y_perm,
                           self.ffn_ws, self.ffn_ws_bytes)
@@ -110,6 +149,11 @@ class MoELayer:
         if self.ws13 is None:
             return
         T = u.shape[0]
+        if self.fp8:
+            L.moe_grouped_ffn(self.u8, self.u_s, self.shared_offsets, 1, T, self.d,
+                              self.shared_inter, self.ws13, self.ws13_s, self.ws2, self.ws2_s,
+                              L.MOE_FP8_E4M3, self.shared_out, self.ffn_ws, self.ffn_ws_bytes)
+            return
         L.moe_grouped_ffn(u, None, self.shared_offsets, 1, T, self.d, self.shared_inter, self.ws13,
                           None, self.ws2, None, L.MOE_BF16, self.shared_out, self.ffn_ws,
                           self.ffn_ws_bytes)
@@ -149,10 +193,11 @@ class MoELayer:
             self.update_bias()
         return out
 
-    # kernels launched by one step(): route (1 + a memset), permute (3),
-    # routed FFN (2), shared FFN (2), combine (1), bias update (1)
+    # kernels launched by one step(): route (1 + a memset), permute (3; FP8:
+    # + the activation quantisation), routed FFN (2), shared FFN (2),
+    # combine (1), bias update (1)
     def launches_per_step(self) -> int:
-        n = 1 + 3 + 2 + 1
+        n = 1 + 3 + 2 + 1 + (1 if self.fp8 else 0)
         if self.ws13 is not None:
             n += 2
         if self.gate_kind == "sigmoid":

@@ -116,7 +116,8 @@ def test_grouped_ffn_rejects_bad_arguments(lib):
     assert rc_ffn(lib, G=0) == L.MOE_ERR_INVALID_ARG
     assert rc_ffn(lib, rows=-1) == L.MOE_ERR_INVALID_ARG
     assert rc_ffn(lib, dt=5) == L.MOE_ERR_INVALID_ARG
-    assert rc_ffn(lib, dt=L.MOE_FP8_E4M3) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    # FP8 without its scale tensors
+    assert rc_ffn(lib, dt=L.MOE_FP8_E4M3) == L.MOE_ERR_INVALID_ARG
     assert rc_ffn(lib, inter=100) == L.MOE_ERR_UNSUPPORTED_SHAPE
     assert rc_ffn(lib, d=384) == L.MOE_ERR_UNSUPPORTED_SHAPE
     assert rc_ffn(lib, G=5000) == L.MOE_ERR_UNSUPPORTED_SHAPE
@@ -144,3 +145,23 @@ def test_binding_raises_moe_error(lib):
     with pytest.raises(L.MoEError) as ei:
         L.moe_combine(A, A, A, None, None, 4, 256, 9, A, stream=0)
     assert ei.value.status == L.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+def test_fp8_entry_points_reject_bad_arguments(lib):
+    assert lib.moe_quant_act_fp8(A, 4, 200, A, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_quant_act_fp8(A, -1, 256, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_quant_act_fp8(MIS, 4, 256, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_quant_act_fp8(A, 4, 256, A, None, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_quant_weights_fp8(A, 2, 100, 256, A, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_quant_weights_fp8(A, 0, 128, 256, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_quant_weights_fp8(A, 2, 128, 256, MIS, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute_fp8(A, None, A, A, 64, 256, 16, 4, A, A, A, A, A, A, 4096,
+                               None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute_fp8(A, A, A, A, 64, 256, 16, 4, A, A, A, A, A, None, 4096,
+                               None) == L.MOE_ERR_WORKSPACE
+    assert lib.moe_expert_up_swiglu_fp8(A, None, A, 4, 256, 256, 128, A, A, A, A,
+                                        None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_down_fp8(A, A, A, 4, 256, 128, 256, A, A, MIS,
+                                   None) == L.MOE_ERR_INVALID_ARG
+    assert L.moe_grouped_ffn_workspace_size(1024, 2048, L.MOE_FP8_E4M3) == \
+        1024 * 2048 + 1024 * 16 * 4
