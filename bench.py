@@ -51,7 +51,7 @@ def peaks():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "gemm.cuh"):
+    for f in ("ptx.cuh", "gemm.cuh", "gemm2sm.cuh"):
         h.update(open(os.path.join(ROOT, "mixture_experts_layer_58_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -83,7 +83,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -388,7 +388,7 @@ def main():
     ratio = 2.0 if cfg.fp8 else 1.0
     peak = (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * ratio
     kname = ("grouped_gemm_fp8_kernel<SwiGLU+quant> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
-             "grouped_gemm_bf16_kernel<256,SwiGLU> (moe_expert_up_swiglu)")
+             "grouped_gemm_bf16_pair_kernel<SwiGLU> (moe_expert_up_swiglu)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
                 "kernel": kname, "kernel_ms": up_ms,

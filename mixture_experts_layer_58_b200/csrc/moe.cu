@@ -15,6 +15,7 @@
 #include "dispatch.cuh"
 #include "fp8.cuh"
 #include "gemm.cuh"
+#include "gemm2sm.cuh"
 #include "gemm_fp8.cuh"
 #include "route.cuh"
 
@@ -188,6 +189,30 @@ int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int 
 
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+// CTA-pair form of the grouped GEMM (256-row tiles, tcgen05 cta_group::2).
+template <int EPI>
+int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int G,
+                             int n_per_group, const int32_t* offsets, void* out, int ldo,
+                             cudaStream_t st) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  CUtensorMap tmA, tmB;
+  if ((rc = make_tmap_bf16(&tmA, A, K, rows, 128)) != MOE_OK) return rc;
+  if ((rc = make_tmap_bf16(&tmB, B, K, static_cast<uint64_t>(G) * n_per_group, 128)) != MOE_OK)
+    return rc;
+  const size_t smem = Gemm2smCfg::smem_bytes(G);
+  auto kern = grouped_gemm_bf16_pair_kernel<EPI>;
+  if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
+  const long long max_tiles =
+      (static_cast<long long>(rows) / kBM2 + G) * static_cast<long long>(n_per_group / 256);
+  const int pairs = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms / 2, max_tiles)));
+  kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
+                                               static_cast<__nv_bfloat16*>(out), ldo, di->status);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
 int check_ffn_shape(int G, int rows, int d, int inter) {
   if (G < 1 || rows < 0 || d <= 0 || inter <= 0) return MOE_ERR_INVALID_ARG;
   if (G > kMaxGroups || d % 256 != 0 || inter % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -355,7 +380,7 @@ int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, int G, int
   if (rows == 0) return MOE_OK;
   if (!x || !group_offsets || !w13 || !h || !aligned16(x) || !aligned16(w13) || !aligned16(h))
     return MOE_ERR_INVALID_ARG;
-  return launch_grouped_gemm<256, EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
+  return launch_grouped_gemm_pair<EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
                                               inter, as_stream(stream));
 }
 
@@ -366,7 +391,7 @@ int moe_expert_down(const void* h, const int32_t* group_offsets, int G, int rows
   if (rows == 0) return MOE_OK;
   if (!h || !group_offsets || !w2 || !y || !aligned16(h) || !aligned16(w2) || !aligned16(y))
     return MOE_ERR_INVALID_ARG;
-  return launch_grouped_gemm<256, EPI_STORE>(h, rows, inter, w2, G, d, group_offsets, y, d,
+  return launch_grouped_gemm_pair<EPI_STORE>(h, rows, inter, w2, G, d, group_offsets, y, d,
                                              as_stream(stream));
 }
 
