@@ -23,8 +23,9 @@ max is 0 gets scale 1; the scale and the division x/scale are evaluated in
 fp32, the precision the kernels use for that decision, and the fp32 quotient
 is rounded to E4M3 to nearest-even, saturating at +-448; dequantisation
 multiplies by BOTH the activation and the weight scale of each 128-wide K
-block ([V3]; the pseudocode's single scale is read as garbled). All other
-arithmetic is fp64.
+block ([V3]; the pseudocode's single scale is read as garbled); the
+intermediate h is held in bf16 between the two expert GEMMs and its codes are
+decided from that value. All other arithmetic is fp64.
 """
 from __future__ import annotations
 
@@ -155,15 +156,24 @@ def _as32(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float32)
 
 
+def round_bf16(x) -> np.ndarray:
+    """Round to the nearest bfloat16 (ties to even), via fp32, as fp32 values."""
+    f = np.asarray(x, dtype=np.float32)
+    bits = f.view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
+    return bits.astype(np.uint32).view(np.float32)
+
+
 def ffn_fp8(xq, xs, qexpert) -> np.ndarray:
     """SwiGLU expert with FP8 operands: a = x W1^T, g = x W3^T (promoted FP8
-    GEMMs), h = silu(a) * g in fp64, h re-quantised per 1x128 tile, then
+    GEMMs), h = silu(a) * g in fp64, h held in bf16 between the two GEMMs (as
+    in the bf16 path) and quantised per 1x128 tile from that value, then
     y = h W2^T (promoted FP8 GEMM)."""
     (w1q, w1s), (w3q, w3s), (w2q, w2s) = qexpert
     a = fp8_gemm(xq, xs, w1q, w1s)
     g = fp8_gemm(xq, xs, w3q, w3s)
     h = a / (1.0 + np.exp(-a)) * g
-    hq, hs = quant_act_1x128(h.astype(np.float32))
+    hq, hs = quant_act_1x128(round_bf16(h))
     return fp8_gemm(hq, hs, w2q, w2s)
 
 

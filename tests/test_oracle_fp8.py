@@ -123,3 +123,12 @@ def test_fp8_ffn_close_to_exact_ffn():
     # four E4M3 roundings (x, W1/W3, h, W2) of relative size <= 2^-4 each
     assert np.abs(y8 - y).max() <= 0.25 * np.abs(y).max()
     assert np.abs(y8 - y).mean() <= 0.1 * np.abs(y).mean()
+
+
+def test_round_bf16_matches_torch_cast():
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.standard_normal(100000) * 10, rng.standard_normal(1000) * 1e-30,
+                        np.array([1.0, -2.5, 0.0, 65504.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9])])
+    x32 = x.astype(np.float32)
+    want = torch.from_numpy(x32).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(fp8.round_bf16(x32), want)
