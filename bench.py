@@ -210,6 +210,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="v3p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--mode", default="five-call", choices=["five-call", "fused"],
+                    help="five-call: route, permute (copy), grouped FFN, combine, bias update; "
+                         "fused: the up-projection gathers the token rows itself (bf16; measured "
+                         "slower: the TMA gathers are request-rate bound)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -248,7 +252,7 @@ def main():
     shared = synth.shared_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
     lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
                    routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
-                   fp8=cfg.fp8, device=dev)
+                   fp8=cfg.fp8, fused_gather=(args.mode == "fused"), device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
     torch.cuda.empty_cache()
@@ -264,17 +268,22 @@ def main():
         lay.permute(u)
         if i is not None:
             up_ev[i][0].record(stream)
-        if cfg.fp8:
-            h8 = lay.ffn_ws
-            hs = lay.ffn_ws[(T * K * I + 255) // 256 * 256:]
+        if lay.fused_gather:
+            L.moe_expert_up_swiglu_gather(u, T, lay.src, lay.offsets, cfg.n_routed, T * K, d, I,
+                                          lay.w13, lay.ffn_ws)
+        elif cfg.fp8:
+            hb = lay.ffn_ws
+            h8 = lay.ffn_ws[(T * K * I * 2 + 255) // 256 * 256:]
+            hs = h8[(T * K * I + 255) // 256 * 256:]
             L.moe_expert_up_swiglu_fp8(lay.x8, lay.x_s, lay.offsets, cfg.n_routed, T * K, d, I,
-                                       lay.w13, lay.w13_s, h8, hs)
+                                       lay.w13, lay.w13_s, hb)
         else:
             L.moe_expert_up_swiglu(lay.x_perm, lay.offsets, cfg.n_routed, T * K, d, I, lay.w13,
                                    lay.ffn_ws)
         if i is not None:
             up_ev[i][1].record(stream)
         if cfg.fp8:
+            L.moe_quant_act_fp8(hb, T * K, I, h8, hs)
             L.moe_expert_down_fp8(h8, hs, lay.offsets, cfg.n_routed, T * K, I, d, lay.w2,
                                   lay.w2_s, lay.y_perm)
         else:
@@ -387,7 +396,9 @@ def main():
     # an FP8 contraction takes the measured bf16 peak x the nominal fp8/bf16 ratio (2)
     ratio = 2.0 if cfg.fp8 else 1.0
     peak = (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * ratio
-    kname = ("grouped_gemm_fp8_kernel<SwiGLU+quant> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
+    kname = ("grouped_gemm_fp8_kernel<SwiGLU> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
+             "grouped_gemm_bf16_pair_kernel<SwiGLU, gather> (moe_expert_up_swiglu_gather)"
+             if lay.fused_gather else
              "grouped_gemm_bf16_pair_kernel<SwiGLU> (moe_expert_up_swiglu)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
@@ -405,6 +416,7 @@ def main():
         "config": {"workload": cfg.name, "T": T, "d": d, "n_routed": cfg.n_routed, "top_k": K,
                    "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
                    "gate": cfg.gate_kind, "global_batch_tokens": T * world,
+                   "mode": "fused gather" if lay.fused_gather else "five-call",
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (22.6 GB of expert weights streamed per step)"
                    if cfg.weights_on_gpu else "L2 not flushed: small workload",

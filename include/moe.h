@@ -121,6 +121,15 @@ MOE_API int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* e
 
 MOE_API size_t moe_permute_workspace_size(int T, int n_routed);
 
+/* moe_permute_index: the index half of moe_permute (expert_offsets, pos,
+ * src_token, same definitions and arguments) without copying any row. For
+ * the fused mode, where the up-projection gathers the token rows itself
+ * (moe_expert_up_swiglu_gather). */
+MOE_API int moe_permute_index(const int32_t* topk_idx, const int32_t* expert_counts, int T,
+                              int n_routed, int top_k, int32_t* expert_offsets, int32_t* pos,
+                              int32_t* src_token, void* workspace, size_t ws_bytes,
+                              moe_stream_t stream);
+
 /* moe_permute_noalloc: moe_permute without a workspace argument. The pages
  * have no counterpart: this entry point exists for callers that cannot
  * allocate device memory where they call the library — for example a plugin
@@ -168,9 +177,10 @@ MOE_API int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
  * dtype MOE_BF16: x, w13, w2 bf16; x_scales / w13_scales / w2_scales unused
  *   (pass NULL); workspace holds h as bf16 [rows, inter].
  * dtype MOE_FP8_E4M3: x, w13, w2 are E4M3 codes (1 byte) with fp32 scales
- *   x_scales [rows, d/128], w13_scales [G, 2*inter/128, d/128],
- *   w2_scales [G, d/128, inter/128] (see the FP8 section); y stays bf16;
- *   workspace holds h as E4M3 [rows, inter] + its scales [rows, inter/128].
+ *   x_scales [rows, d/128], w13_scales [G, 2, inter/128, d/128] (w13 packed by
+ *   moe_pack_w13_fp8), w2_scales [G, d/128, inter/128] (see the FP8 section);
+ *   y stays bf16; workspace holds h as bf16 [rows, inter], then as E4M3
+ *   [rows, inter] + its scales [rows, inter/128].
  */
 MOE_API int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_offsets,
                             int G, int rows, int d, int inter, const void* w13,
@@ -187,6 +197,15 @@ MOE_API size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dty
 MOE_API int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, int G, int rows,
                                  int d, int inter, const void* w13, void* h,
                                  moe_stream_t stream);
+/* moe_expert_up_swiglu_gather: moe_expert_up_swiglu whose x is not copied:
+ * logical row r of x is row src_token[r] of u [T, d] (bf16, 16-B aligned),
+ * read by the kernel itself (TMA gather, four rows per load). src_token,
+ * group_offsets: from moe_permute_index. Removes the expert-contiguous copy
+ * of the dispatch (the "fused gather" of the build plan). */
+MOE_API int moe_expert_up_swiglu_gather(const void* u, int T, const int32_t* src_token,
+                                        const int32_t* group_offsets, int G, int rows, int d,
+                                        int inter, const void* w13, void* h,
+                                        moe_stream_t stream);
 MOE_API int moe_expert_down(const void* h, const int32_t* group_offsets, int G, int rows,
                             int inter, int d, const void* w2, void* y, moe_stream_t stream);
 
@@ -198,7 +217,9 @@ MOE_API int moe_expert_down(const void* h, const int32_t* group_offsets, int G, 
  * (block-quantisation pseudocode of "DeepSeek model architecture explained",
  * 448 = largest E4M3 value). Codes are decided in fp32: scale = amax / 448
  * (an all-zero tile gets 1) and x / scale are IEEE fp32 divisions, the
- * quotient is rounded to E4M3 to nearest-even, saturating at +-448.
+ * quotient is rounded to E4M3 to nearest-even, saturating at +-448. The
+ * intermediate h is held in bf16 between the two GEMMs (as in the bf16 path)
+ * and quantised from that value.
  * E4M3 tensors are 1 byte per element, 16-B aligned; scales fp32, 4-B aligned.
  * The routing (moe_route) stays bf16: the expert indices must be exact.
  *
@@ -206,21 +227,29 @@ MOE_API int moe_expert_down(const void* h, const int32_t* group_offsets, int G, 
  *   scales [rows, cols/128] (one per 1x128 tile). cols % 128 == 0.
  * moe_quant_weights_fp8: w [G, R, C] bf16 -> q [G, R, C] E4M3 and
  *   scales [G, R/128, C/128] (one per 128x128 block). R, C % 128 == 0.
- *   For w13 quantise the packed (interleaved) [G, 2*inter, d] tensor: its
- *   128-row chunks are whole W1 or W3 blocks.
+ * moe_pack_w13_fp8: FP8 expert weights for the up-projection. Quantise W1 and
+ *   W3 stacked as [G, 2, inter, d] (i.e. moe_quant_weights_fp8 with 2G groups:
+ *   its scales [G, 2, inter/128, d/128] are the w13_scales the FP8 FFN takes),
+ *   then pack the codes into w13 [G, 2*inter, d] with 64-row chunks
+ *   interleaved (W1 rows 0..63, W3 rows 0..63, W1 rows 64..127, ...).
+ *   inter % 64 == 0.
  * moe_permute_fp8: moe_permute for E4M3 rows: u8 [T, d] codes + u_scales
  *   [T, d/128] (from moe_quant_act_fp8, quantised once per token) are copied
  *   to x8 [T*top_k, d] + x_scales [T*top_k, d/128]; other arguments as
  *   moe_permute.
  * moe_expert_up_swiglu_fp8 / moe_expert_down_fp8: the two halves of
- *   moe_grouped_ffn in FP8; the first writes h as E4M3 h8 [rows, inter] with
- *   h_scales [rows, inter/128] (h = silu(a) * b is quantised per 1x128 tile
- *   in the GEMM's epilogue), the second reads them and writes bf16 y.
+ *   moe_grouped_ffn in FP8. The first reads x8/x_scales and the packed w13 with
+ *   w13_scales [G, 2, inter/128, d/128] and writes h = silu(a) * b as bf16
+ *   [rows, inter]; the caller quantises h per 1x128 tile with
+ *   moe_quant_act_fp8 (h8, h_scales); the second reads h8/h_scales and w2 with
+ *   w2_scales [G, d/128, inter/128] and writes bf16 y.
  */
 MOE_API int moe_quant_act_fp8(const void* x, int rows, int cols, void* q, float* scales,
                               moe_stream_t stream);
 MOE_API int moe_quant_weights_fp8(const void* w, int G, int R, int C, void* q, float* scales,
                                   moe_stream_t stream);
+MOE_API int moe_pack_w13_fp8(const void* w13_stacked, int G, int inter, int d, void* w13,
+                             moe_stream_t stream);
 MOE_API int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_idx,
                             const int32_t* expert_counts, int T, int d, int n_routed, int top_k,
                             void* x8, float* x_scales, int32_t* expert_offsets, int32_t* pos,
@@ -228,8 +257,8 @@ MOE_API int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t
                             moe_stream_t stream);
 MOE_API int moe_expert_up_swiglu_fp8(const void* x8, const float* x_scales,
                                      const int32_t* group_offsets, int G, int rows, int d,
-                                     int inter, const void* w13, const float* w13_scales, void* h8,
-                                     float* h_scales, moe_stream_t stream);
+                                     int inter, const void* w13, const float* w13_scales, void* h,
+                                     moe_stream_t stream);
 MOE_API int moe_expert_down_fp8(const void* h8, const float* h_scales,
                                 const int32_t* group_offsets, int G, int rows, int inter, int d,
                                 const void* w2, const float* w2_scales, void* y,

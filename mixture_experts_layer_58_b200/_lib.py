@@ -48,6 +48,8 @@ _SIGS = {
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "moe_permute_index": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_up_swiglu_gather": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "moe_grouped_ffn": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp,
                              _sz, _vp]),
     "moe_grouped_ffn_workspace_size": (_sz, [_i, _i, _i]),
@@ -57,7 +59,8 @@ _SIGS = {
     "moe_quant_weights_fp8": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_permute_fp8": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                              _sz, _vp]),
-    "moe_expert_up_swiglu_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "moe_expert_up_swiglu_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_pack_w13_fp8": (_i, [_vp, _i, _i, _i, _vp, _vp]),
     "moe_expert_down_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_bias_update": (_i, [_vp, _vp, _i, _ll, _i, _f, _vp]),
@@ -138,6 +141,20 @@ def moe_permute_noalloc(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_per
                                     _p(src_token), _stream(stream)), "moe_permute_noalloc")
 
 
+def moe_permute_index(topk_idx, expert_counts, T, n_routed, top_k, expert_offsets, pos, src_token,
+                      workspace, ws_bytes, stream=None):
+    _check(_L().moe_permute_index(_p(topk_idx), _p(expert_counts), T, n_routed, top_k,
+                                  _p(expert_offsets), _p(pos), _p(src_token), _p(workspace),
+                                  ws_bytes, _stream(stream)), "moe_permute_index")
+
+
+def moe_expert_up_swiglu_gather(u, T, src_token, group_offsets, G, rows, d, inter, w13, h,
+                                stream=None):
+    _check(_L().moe_expert_up_swiglu_gather(_p(u), T, _p(src_token), _p(group_offsets), G, rows, d,
+                                            inter, _p(w13), _p(h), _stream(stream)),
+           "moe_expert_up_swiglu_gather")
+
+
 def moe_permute_workspace_size(T, n_routed) -> int:
     return _L().moe_permute_workspace_size(T, n_routed)
 
@@ -181,11 +198,16 @@ def moe_permute_fp8(u8, u_scales, topk_idx, expert_counts, T, d, n_routed, top_k
            "moe_permute_fp8")
 
 
-def moe_expert_up_swiglu_fp8(x8, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales, h8,
-                             h_scales, stream=None):
+def moe_expert_up_swiglu_fp8(x8, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales, h,
+                             stream=None):
     _check(_L().moe_expert_up_swiglu_fp8(_p(x8), _p(x_scales), _p(group_offsets), G, rows, d,
-                                         inter, _p(w13), _p(w13_scales), _p(h8), _p(h_scales),
-                                         _stream(stream)), "moe_expert_up_swiglu_fp8")
+                                         inter, _p(w13), _p(w13_scales), _p(h), _stream(stream)),
+           "moe_expert_up_swiglu_fp8")
+
+
+def moe_pack_w13_fp8(w13_stacked, G, inter, d, w13, stream=None):
+    _check(_L().moe_pack_w13_fp8(_p(w13_stacked), G, inter, d, _p(w13), _stream(stream)),
+           "moe_pack_w13_fp8")
 
 
 def moe_expert_down_fp8(h8, h_scales, group_offsets, G, rows, inter, d, w2, w2_scales, y,

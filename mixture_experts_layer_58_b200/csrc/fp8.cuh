@@ -170,4 +170,27 @@ permute_copy_fp8_kernel(const uint8_t* __restrict__ u8, const float* __restrict_
   }
 }
 
+// ---------------------------------------------------------------- w13 packing (E4M3)
+// Codes of W1 and W3 stacked as [G, 2, inter, d] -> [G, 2*inter, d] with 64-row
+// chunks interleaved: rows [128c, 128c+64) = W1 rows [64c, 64c+64), rows
+// [128c+64, 128c+128) = W3 rows [64c, 64c+64). A 128-row tile of the result
+// then holds the gate and up rows of the same 64 h columns.
+__global__ void pack_w13_fp8_kernel(const uint8_t* __restrict__ stacked, int G, int inter, int d,
+                                    uint8_t* __restrict__ w13) {
+  const size_t nvec_row = static_cast<size_t>(d) >> 4;
+  const size_t total = static_cast<size_t>(G) * 2 * inter * nvec_row;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t v = i % nvec_row;
+    const size_t r = i / nvec_row;
+    const size_t g = r / (2 * static_cast<size_t>(inter));
+    const int row13 = static_cast<int>(r - g * 2 * inter);
+    const int c = row13 >> 7;
+    const int within = row13 & 127;
+    const int which = within >> 6;                     // 0 = W1, 1 = W3
+    const size_t srow = (g * 2 + which) * inter + c * 64 + (within & 63);
+    reinterpret_cast<uint4*>(w13)[i] = __ldg(reinterpret_cast<const uint4*>(stacked + srow * d) + v);
+  }
+}
+
 }  // namespace moe

@@ -84,6 +84,21 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// Four rows (r0..r3) of a tensor map whose box is one row high, 64 bf16 wide,
+// into four consecutive 128-byte rows of this CTA's shared memory; completion
+// counted on the leader's barrier.
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int x, int r0, int r1,
+                                                 int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -147,13 +162,16 @@ __device__ __forceinline__ void decode_tile_pair(int t, const int* s_tstart, con
   m_blk = local - n_blk * mt;
 }
 
-template <int EPI>
+// GATHER: the A rows of a tile are not contiguous; logical row r of A is row
+// src_rows[r] of the tensor behind tmA (the token rows of u, read in place
+// of an expert-contiguous copy), fetched four at a time with tile::gather4.
+template <int EPI, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                               const __grid_constant__ CUtensorMap tmB,
                               const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
                               int rows, __nv_bfloat16* __restrict__ out, int ldo,
-                              unsigned int* status) {
+                              const int32_t* __restrict__ src_rows, unsigned int* status) {
   constexpr int BN = 256;
   using C = Gemm2smCfg;
   extern __shared__ uint8_t smem_raw[];
@@ -227,8 +245,10 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = s_tstart[G];
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0 && (GATHER || lane == 0)) {
     // ------------------------------------------------------------ producer (both CTAs)
+    // Gather form: the whole warp issues loads, lane i the four A rows
+    // 4i..4i+3 of this CTA's 128; lane 0 waits and signals.
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0, issued_par = 0;
@@ -238,15 +258,34 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       decode_tile_pair(t, s_tstart, s_off, G, g, m_blk, n_blk);
       const int a_row = s_off[g] + m_blk * kBM2 + static_cast<int>(rank) * 128;
       const int b_row = g * n_per_group + n_blk * BN + static_cast<int>(rank) * 128;
+      int src[4] = {0, 0, 0, 0};
+      if constexpr (GATHER) {
+        // rows past the group's end load any row of the group (masked later)
+        const int first = (s_off[g] >= 0 && s_off[g] < rows) ? s_off[g] : 0;
+        const int end = min(s_off[g + 1], rows);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = a_row + 4 * lane + j;
+          src[j] = __ldg(src_rows + (r >= 0 && r < end ? r : first));
+        }
+      }
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, status, kStatusTimeoutProducer)) {
+        bool got = true;
+        if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, status, kStatusTimeoutProducer);
+        if constexpr (GATHER) got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+        if (!got) {
           ok = false;
           break;
         }
-        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+        if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-        tma_load_2d_pair(sA + stage * C::kABytes, &tmA, bar, kb * kBK, a_row);
-        tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, bar, kb * kBK, b_row);
+        if constexpr (GATHER) {
+          tma_gather4_pair(sA + stage * C::kABytes + lane * 4 * 128, &tmA, bar, kb * kBK, src[0],
+                           src[1], src[2], src[3]);
+        } else {
+          tma_load_2d_pair(sA + stage * C::kABytes, &tmA, bar, kb * kBK, a_row);
+        }
+        if (lane == 0) tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, bar, kb * kBK, b_row);
         issued |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages2) {
@@ -257,7 +296,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     // The leader's full barriers count both CTAs' bytes: once they have all
     // completed no TMA write into either CTA's shared memory is in flight.
-    if (rank == 0)
+    if (rank == 0 && lane == 0)
       for (int s = 0; s < kStages2; ++s)
         if (issued & (1u << s))
           mbar_wait(&full[s], (issued_par >> s) & 1u, status, kStatusTimeoutProducer);

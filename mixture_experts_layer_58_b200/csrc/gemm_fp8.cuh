@@ -8,23 +8,26 @@
 // For every 128-wide K block kb the tensor cores form the block's product
 //   P_kb[m, n] = sum_{k in kb} qa[m, k] * qw[n, k]
 // from a fresh start (tcgen05.mma kind::f8f6f4, 4 x K=32) into one of two
-// 256-column TMEM buffers, and the epilogue warps fold it into fp32 registers:
-//   acc[m, n] += P_kb[m, n] * s_a[m, kb] * s_w[n / 128, kb].
+// 128-column TMEM buffers, and the epilogue warps fold it into fp32 registers:
+//   acc[m, n] += P_kb[m, n] * s_a[m, kb] * s_w[block of n, kb].
 // The scales are the pages' arbitrary fp32 values (max|x| / 448), which the
 // hardware's block-scaled MMA (power-of-two, 32-element scale blocks) cannot
 // express; promotion on the CUDA cores keeps them exact.
 //
-// 10 warps, one persistent CTA per SM:
-//   warp 0      TMA producer: A [128 rows x 128 B] + B [256 rows x 128 B] per stage.
-//   warp 1      MMA issuer: one K block per P buffer, alternating buffers.
+// 10 warps, one persistent CTA per SM, 128 x 128 tiles:
+//   warp 0      TMA producer: A [128 rows x 128 B] + B [128 rows x 128 B] per stage,
+//               6 stages.
+//   warp 1      MMA issuer: one K block (4 x K=32) per P buffer, two buffers of
+//               128 TMEM columns.
 //   warps 2-9   promotion + epilogue. Warp w reads TMEM lane quarter w % 4;
-//               half = (w - 2) / 4 picks its columns [64*half, +64) and
-//               [128 + 64*half, +64): the gate and up columns of the same 64 h
-//               columns when B is an interleaved W1/W3 tile. 128 fp32
-//               accumulators per thread.
-// Epilogues: EPI8_SWIGLU_Q — h = silu(a) * b, then h is quantised to E4M3 with
-// one 1x128 scale per row per tile (the two halves of a row trade their amax
-// through shared memory); EPI8_STORE — bf16 output.
+//               half = (w - 2) / 4 picks its 64 columns: for the up-projection
+//               the gate columns [32*half, +32) and the up columns
+//               [64 + 32*half, +32) of the same 32 h columns (B is W1/W3
+//               interleaved in 64-row chunks), for the down-projection the
+//               columns [64*half, +64). 64 fp32 accumulators per thread.
+// Epilogues: EPI8_SWIGLU — h = silu(a) * b written as bf16 (the caller
+// quantises it per 1x128 tile with the activation quantiser); EPI8_STORE —
+// bf16 output.
 #pragma once
 #include "fp8.cuh"
 #include "gemm.cuh"
@@ -33,11 +36,12 @@ namespace moe {
 
 constexpr int kF8BK = 128;        // K elements (= bytes) per stage = one scale block
 constexpr int kF8UmmaK = 32;      // K of one tcgen05.mma kind::f8f6f4
-constexpr int kF8BN = 256;
+constexpr int kF8BN = 128;
+constexpr int kF8Stages = 6;
 constexpr int kF8Threads = 320;
 constexpr int kF8EpiThreads = 256;
 
-enum { EPI8_STORE = 0, EPI8_SWIGLU_Q = 1 };
+enum { EPI8_STORE = 0, EPI8_SWIGLU = 1 };
 
 struct GemmF8Cfg {
   static constexpr int kABytes = kBM * kF8BK;
@@ -45,9 +49,8 @@ struct GemmF8Cfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * kF8BN;
   static constexpr int kBarBytes = 256;
-  static constexpr int kXchgBytes = 2 * 2 * kBM * static_cast<int>(sizeof(float));
   static size_t smem_bytes(int G) {
-    return 1024 + static_cast<size_t>(kStages) * kStageBytes + kBarBytes + kXchgBytes +
+    return 1024 + static_cast<size_t>(kF8Stages) * kStageBytes + kBarBytes +
            2 * static_cast<size_t>(G + 1) * sizeof(int);
   }
 };
@@ -74,32 +77,30 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const float* __restrict__ a_scales, const float* __restrict__ b_scales,
                         const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
-                        int rows, void* __restrict__ out, int ldo, float* __restrict__ out_scales,
+                        int rows, __nv_bfloat16* __restrict__ out, int ldo,
                         unsigned int* status) {
   using C = GemmF8Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * C::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * C::kBBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* pfull = empty + kStages;
+  uint8_t* sB = smem + kF8Stages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kF8Stages * C::kBBytes);
+  uint64_t* empty = full + kF8Stages;
+  uint64_t* pfull = empty + kF8Stages;
   uint64_t* pempty = pfull + 2;
   uint64_t* mma_done = pempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  float* xchg = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
-  int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(xchg) + C::kXchgBytes);
+  int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_tstart = s_off + (G + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_blocks_n = n_per_group / kF8BN;
   const int num_kb = K / kF8BK;
-  const int nsb = n_per_group / kQBlock;   // weight scale blocks along N, per group
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < kF8Stages; ++s) {
         mbar_init(&full[s], 1);
         mbar_init(&empty[s], 1);
       }
@@ -167,13 +168,13 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         tma_load_2d(sB + stage * C::kBBytes, &tmB, &full[stage], kb * kF8BK, b_row);
         issued |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages) {
+        if (++stage == kF8Stages) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    for (int s = 0; s < kStages; ++s)
+    for (int s = 0; s < kF8Stages; ++s)
       if (issued & (1u << s))
         mbar_wait(&full[s], (issued_par >> s) & 1u, status, kStatusTimeoutProducer);
   } else if (warp == 1 && lane == 0) {
@@ -201,7 +202,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
           umma_e4m3(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, k != 0);
         umma_commit(&empty[stage]);
         umma_commit(&pfull[pb]);
-        if (++stage == kStages) {
+        if (++stage == kF8Stages) {
           stage = 0;
           phase ^= 1u;
         }
@@ -215,29 +216,44 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     const int half = (warp - 2) >> 2;
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const int col0 = half * 64;            // gate (or first-half) columns
-    const int col1 = 128 + half * 64;      // up (or second-half) columns
+    // the thread's two runs of 32 columns
+    const int col0 = (EPI == EPI8_SWIGLU) ? 32 * half : 64 * half;
+    const int col1 = (EPI == EPI8_SWIGLU) ? 64 + 32 * half : 64 * half + 32;
+    const int ksb = num_kb;                   // scale blocks along K
     uint32_t kcount = 0;
     bool broken = false;
-    int local = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       int g, m_blk, n_blk;
       decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
       const int row0 = s_off[g] + m_blk * kBM;
       const int row_end = min(s_off[g + 1], rows);
       const int grow = row0 + row_in_tile;
       const bool valid = grow >= 0 && grow < row_end;
-      const float* sa_row = a_scales + static_cast<size_t>(valid ? grow : 0) * num_kb;
-      const float* sw0 = b_scales + (static_cast<size_t>(g) * nsb + 2 * n_blk) * num_kb;
-      const float* sw1 = sw0 + num_kb;
-      float acc0[64], acc1[64];
+      const float* sa_row = a_scales + static_cast<size_t>(valid ? grow : 0) * ksb;
+      // weight scale rows of the two column runs
+      const float* sw0;
+      const float* sw1;
+      if constexpr (EPI == EPI8_SWIGLU) {
+        // b_scales [G, 2, inter/128, K/128]: W1 blocks, then W3 blocks
+        const int nb = n_per_group / 2 / kQBlock;
+        const int hb = (n_blk * 64) / kQBlock;
+        sw0 = b_scales + ((static_cast<size_t>(g) * 2 + 0) * nb + hb) * ksb;
+        sw1 = b_scales + ((static_cast<size_t>(g) * 2 + 1) * nb + hb) * ksb;
+      } else {
+        // b_scales [G, N/128, K/128]
+        const int nb = n_per_group / kQBlock;
+        sw0 = b_scales + (static_cast<size_t>(g) * nb + n_blk) * ksb;
+        sw1 = sw0;
+      }
+      float acc0[32], acc1[32];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
+      for (int j = 0; j < 32; ++j) {
         acc0[j] = 0.0f;
         acc1[j] = 0.0f;
       }
       float sa_n = valid ? __ldg(sa_row) : 0.0f;
       float w0_n = __ldg(sw0), w1_n = __ldg(sw1);
+#pragma unroll 1
       for (int kb = 0; kb < num_kb; ++kb, ++kcount) {
         const float s0 = sa_n * w0_n;
         const float s1 = sa_n * w1_n;
@@ -251,64 +267,35 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!broken && !mbar_wait(&pfull[pb], ppar, status, kStatusTimeoutEpilogue)) broken = true;
         tc_fence_after();
         const uint32_t taddr = tmem_base + pb * kF8BN + lane_addr;
-        uint32_t r[32];
-        tmem_ld_32cols(taddr + col0, r);
+        uint32_t r0[32], r1[32];
+        tmem_ld_32cols(taddr + col0, r0);
+        tmem_ld_32cols(taddr + col1, r1);
         tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc0[i] = fmaf(__uint_as_float(r[i]), s0, acc0[i]);
-        tmem_ld_32cols(taddr + col0 + 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc0[32 + i] = fmaf(__uint_as_float(r[i]), s0, acc0[32 + i]);
-        tmem_ld_32cols(taddr + col1, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc1[i] = fmaf(__uint_as_float(r[i]), s1, acc1[i]);
-        tmem_ld_32cols(taddr + col1 + 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc1[32 + i] = fmaf(__uint_as_float(r[i]), s1, acc1[32 + i]);
         tc_fence_before();
         mbar_arrive(&pempty[pb]);
-      }
-      if constexpr (EPI == EPI8_SWIGLU_Q) {
-        float amax = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          acc0[j] = silu_f32(acc0[j]) * acc1[j];
-          amax = fmaxf(amax, fabsf(acc0[j]));
+        for (int i = 0; i < 32; ++i) {
+          acc0[i] = fmaf(__uint_as_float(r0[i]), s0, acc0[i]);
+          acc1[i] = fmaf(__uint_as_float(r1[i]), s1, acc1[i]);
         }
-        float* xc = xchg + (local & 1) * (2 * kBM);
-        xc[half * kBM + row_in_tile] = amax;
-        named_bar_sync(1, kF8EpiThreads);
-        amax = fmaxf(amax, xc[(1 - half) * kBM + row_in_tile]);
-        const float s = fp8_scale_of(amax);
-        if (valid) {
-          uint8_t* dst = static_cast<uint8_t*>(out) + static_cast<size_t>(grow) * ldo +
-                         n_blk * 128 + half * 64;
+      }
+      if (valid) {
+        __nv_bfloat16* yrow = out + static_cast<size_t>(grow) * ldo;
+        if constexpr (EPI == EPI8_SWIGLU) {
+          uint4* dst = reinterpret_cast<uint4*>(yrow + n_blk * 64 + 32 * half);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            uint4 o;
-            o.x = to_e4m3x4(__fdiv_rn(acc0[16 * v + 0], s), __fdiv_rn(acc0[16 * v + 1], s),
-                            __fdiv_rn(acc0[16 * v + 2], s), __fdiv_rn(acc0[16 * v + 3], s));
-            o.y = to_e4m3x4(__fdiv_rn(acc0[16 * v + 4], s), __fdiv_rn(acc0[16 * v + 5], s),
-                            __fdiv_rn(acc0[16 * v + 6], s), __fdiv_rn(acc0[16 * v + 7], s));
-            o.z = to_e4m3x4(__fdiv_rn(acc0[16 * v + 8], s), __fdiv_rn(acc0[16 * v + 9], s),
-                            __fdiv_rn(acc0[16 * v + 10], s), __fdiv_rn(acc0[16 * v + 11], s));
-            o.w = to_e4m3x4(__fdiv_rn(acc0[16 * v + 12], s), __fdiv_rn(acc0[16 * v + 13], s),
-                            __fdiv_rn(acc0[16 * v + 14], s), __fdiv_rn(acc0[16 * v + 15], s));
-            reinterpret_cast<uint4*>(dst)[v] = o;
-          }
-          if (half == 0) out_scales[static_cast<size_t>(grow) * (ldo / kQBlock) + n_blk] = s;
-        }
-      } else {
-        if (valid) {
-          __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(out) + static_cast<size_t>(grow) * ldo +
-                                n_blk * kF8BN;
-          uint4* d0 = reinterpret_cast<uint4*>(yrow + col0);
-          uint4* d1 = reinterpret_cast<uint4*>(yrow + col1);
+            float h[8];
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
+            for (int i = 0; i < 8; ++i) h[i] = silu_f32(acc0[8 * v + i]) * acc1[8 * v + i];
+            dst[v] = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
+                                pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+          }
+        } else {
+          uint4* d0 = reinterpret_cast<uint4*>(yrow + n_blk * kF8BN + col0);
+          uint4* d1 = reinterpret_cast<uint4*>(yrow + n_blk * kF8BN + col1);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
             d0[v] = make_uint4(pack_bf16x2(acc0[8 * v], acc0[8 * v + 1]),
                                pack_bf16x2(acc0[8 * v + 2], acc0[8 * v + 3]),
                                pack_bf16x2(acc0[8 * v + 4], acc0[8 * v + 5]),

@@ -166,8 +166,7 @@ int make_tmap_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 template <int EPI>
 int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int K, const void* B,
                             const float* b_scales, int G, int n_per_group,
-                            const int32_t* offsets, void* out, int ldo, float* out_scales,
-                            cudaStream_t st) {
+                            const int32_t* offsets, void* out, int ldo, cudaStream_t st) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
@@ -182,7 +181,7 @@ int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int 
       (static_cast<long long>(rows) / kBM + G) * static_cast<long long>(n_per_group / kF8BN);
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
   kern<<<grid, kF8Threads, smem, st>>>(tmA, tmB, a_scales, b_scales, offsets, G, K, n_per_group,
-                                       rows, out, ldo, out_scales, di->status);
+                                       rows, static_cast<__nv_bfloat16*>(out), ldo, di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -190,25 +189,40 @@ int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int 
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // CTA-pair form of the grouped GEMM (256-row tiles, tcgen05 cta_group::2).
+// With src_rows, logical A row r is row src_rows[r] of A ([a_rows, K]),
+// gathered by the kernel (box one row high).
 template <int EPI>
 int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int G,
                              int n_per_group, const int32_t* offsets, void* out, int ldo,
-                             cudaStream_t st) {
+                             cudaStream_t st, const int32_t* src_rows = nullptr, int a_rows = 0) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
   CUtensorMap tmA, tmB;
-  if ((rc = make_tmap_bf16(&tmA, A, K, rows, 128)) != MOE_OK) return rc;
+  if (src_rows) {
+    if ((rc = make_tmap_bf16(&tmA, A, K, a_rows, 1)) != MOE_OK) return rc;
+  } else if ((rc = make_tmap_bf16(&tmA, A, K, rows, 128)) != MOE_OK) {
+    return rc;
+  }
   if ((rc = make_tmap_bf16(&tmB, B, K, static_cast<uint64_t>(G) * n_per_group, 128)) != MOE_OK)
     return rc;
   const size_t smem = Gemm2smCfg::smem_bytes(G);
-  auto kern = grouped_gemm_bf16_pair_kernel<EPI>;
-  if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
   const long long max_tiles =
       (static_cast<long long>(rows) / kBM2 + G) * static_cast<long long>(n_per_group / 256);
   const int pairs = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms / 2, max_tiles)));
-  kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
-                                               static_cast<__nv_bfloat16*>(out), ldo, di->status);
+  if (src_rows) {
+    auto kern = grouped_gemm_bf16_pair_kernel<EPI, true>;
+    if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
+    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
+                                                 static_cast<__nv_bfloat16*>(out), ldo, src_rows,
+                                                 di->status);
+  } else {
+    auto kern = grouped_gemm_bf16_pair_kernel<EPI, false>;
+    if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
+    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
+                                                 static_cast<__nv_bfloat16*>(out), ldo, nullptr,
+                                                 di->status);
+  }
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -362,13 +376,40 @@ int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* expert_co
   return MOE_OK;
 }
 
+int moe_permute_index(const int32_t* topk_idx, const int32_t* expert_counts, int T,
+                      int n_routed, int top_k, int32_t* expert_offsets, int32_t* pos,
+                      int32_t* src_token, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = as_stream(stream);
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (n_routed + 1), st));
+    return MOE_OK;
+  }
+  if (!topk_idx || !pos || !src_token) return MOE_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < moe_permute_workspace_size(T, n_routed) || !aligned16(workspace))
+    return MOE_ERR_WORKSPACE;
+  const int chunks = (T + kPermChunk - 1) / kPermChunk;
+  int32_t* hist = static_cast<int32_t*>(workspace);
+  permute_hist_kernel<<<chunks, 256, 0, st>>>(topk_idx, T, top_k, n_routed, hist);
+  MOE_CUDA(cudaGetLastError());
+  permute_index_kernel<<<chunks, 256, 0, st>>>(topk_idx, expert_counts, hist, T, top_k, n_routed,
+                                               expert_offsets, pos, src_token);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
 // ------------------------------------------------------------------ expert FFN
 size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dtype) {
   if (rows <= 0 || inter <= 0) return 256;
   if (dtype == MOE_FP8_E4M3) {
+    const size_t hbf = (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
     const size_t codes = (static_cast<size_t>(rows) * inter + 255) / 256 * 256;
     const size_t scales = (static_cast<size_t>(rows) * (inter / 128) * 4 + 255) / 256 * 256;
-    return codes + scales;
+    return hbf + codes + scales;
   }
   return (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
 }
@@ -382,6 +423,20 @@ int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, int G, int
     return MOE_ERR_INVALID_ARG;
   return launch_grouped_gemm_pair<EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
                                               inter, as_stream(stream));
+}
+
+int moe_expert_up_swiglu_gather(const void* u, int T, const int32_t* src_token,
+                                const int32_t* group_offsets, int G, int rows, int d, int inter,
+                                const void* w13, void* h, moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (T == 0 || !u || !src_token || !group_offsets || !w13 || !h || !aligned16(u) ||
+      !aligned16(w13) || !aligned16(h))
+    return MOE_ERR_INVALID_ARG;
+  return launch_grouped_gemm_pair<EPI_SWIGLU>(u, rows, d, w13, G, 2 * inter, group_offsets, h,
+                                              inter, as_stream(stream), src_token, T);
 }
 
 int moe_expert_down(const void* h, const int32_t* group_offsets, int G, int rows, int inter, int d,
@@ -407,10 +462,13 @@ int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_o
       !aligned16(workspace))
     return MOE_ERR_WORKSPACE;
   if (dtype == MOE_FP8_E4M3) {
-    uint8_t* h8 = static_cast<uint8_t*>(workspace);
+    uint8_t* hbf = static_cast<uint8_t*>(workspace);
+    uint8_t* h8 = hbf + (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
     float* hs = reinterpret_cast<float*>(h8 + (static_cast<size_t>(rows) * inter + 255) / 256 * 256);
     rc = moe_expert_up_swiglu_fp8(x, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales,
-                                  h8, hs, stream);
+                                  hbf, stream);
+    if (rc != MOE_OK) return rc;
+    rc = moe_quant_act_fp8(hbf, rows, inter, h8, hs, stream);
     if (rc != MOE_OK) return rc;
     return moe_expert_down_fp8(h8, hs, group_offsets, G, rows, inter, d, w2, w2_scales, y, stream);
   }
@@ -488,18 +546,31 @@ int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_i
 
 int moe_expert_up_swiglu_fp8(const void* x8, const float* x_scales, const int32_t* group_offsets,
                              int G, int rows, int d, int inter, const void* w13,
-                             const float* w13_scales, void* h8, float* h_scales,
-                             moe_stream_t stream) {
+                             const float* w13_scales, void* h, moe_stream_t stream) {
   int rc = check_ffn_shape(G, rows, d, inter);
   if (rc != MOE_OK) return rc;
   if (rows == 0) return MOE_OK;
-  if (!x8 || !x_scales || !group_offsets || !w13 || !w13_scales || !h8 || !h_scales ||
-      !aligned16(x8) || !aligned16(w13) || !aligned16(h8) || !aligned4(x_scales) ||
-      !aligned4(w13_scales) || !aligned4(h_scales))
+  if (!x8 || !x_scales || !group_offsets || !w13 || !w13_scales || !h || !aligned16(x8) ||
+      !aligned16(w13) || !aligned16(h) || !aligned4(x_scales) || !aligned4(w13_scales))
     return MOE_ERR_INVALID_ARG;
-  return launch_grouped_gemm_fp8<EPI8_SWIGLU_Q>(x8, x_scales, rows, d, w13, w13_scales, G,
-                                                2 * inter, group_offsets, h8, inter, h_scales,
-                                                as_stream(stream));
+  return launch_grouped_gemm_fp8<EPI8_SWIGLU>(x8, x_scales, rows, d, w13, w13_scales, G,
+                                              2 * inter, group_offsets, h, inter,
+                                              as_stream(stream));
+}
+
+int moe_pack_w13_fp8(const void* w13_stacked, int G, int inter, int d, void* w13,
+                     moe_stream_t stream) {
+  if (G <= 0 || inter <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (inter % 64 != 0 || d % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!w13_stacked || !w13 || !aligned16(w13_stacked) || !aligned16(w13))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  pack_w13_fp8_kernel<<<di->num_sms * 4, 256, 0, as_stream(stream)>>>(
+      static_cast<const uint8_t*>(w13_stacked), G, inter, d, static_cast<uint8_t*>(w13));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
 }
 
 int moe_expert_down_fp8(const void* h8, const float* h_scales, const int32_t* group_offsets, int G,
@@ -512,7 +583,7 @@ int moe_expert_down_fp8(const void* h8, const float* h_scales, const int32_t* gr
       !aligned16(w2) || !aligned16(y) || !aligned4(h_scales) || !aligned4(w2_scales))
     return MOE_ERR_INVALID_ARG;
   return launch_grouped_gemm_fp8<EPI8_STORE>(h8, h_scales, rows, inter, w2, w2_scales, G, d,
-                                             group_offsets, y, d, nullptr, as_stream(stream));
+                                             group_offsets, y, d, as_stream(stream));
 }
 
 // ------------------------------------------------------------------ combine

@@ -27,7 +27,7 @@ class MoELayer:
 
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
-                 fp8: bool = False, device="cuda"):
+                 fp8: bool = False, fused_gather: bool = False, device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -38,28 +38,31 @@ class MoELayer:
         self.gate_kind = gate_kind
         self.gamma = float(gamma)
         bf = torch.bfloat16
+        self.fp8 = bool(fp8)
+        # fused gather (bf16): the up-projection reads the token rows of u
+        # itself, so the dispatch only computes row indices (no x_perm copy)
+        self.fused_gather = bool(fused_gather) and not self.fp8
         self.centroids = centroids.to(dev, bf).contiguous()
         self.bias = (bias.to(dev, torch.float32).contiguous() if bias is not None
                      else torch.zeros(self.n_routed, dtype=torch.float32, device=dev))
-        self.w13 = self.pack_w13(w1.to(dev, bf).contiguous(), w3.to(dev, bf).contiguous())
+        pack = self.pack_w13_fp8 if self.fp8 else self.pack_w13
+        self.w13 = pack(w1.to(dev, bf).contiguous(), w3.to(dev, bf).contiguous())
         self.w2 = w2.to(dev, bf).contiguous()
         if shared is not None:
             ws1, ws3, ws2 = shared
             self.shared_inter = ws1.shape[0]
-            self.ws13 = self.pack_w13(ws1.to(dev, bf).contiguous()[None],
-                                      ws3.to(dev, bf).contiguous()[None])
+            self.ws13 = pack(ws1.to(dev, bf).contiguous()[None], ws3.to(dev, bf).contiguous()[None])
             self.ws2 = ws2.to(dev, bf).contiguous()
         else:
             self.shared_inter = 0
             self.ws13 = self.ws2 = None
-        self.fp8 = bool(fp8)
         if self.fp8:
             # E4M3 weights with one fp32 scale per 128x128 block (the bf16
             # copies are dropped)
-            self.w13, self.w13_s = self.quant_weights(self.w13)
+            self.w13, self.w13_s = self.w13
             self.w2, self.w2_s = self.quant_weights(self.w2)
             if self.ws13 is not None:
-                self.ws13, self.ws13_s = self.quant_weights(self.ws13)
+                self.ws13, self.ws13_s = self.ws13
                 self.ws2, self.ws2_s = self.quant_weights(self.ws2[None])
         self._T = -1
 
@@ -69,6 +72,17 @@ class MoELayer:
         w13 = torch.empty((G, 2 * inter, d), dtype=torch.bfloat16, device=self.device)
         L.moe_pack_w13(w1, w3, G, inter, d, w13)
         return w13
+
+    def pack_w13_fp8(self, w1, w3):
+        """(E4M3 w13 [G, 2I, d] with W1/W3 interleaved in 64-row chunks,
+        scales [G, 2, I/128, d/128]) from bf16 w1, w3 [G, I, d]."""
+        G, inter, d = w1.shape
+        stacked = torch.stack([w1, w3], dim=1).view(2 * G, inter, d)
+        q, s = self.quant_weights(stacked)
+        del stacked
+        w13 = torch.empty((G, 2 * inter, d), dtype=torch.uint8, device=self.device)
+        L.moe_pack_w13_fp8(q, G, inter, d, w13)
+        return w13, s.view(G, 2, inter // 128, d // 128)
 
     def quant_weights(self, w):
         """E4M3 codes [G, R, C] and fp32 scales [G, R/128, C/128] of bf16 w."""
@@ -93,7 +107,7 @@ class MoELayer:
         self.offsets = torch.empty(self.n_routed + 1, dtype=i32, device=dev)
         self.pos = torch.empty((T, K), dtype=i32, device=dev)
         self.src = torch.empty(rows, dtype=i32, device=dev)
-        self.x_perm = (None if self.fp8 else
+        self.x_perm = (None if (self.fp8 or self.fused_gather) else
                        torch.empty((rows, d), dtype=torch.bfloat16, device=dev))
         self.y_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
         self.perm_ws_bytes = L.moe_permute_workspace_size(T, self.n_routed)
@@ -124,6 +138,10 @@ class MoELayer:
 
     def permute(self, u):
         T = u.shape[0]
+        if self.fused_gather:
+            L.moe_permute_index(self.topk_idx, self.counts, T, self.n_routed, self.top_k,
+                                self.offsets, self.pos, self.src, self.perm_ws, self.perm_ws_bytes)
+            return
         if self.fp8:
             # quantise each token once (1x128 tiles), then copy its codes K times
             L.moe_quant_act_fp8(u, T, self.d, self.u8, self.u_s)
@@ -135,7 +153,14 @@ class MoELayer:
                       self.x_perm, self.offsets, self.pos, self.src, self.perm_ws,
                       self.perm_ws_bytes)
 
-    def routed_ffn(self, T):
+    def routed_ffn(self, T, u=None):
+        if self.fused_gather:
+            rows = T * self.top_k
+            L.moe_expert_up_swiglu_gather(u, T, self.src, self.offsets, self.n_routed, rows, self.d,
+                                          self.inter, self.w13, self.ffn_ws)
+            L.moe_expert_down(self.ffn_ws, self.offsets, self.n_routed, rows, self.inter, self.d,
+                              self.w2, self.y_perm)
+            return
         if self.fp8:
             L.moe_grouped_ffn(self.x8, self.x_s, self.offsets, self.n_routed, T * self.top_k,
                               self.d, self.inter, self.w13, self.w13_s, self.w2, self.w2_s,
@@ -175,7 +200,7 @@ class MoELayer:
         self.route(u)
         if T > 0:
             self.permute(u)
-            self.routed_ffn(T)
+            self.routed_ffn(T, u)
             self.shared_ffn(u)
             self.combine(u, residual, dst)
         return dst
@@ -197,9 +222,11 @@ class MoELayer:
     # + the activation quantisation), routed FFN (2), shared FFN (2),
     # combine (1), bias update (1)
     def launches_per_step(self) -> int:
-        n = 1 + 3 + 2 + 1 + (1 if self.fp8 else 0)
+        ffn = 3 if self.fp8 else 2      # FP8: up-projection, h quantisation, down-projection
+        perm = 2 if self.fused_gather else 3
+        n = 1 + perm + ffn + 1 + (1 if self.fp8 else 0)
         if self.ws13 is not None:
-            n += 2
+            n += ffn
         if self.gate_kind == "sigmoid":
             n += 1
         return n

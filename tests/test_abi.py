@@ -159,9 +159,26 @@ def test_fp8_entry_points_reject_bad_arguments(lib):
                                None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_permute_fp8(A, A, A, A, 64, 256, 16, 4, A, A, A, A, A, None, 4096,
                                None) == L.MOE_ERR_WORKSPACE
-    assert lib.moe_expert_up_swiglu_fp8(A, None, A, 4, 256, 256, 128, A, A, A, A,
+    assert lib.moe_expert_up_swiglu_fp8(A, None, A, 4, 256, 256, 128, A, A, A,
                                         None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_up_swiglu_fp8(A, A, A, 4, 256, 256, 128, A, A, MIS,
+                                        None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_pack_w13_fp8(A, 2, 100, 256, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_pack_w13_fp8(None, 2, 128, 256, A, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_down_fp8(A, A, A, 4, 256, 128, 256, A, A, MIS,
                                    None) == L.MOE_ERR_INVALID_ARG
     assert L.moe_grouped_ffn_workspace_size(1024, 2048, L.MOE_FP8_E4M3) == \
-        1024 * 2048 + 1024 * 16 * 4
+        1024 * 2048 * 2 + 1024 * 2048 + 1024 * 16 * 4
+
+
+def test_fused_gather_entry_points_reject_bad_arguments(lib):
+    assert lib.moe_permute_index(A, A, -1, 16, 4, A, A, A, A, 4096, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute_index(A, A, 64, 16, 9, A, A, A, A, 4096, None) == \
+        L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_permute_index(A, A, 64, 16, 4, A, A, A, None, 4096, None) == L.MOE_ERR_WORKSPACE
+    assert lib.moe_expert_up_swiglu_gather(MIS, 64, A, A, 16, 256, 256, 128, A, A, None) == \
+        L.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_up_swiglu_gather(A, 64, None, A, 16, 256, 256, 128, A, A, None) == \
+        L.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_up_swiglu_gather(A, 0, A, A, 16, 256, 256, 128, A, A, None) == \
+        L.MOE_ERR_INVALID_ARG

@@ -71,14 +71,17 @@ def test_fp8_grouped_ffn_vs_oracle_emulation():
     w1 = _rand_bf16((G, inter, d), 4, 0.05)
     w3 = _rand_bf16((G, inter, d), 5, 0.05)
     w2 = _rand_bf16((G, d, inter), 6, 0.05)
-    w13 = torch.empty((G, 2 * inter, d), dtype=torch.bfloat16, device="cuda")
-    L.moe_pack_w13(w1, w3, G, inter, d, w13)
     x8 = torch.empty((rows, d), dtype=torch.uint8, device="cuda")
     xs = torch.empty((rows, d // 128), dtype=torch.float32, device="cuda")
     L.moe_quant_act_fp8(x, rows, d, x8, xs)
-    w13q = torch.empty_like(w13, dtype=torch.uint8)
-    w13s = torch.empty((G, 2 * inter // 128, d // 128), dtype=torch.float32, device="cuda")
-    L.moe_quant_weights_fp8(w13, G, 2 * inter, d, w13q, w13s)
+    stacked = torch.stack([w1, w3], dim=1).contiguous()            # [G, 2, inter, d]
+    sq = torch.empty((G, 2, inter, d), dtype=torch.uint8, device="cuda")
+    w13s = torch.empty((G, 2, inter // 128, d // 128), dtype=torch.float32, device="cuda")
+    L.moe_quant_weights_fp8(stacked, 2 * G, inter, d, sq, w13s)
+    w13q = torch.empty((G, 2 * inter, d), dtype=torch.uint8, device="cuda")
+    L.moe_pack_w13_fp8(sq, G, inter, d, w13q)
+    # 64-row interleave: rows [128c, 128c+64) of w13 are W1 rows [64c, 64c+64)
+    assert torch.equal(w13q[:, 64:128], sq[:, 1, 0:64]) and torch.equal(w13q[:, 128:192], sq[:, 0, 64:128])
     w2q = torch.empty_like(w2, dtype=torch.uint8)
     w2s = torch.empty((G, d // 128, inter // 128), dtype=torch.float32, device="cuda")
     L.moe_quant_weights_fp8(w2, G, d, inter, w2q, w2s)

@@ -258,3 +258,33 @@ def test_grouped_ffn_tile_paths_by_group_size():
         ref = h.float() @ w2[i].float().T
         check_close(y[a:b].float().cpu().numpy(), ref.cpu().numpy(), max_tol=1e-2,
                     mean_tol=3e-3, what=f"group {i} ({b - a} rows)")
+
+
+@pytest.mark.parametrize("name,T", [("tiny", None), ("tiny", 383), ("mid", None)])
+def test_fused_gather_layer_matches_oracle(name, T):
+    """The fused mode: dispatch computes only row indices and the up-projection
+    gathers the token rows of u itself (TMA gather, four rows per load)."""
+    cfg = synth.CONFIGS[name] if T is None else synth.CONFIGS[name].replace(T=512)
+    inp = Inputs(cfg, T=T, fused_gather=True)
+    _full_check(inp)
+    assert inp.layer.x_perm is None           # no expert-contiguous copy was made
+
+
+def test_gather_up_projection_bit_identical_to_copy():
+    """moe_expert_up_swiglu_gather on u + src_token equals moe_expert_up_swiglu
+    on the copied x_perm bit for bit (same tiles, same MMA order)."""
+    cfg = synth.CONFIGS["mid"]
+    inp = Inputs(cfg)
+    lay = inp.layer
+    _run_forward(inp)
+    T, K = cfg.T, cfg.top_k
+    rows = T * K
+    h_copy = torch.empty((rows, cfg.inter), dtype=torch.bfloat16, device="cuda")
+    h_gath = torch.full((rows, cfg.inter), 9.0, dtype=torch.bfloat16, device="cuda")
+    L.moe_expert_up_swiglu(lay.x_perm, lay.offsets, cfg.n_routed, rows, cfg.d, cfg.inter, lay.w13,
+                           h_copy)
+    L.moe_expert_up_swiglu_gather(inp.u_dev, T, lay.src, lay.offsets, cfg.n_routed, rows, cfg.d,
+                                  cfg.inter, lay.w13, h_gath)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    assert torch.equal(h_copy, h_gath)

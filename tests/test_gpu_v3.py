@@ -126,3 +126,23 @@ def test_v3_decode_layer(name, cuda_ok):
     _check_sampled_output(inp, lay, tokens)
     del inp
     torch.cuda.empty_cache()
+
+
+def test_v3p_fused_gather_sampled(cuda_ok):
+    """V3 prefill in the fused mode (no x_perm copy): routing of every token and
+    sampled outputs against the oracle."""
+    from mixture_experts_layer_58_b200 import build
+    build.build()
+    inp = Inputs(synth.CONFIGS["v3p"], fused_gather=True)
+    cfg, lay = inp.cfg, inp.layer
+    lay.forward(inp.u_dev)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    r = inp.oracle_route()
+    check_route(lay.topk_idx.cpu().numpy(), lay.topk_gate.cpu().numpy(),
+                lay.counts.cpu().numpy(), r, cfg.routed_scale, inp.u, inp.e, cfg.gate_kind)
+    tokens, _ = _sample_tokens(lay.topk_idx.cpu().numpy(), lay.counts.cpu().numpy(),
+                               np.random.default_rng(5), n_random=4)
+    _check_sampled_output(inp, lay, tokens)
+    del inp
+    torch.cuda.empty_cache()
