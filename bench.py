@@ -399,7 +399,8 @@ def main():
     kname = ("grouped_gemm_fp8_kernel<SwiGLU> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
              "grouped_gemm_bf16_pair_kernel<SwiGLU, gather> (moe_expert_up_swiglu_gather)"
              if lay.fused_gather else
-             "grouped_gemm_bf16_pair_kernel<SwiGLU> (moe_expert_up_swiglu)")
+             "grouped_gemm bf16 <SwiGLU>, CTA-pair or 1-CTA tiles by group size "
+             "(moe_expert_up_swiglu)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
                 "kernel": kname, "kernel_ms": up_ms,

@@ -310,6 +310,14 @@ MOE_API int moe_last_cuda_error(void);
  * Returns MOE_ERR_DEVICE_TIMEOUT if the word was non-zero. */
 MOE_API int moe_get_device_status(unsigned int* status, int clear);
 
+/* Diagnostic for the failure-detection path: enqueues a one-thread kernel that
+ * waits on a barrier nothing will complete, gives up after limit_ms
+ * (1..10000) the way every pipeline wait of the library does, and ORs 8
+ * into the device status word; moe_get_device_status() then
+ * returns MOE_ERR_DEVICE_TIMEOUT. The device context stays usable. No
+ * counterpart in the pages. */
+MOE_API int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream);
+
 /* Library version, major*10000 + minor*100 + patch. */
 MOE_API int moe_version(void);
 

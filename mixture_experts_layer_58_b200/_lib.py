@@ -69,6 +69,7 @@ _SIGS = {
     "moe_last_cuda_error": (_i, []),
     "moe_get_device_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i]),
     "moe_version": (_i, []),
+    "moe_selftest_wait_timeout": (_i, [_i, _vp]),
 }
 
 _LIB = None
@@ -238,6 +239,10 @@ def moe_get_device_status(clear: bool = True) -> int:
     if rc not in (MOE_OK, MOE_ERR_DEVICE_TIMEOUT):
         raise MoEError(rc, "moe_get_device_status")
     return int(v.value)
+
+
+def moe_selftest_wait_timeout(limit_ms: int, stream=None):
+    _check(_L().moe_selftest_wait_timeout(limit_ms, _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def moe_strerror(status: int) -> str:

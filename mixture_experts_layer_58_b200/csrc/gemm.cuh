@@ -38,7 +38,7 @@ struct GemmCfg {
   static constexpr int kBarBytes = 256;
   static size_t smem_bytes(int G) {
     return 1024 + static_cast<size_t>(kStages) * kStageBytes + kBarBytes +
-           2 * static_cast<size_t>(G + 1) * sizeof(int);
+           3 * static_cast<size_t>(G + 1) * sizeof(int);
   }
 };
 
@@ -47,8 +47,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // tile index -> (group, m block, n block); m blocks fastest inside a group.
-__device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const int* s_off, int G,
-                                            int& g, int& m_blk, int& n_blk) {
+// Group g covers rows [s_off[g], s_end[g]).
+__device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const int* s_off,
+                                            const int* s_end, int G, int& g, int& m_blk,
+                                            int& n_blk) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -56,7 +58,7 @@ __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const in
   }
   g = lo;
   const int local = t - s_tstart[g];
-  const int mt = (s_off[g + 1] - s_off[g] + kBM - 1) / kBM;
+  const int mt = (s_end[g] - s_off[g] + kBM - 1) / kBM;
   n_blk = local / mt;
   m_blk = local - n_blk * mt;
 }
@@ -83,6 +85,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_tstart = s_off + (G + 1);
+  int* s_end = s_tstart + (G + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -117,6 +120,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         const int o0 = offsets[g];
         const int o1 = offsets[g + 1];
         s_off[g] = o0;
+        s_end[g] = o1 > o0 ? o1 : o0;
         nt = (o1 > o0 ? (o1 - o0 + kBM - 1) / kBM : 0) * n_blocks_n;
       }
       int v = nt;
@@ -131,6 +135,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0) {
       s_tstart[G] = carry;
       s_off[G] = offsets[G];
+      s_end[G] = offsets[G];
     }
   }
   tc_fence_before();
@@ -147,7 +152,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
       int g, m_blk, n_blk;
-      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int a_row = s_off[g] + m_blk * kBM;
       const int b_row = g * n_per_group + n_blk * BN;
       for (int kb = 0; kb < num_kb; ++kb) {
@@ -215,13 +220,13 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     int local = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
       int g, m_blk, n_blk;
-      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_par, status, kStatusTimeoutEpilogue)) break;
       tc_fence_after();
       const int grow = s_off[g] + m_blk * kBM + row_in_tile;
-      const int row_end = min(s_off[g + 1], rows);
+      const int row_end = min(s_end[g], rows);
       const bool valid = grow < row_end;
       const uint32_t taddr = tmem_base + acc * BN + lane_addr;
       if constexpr (EPI == EPI_SWIGLU) {

@@ -35,7 +35,7 @@ struct Gemm2smCfg {
   static constexpr int kBarBytes = 256;
   static size_t smem_bytes(int G) {
     return 1024 + static_cast<size_t>(kStages2) * kStageBytes + kBarBytes +
-           2 * static_cast<size_t>(G + 1) * sizeof(int);
+           3 * static_cast<size_t>(G + 1) * sizeof(int);
   }
 };
 
@@ -149,7 +149,8 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 
 // tile index -> (group, 256-row block, n block); row blocks fastest in a group.
 __device__ __forceinline__ void decode_tile_pair(int t, const int* s_tstart, const int* s_off,
-                                                 int G, int& g, int& m_blk, int& n_blk) {
+                                                 const int* s_end, int G, int& g, int& m_blk,
+                                                 int& n_blk) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -157,7 +158,7 @@ __device__ __forceinline__ void decode_tile_pair(int t, const int* s_tstart, con
   }
   g = lo;
   const int local = t - s_tstart[g];
-  const int mt = (s_off[g + 1] - s_off[g] + kBM2 - 1) / kBM2;
+  const int mt = (s_end[g] - s_off[g] + kBM2 - 1) / kBM2;
   n_blk = local / mt;
   m_blk = local - n_blk * mt;
 }
@@ -186,6 +187,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_tstart = s_off + (G + 1);
+  int* s_end = s_tstart + (G + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -222,6 +224,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         const int o0 = offsets[g];
         const int o1 = offsets[g + 1];
         s_off[g] = o0;
+        s_end[g] = o1 > o0 ? o1 : o0;
         nt = (o1 > o0 ? (o1 - o0 + kBM2 - 1) / kBM2 : 0) * n_blocks_n;
       }
       int v = nt;
@@ -236,6 +239,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0) {
       s_tstart[G] = carry;
       s_off[G] = offsets[G];
+      s_end[G] = offsets[G];
     }
   }
   tc_fence_before();
@@ -255,14 +259,14 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     bool ok = true;
     for (int t = pair; t < total_tiles && ok; t += npairs) {
       int g, m_blk, n_blk;
-      decode_tile_pair(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      decode_tile_pair(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int a_row = s_off[g] + m_blk * kBM2 + static_cast<int>(rank) * 128;
       const int b_row = g * n_per_group + n_blk * BN + static_cast<int>(rank) * 128;
       int src[4] = {0, 0, 0, 0};
       if constexpr (GATHER) {
         // rows past the group's end load any row of the group (masked later)
         const int first = (s_off[g] >= 0 && s_off[g] < rows) ? s_off[g] : 0;
-        const int end = min(s_off[g + 1], rows);
+        const int end = min(s_end[g], rows);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int r = a_row + 4 * lane + j;
@@ -350,13 +354,13 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     int local = 0;
     for (int t = pair; t < total_tiles; t += npairs, ++local) {
       int g, m_blk, n_blk;
-      decode_tile_pair(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      decode_tile_pair(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_par, status, kStatusTimeoutEpilogue)) break;
       tc_fence_after();
       const int grow = s_off[g] + m_blk * kBM2 + static_cast<int>(rank) * 128 + row_in_half;
-      const int row_end = min(s_off[g + 1], rows);
+      const int row_end = min(s_end[g], rows);
       const bool valid = grow >= 0 && grow < row_end;
       const uint32_t taddr = tmem_base + acc * BN + lane_addr;
       if constexpr (EPI == EPI_SWIGLU) {

@@ -51,7 +51,7 @@ struct GemmF8Cfg {
   static constexpr int kBarBytes = 256;
   static size_t smem_bytes(int G) {
     return 1024 + static_cast<size_t>(kF8Stages) * kStageBytes + kBarBytes +
-           2 * static_cast<size_t>(G + 1) * sizeof(int);
+           3 * static_cast<size_t>(G + 1) * sizeof(int);
   }
 };
 
@@ -92,6 +92,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_tstart = s_off + (G + 1);
+  int* s_end = s_tstart + (G + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -125,6 +126,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         const int o0 = offsets[g];
         const int o1 = offsets[g + 1];
         s_off[g] = o0;
+        s_end[g] = o1 > o0 ? o1 : o0;
         nt = (o1 > o0 ? (o1 - o0 + kBM - 1) / kBM : 0) * n_blocks_n;
       }
       int v = nt;
@@ -139,6 +141,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0) {
       s_tstart[G] = carry;
       s_off[G] = offsets[G];
+      s_end[G] = offsets[G];
     }
   }
   tc_fence_before();
@@ -155,7 +158,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
       int g, m_blk, n_blk;
-      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int a_row = s_off[g] + m_blk * kBM;
       const int b_row = g * n_per_group + n_blk * kF8BN;
       for (int kb = 0; kb < num_kb; ++kb) {
@@ -224,9 +227,9 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     bool broken = false;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       int g, m_blk, n_blk;
-      decode_tile(t, s_tstart, s_off, G, g, m_blk, n_blk);
+      decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int row0 = s_off[g] + m_blk * kBM;
-      const int row_end = min(s_off[g + 1], rows);
+      const int row_end = min(s_end[g], rows);
       const int grow = row0 + row_in_tile;
       const bool valid = grow >= 0 && grow < row_end;
       const float* sa_row = a_scales + static_cast<size_t>(valid ? grow : 0) * ksb;

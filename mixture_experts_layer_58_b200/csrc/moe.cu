@@ -194,7 +194,8 @@ inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3
 template <int EPI>
 int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int G,
                              int n_per_group, const int32_t* offsets, void* out, int ldo,
-                             cudaStream_t st, const int32_t* src_rows = nullptr, int a_rows = 0) {
+                             cudaStream_t st, const int32_t* src_rows = nullptr,
+                             int a_rows = 0) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
@@ -227,6 +228,14 @@ int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int 
   return MOE_OK;
 }
 
+// Tile shape of the bf16 expert GEMMs, chosen per call from the average
+// group size: CTA-pair 256-row tiles move less data per flop, but a group of a
+// few rows (decode) would fill a 256-row tile with padding, so groups that
+// average fewer than 256 rows run on single-CTA 128-row tiles.
+inline bool use_pair_tiles(int rows, int G) {
+  return static_cast<long long>(rows) >= 256LL * G;
+}
+
 int check_ffn_shape(int G, int rows, int d, int inter) {
   if (G < 1 || rows < 0 || d <= 0 || inter <= 0) return MOE_ERR_INVALID_ARG;
   if (G > kMaxGroups || d % 256 != 0 || inter % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -257,11 +266,40 @@ int launch_route_k(int kind, const CUtensorMap& tmU, const CUtensorMap& tmE, con
   return MOE_OK;
 }
 
+// Diagnostic: one thread waits on an mbarrier that nothing arrives on, for at
+// most limit_ns, then records kStatusTimeoutSelfTest in the status word, the
+// way every pipeline wait of the library gives up.
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, unsigned int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        atomicOr(status, kStatusTimeoutSelfTest);
+        break;
+      }
+    }
+  }
+}
+
 }  // namespace
 
 extern "C" {
 
 int moe_version(void) { return 100; }
+
+int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream) {
+  if (limit_ms <= 0 || limit_ms > 10000) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(
+      static_cast<unsigned long long>(limit_ms) * 1000000ull, di->status);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
 
 const char* moe_strerror(int s) {
   switch (s) {
@@ -421,7 +459,10 @@ int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, int G, int
   if (rows == 0) return MOE_OK;
   if (!x || !group_offsets || !w13 || !h || !aligned16(x) || !aligned16(w13) || !aligned16(h))
     return MOE_ERR_INVALID_ARG;
-  return launch_grouped_gemm_pair<EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
+  if (use_pair_tiles(rows, G))
+    return launch_grouped_gemm_pair<EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
+                                                inter, as_stream(stream));
+  return launch_grouped_gemm<256, EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
                                               inter, as_stream(stream));
 }
 
@@ -446,7 +487,10 @@ int moe_expert_down(const void* h, const int32_t* group_offsets, int G, int rows
   if (rows == 0) return MOE_OK;
   if (!h || !group_offsets || !w2 || !y || !aligned16(h) || !aligned16(w2) || !aligned16(y))
     return MOE_ERR_INVALID_ARG;
-  return launch_grouped_gemm_pair<EPI_STORE>(h, rows, inter, w2, G, d, group_offsets, y, d,
+  if (use_pair_tiles(rows, G))
+    return launch_grouped_gemm_pair<EPI_STORE>(h, rows, inter, w2, G, d, group_offsets, y, d,
+                                               as_stream(stream));
+  return launch_grouped_gemm<256, EPI_STORE>(h, rows, inter, w2, G, d, group_offsets, y, d,
                                              as_stream(stream));
 }
 

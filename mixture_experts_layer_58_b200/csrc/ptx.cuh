@@ -13,6 +13,7 @@ enum : unsigned int {
   kStatusTimeoutProducer = 1u,
   kStatusTimeoutMma = 2u,
   kStatusTimeoutEpilogue = 4u,
+  kStatusTimeoutSelfTest = 8u,
 };
 
 // Upper bound for any single wait on an mbarrier, in nanoseconds of the

@@ -219,10 +219,12 @@ class MoELayer:
         return out
 
     # kernels launched by one step(): route (1 + a memset), permute (3; FP8:
-    # + the activation quantisation), routed FFN (2), shared FFN (2),
-    # combine (1), bias update (1)
+    # + the activation quantisation), routed and shared FFN, combine (1),
+    # bias update (1)
     def launches_per_step(self) -> int:
-        ffn = 3 if self.fp8 else 2      # FP8: up-projection, h quantisation, down-projection
+        # bf16: up and down one launch each; FP8: up-projection, h
+        # quantisation, down-projection
+        ffn = 3 if self.fp8 else 2
         perm = 2 if self.fused_gather else 3
         n = 1 + perm + ffn + 1 + (1 if self.fp8 else 0)
         if self.ws13 is not None:

@@ -182,3 +182,8 @@ def test_fused_gather_entry_points_reject_bad_arguments(lib):
         L.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_up_swiglu_gather(A, 0, A, A, 16, 256, 256, 128, A, A, None) == \
         L.MOE_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_bad_limit(lib):
+    assert lib.moe_selftest_wait_timeout(0, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_wait_timeout(20000, None) == L.MOE_ERR_INVALID_ARG

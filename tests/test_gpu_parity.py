@@ -226,12 +226,17 @@ def test_grouped_ffn_single_group_vs_torch_matmul():
                 what="h")
 
 
-def test_grouped_ffn_tile_paths_by_group_size():
-    """Group sizes that hit every tile path of the grouped GEMM: empty groups,
-    swapped tiles of 1..127 rows (N rounded up to 16), full 128-row tiles and
-    full + ragged combinations. Each group against fp32 torch matmuls of the
-    same bf16 operands, h rounded to bf16 as the kernel does."""
-    sizes = [1, 15, 0, 16, 17, 31, 32, 33, 100, 127, 128, 129, 255, 256, 0, 300]
+@pytest.mark.parametrize("extra", [0, 600])
+def test_grouped_ffn_tile_paths_by_group_size(extra):
+    """Group sizes that hit every tile path of both grouped-GEMM forms: empty
+    groups, ragged last tiles of every size, full tiles. Each group against fp32
+    torch matmuls of the same bf16 operands, h rounded to bf16 as the kernel
+    does."""
+    # extra = 0: groups average < 256 rows -> single-CTA 128-row tiles;
+    # extra = 600: larger groups -> CTA-pair 256-row tiles. Either way the
+    # last tile of a group is ragged in every way (1..255 valid rows).
+    sizes = [1, 15, 0, 16, 17, 31, 32, 33, 100, 127, 128, 129, 255, 256, 0, 300, 384, 385, 513]
+    sizes = [s + extra if s else 0 for s in sizes]
     G, d, inter = len(sizes), 256, 256
     rows = sum(sizes)
     g = torch.Generator(device="cuda").manual_seed(12)
@@ -288,3 +293,17 @@ def test_gather_up_projection_bit_identical_to_copy():
     torch.cuda.synchronize()
     assert L.moe_get_device_status() == 0
     assert torch.equal(h_copy, h_gath)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait that nothing completes gives up after its limit (50 ms here),
+    the host reads MOE_ERR_DEVICE_TIMEOUT with the self-test bit, the status is
+    cleared, and the layer still runs correctly afterwards."""
+    assert L.moe_get_device_status() == 0
+    L.moe_selftest_wait_timeout(50)
+    torch.cuda.synchronize()
+    st = L.moe_get_device_status(clear=True)
+    assert st & 8
+    assert L.moe_get_device_status() == 0
+    inp = Inputs(synth.CONFIGS["tiny"])
+    _full_check(inp)
