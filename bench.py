@@ -49,6 +49,24 @@ def peaks():
     return d
 
 
+def cublas_fp8_tflops(dev, n: int = 8192, reps: int = 10) -> float:
+    """Best-of-`reps` rate of one cuBLAS E4M3 GEMM (torch._scaled_mm, n^3, fp32
+    scales, bf16 out), as context for the FP8 roofline; measured on `dev`."""
+    import torch
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    best = float("inf")
+    for _ in range(reps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for f in ("ptx.cuh", "gemm.cuh", "gemm2sm.cuh"):
@@ -203,6 +221,134 @@ def run_reference(args, cfg, rank):
 
 
 # ----------------------------------------------------------------------------- our arm
+def run_train(args, cfg, rank, world, local, dev):
+    """Training step of the layer: forward (train=True), backward from a
+    seeded dL/dh', bias update. Value = routed tokens per second of whole
+    steps; roofline of the larger of the two biggest backward GEMMs (the
+    routed up-projection dgrad dx = dac W13 and the W13 weight gradient,
+    2 T K (2I) d flops each), timed with CUDA events inside the timed steps."""
+    import torch
+    import torch.distributed as dist
+    from mixture_experts_layer_58_b200 import dp, synth
+    from mixture_experts_layer_58_b200.layer import MoELayer
+    if cfg.fp8:
+        raise SystemExit("train mode runs the bf16 layer")
+    T, K, d, I = cfg.T, cfg.top_k, cfg.d, cfg.inter
+    W1, W3, W2 = synth.all_expert_weights(cfg, "cuda")
+    lay = MoELayer(synth.centroids(cfg), synth.bias(cfg), W1, W3, W2,
+                   synth.shared_weights(cfg, "cuda"), top_k=K, routed_scale=cfg.routed_scale,
+                   gate_kind=cfg.gate_kind, gamma=cfg.gamma, device=dev)
+    del W1, W3, W2
+    torch.cuda.empty_cache()
+    u_host = synth.tokens(cfg)
+    g = torch.Generator().manual_seed(1234 + rank)
+    dout_host = (torch.randn(T, d, generator=g) * 0.05).bfloat16()
+    u = u_host.to(dev)
+    dout = dout_host.to(dev)
+    stream = torch.cuda.current_stream()
+
+    def step(timers=None):
+        lay.forward(u, train=True)
+        lay.backward(dout, timers)
+        if cfg.gate_kind == "sigmoid":
+            if world > 1:
+                lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
+            else:
+                lay.update_bias()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if L_status() != 0:
+        raise SystemExit("device timeout during warm-up")
+    timers = {}
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(timers)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    if L_status() != 0:
+        raise SystemExit("device timeout during the timed region")
+    ms_step = ms / args.steps
+    kms = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in timers.items()}
+    kname = max(kms, key=kms.get)
+    flops = 2.0 * T * K * 2 * I * d
+    pk = peaks()
+    peak = pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]
+    achieved = flops / (kms[kname] * 1e-3) / 1e12
+    fwd_flops = T * cfg.flops_per_token()
+    # backward: dgrad and wgrad of every forward GEMM except the router's
+    # (2x the expert FLOPs), plus O(T K d) elementwise work
+    step_flops = fwd_flops + 2 * (fwd_flops - 2.0 * T * d * cfg.n_routed)
+
+    # e2e: the batch and dL/dh' from pinned host memory, du back, every step
+    u_pin, dout_pin = u_host.pin_memory(), dout_host.pin_memory()
+    du_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        u.copy_(u_pin, non_blocking=True)
+        dout.copy_(dout_pin, non_blocking=True)
+        step()
+        du_pin.copy_(lay.du, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    if rank == 0:
+        print(json.dumps({
+            "metric": "routed tokens/sec per DeepSeekMoE layer training step (forward + backward "
+                      "+ bias update) on 1 B200",
+            "value": T * world / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init weights of the layer shape)",
+            "config": {"workload": cfg.name, "mode": "train", "T": T, "d": d,
+                       "n_routed": cfg.n_routed, "top_k": K, "inter": I,
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2"},
+            "step_tflops": step_flops / (ms_step * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "kernel": {"dx": "grouped_dgrad_bf16_kernel<store> (moe_expert_up_backward)",
+                                    "dw13": "grouped_wgrad_bf16_kernel (moe_expert_wgrad, dW13)"}[kname],
+                         "kernel_ms": kms[kname], "other_ms": kms,
+                         "peak_source": f"{pk['_source']} bf16_tflops_sustained"},
+            "e2e": {"value": T * world / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 2 * T * d * 2, "d2h_bytes_per_step": T * d * 2,
+                    "api": "MoELayer.forward(train=True) + MoELayer.backward"},
+            "gpu_launches": args.steps * (lay.launches_per_step() + lay.launches_per_backward()),
+            "clocks": clk.summary(),
+        }), flush=True)
+
+
+def L_status() -> int:
+    from mixture_experts_layer_58_b200 import _lib as L
+    return L.moe_get_device_status()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -210,10 +356,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="v3p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--mode", default="five-call", choices=["five-call", "fused"],
+    ap.add_argument("--mode", default="five-call", choices=["five-call", "fused", "train"],
                     help="five-call: route, permute (copy), grouped FFN, combine, bias update; "
                          "fused: the up-projection gathers the token rows itself (bf16; measured "
-                         "slower: the TMA gathers are request-rate bound)")
+                         "slower: the TMA gathers are request-rate bound); train: forward with "
+                         "saved pre-activations + backward + bias update (bf16)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -242,6 +389,9 @@ def main():
     from mixture_experts_layer_58_b200 import build, dp
     from mixture_experts_layer_58_b200.layer import MoELayer
     build.build()
+    if args.mode == "train":
+        run_train(args, cfg, rank, world, local, dev)
+        return
     L.load()
 
     # ---- inputs: same workload on every rank, each rank its own batch (seed + rank)
@@ -406,6 +556,11 @@ def main():
                 "kernel": kname, "kernel_ms": up_ms,
                 "peak_source": f"{pk['_source']} bf16_tflops_sustained"
                                + (" x 2 (nominal fp8/bf16)" if cfg.fp8 else "")}
+    if cfg.fp8:
+        try:
+            roofline["cublas_fp8_tflops_live"] = cublas_fp8_tflops(dev)
+        except (RuntimeError, AttributeError) as exc:   # context only
+            roofline["cublas_fp8_tflops_live"] = f"not measured: {exc}"[:120]
     layer_flops = T * cfg.flops_per_token()
     layer_tflops = layer_flops / (ms_step * 1e-3) / 1e12
 

@@ -166,8 +166,8 @@ MOE_API int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
  *
  *   x      [rows, d] bf16, 16-B aligned.
  *   w13    [G, 2*inter, d] bf16, 16-B aligned: W1 and W3 of each group,
- *          row-interleaved in 128-row chunks ([W1 rows 0..127; W3 rows
- *          0..127; W1 rows 128..255; ...]); moe_pack_w13 builds it.
+ *          row-interleaved in 16-row chunks ([W1 rows 0..15; W3 rows
+ *          0..15; W1 rows 16..31; ...]); moe_pack_w13 builds it.
  *   w2     [G, d, inter] bf16, 16-B aligned.
  *   y      [rows, d] bf16 out, 16-B aligned.
  *   workspace >= moe_grouped_ffn_workspace_size(rows, inter, dtype): holds
@@ -291,6 +291,92 @@ MOE_API int moe_combine(const void* y_perm, const int32_t* pos, const float* top
  */
 MOE_API int moe_bias_update(const int32_t* expert_counts, float* bias, int n_routed,
                             long long T, int top_k, float gamma, moe_stream_t stream);
+
+/* ------------------------------------------------------------------ backward
+ * The gradient of the layer forward above ("DeepSeek-V3 technical report",
+ * Method §2, and the softmax-over-top-k variant of "DeepSeek model
+ * architecture explained"). The pages give no backward equations and say
+ * only that gradients are computed in BF16: these calls compute the exact
+ * derivative of the forward with the top-K selection held fixed (no gradient
+ * reaches the bias, which only selects), bf16 tensors in and out, fp32
+ * accumulation. The calls of one backward step, in order:
+ *
+ *   forward (training)  moe_expert_up_swiglu_train also keeps ac
+ *   1 moe_combine_backward      dgate, dy_perm          (from dout, y_perm)
+ *   2 moe_expert_down_backward  dac = SwiGLU'(dy W2)     (routed; shared: G = 1)
+ *   3 moe_expert_up_backward    dx = dac W13
+ *   4 moe_expert_wgrad          dW2 = dy^T h,  dW13 = dac^T x
+ *   5 moe_gate_backward         dz (selected logits), dz_perm
+ *   6 moe_combine_dx            du
+ *   7 moe_centroid_grad         de
+ *
+ * Shapes as for moe_grouped_ffn (d % 256 == 0, inter % 128 == 0, G <= 1024);
+ * all tensors row-major, 16-B aligned, caller-owned; asynchronous on
+ * `stream`; errors as for the forward calls.
+ *
+ * moe_expert_up_swiglu_train: moe_expert_up_swiglu that also writes the
+ * pre-activations ac [rows, 2*inter] bf16 (x W13^T, in the packed W13 column
+ * order: 16 columns of x W1^T, then the same 16 of x W3^T, ...), which the
+ * backward of the SwiGLU needs. */
+MOE_API int moe_expert_up_swiglu_train(const void* x, const int32_t* group_offsets, int G,
+                                       int rows, int d, int inter, const void* w13, void* h,
+                                       void* ac, moe_stream_t stream);
+
+/* moe_combine_backward: for the routed term sum_k g_{t,k} y_{t,k} of h'_t,
+ *   dgate[t,k] = dout_t . y_perm[pos[t,k]]   fp32 [T, top_k]
+ *   dy_perm[pos[t,k]] = topk_gate[t,k] * dout_t   bf16 [T*top_k, d]
+ * dout, y_perm, dy_perm bf16; pos, topk_gate as written by the forward. */
+MOE_API int moe_combine_backward(const void* dout, const void* y_perm, const int32_t* pos,
+                                 const float* topk_gate, int T, int d, int top_k, void* dy_perm,
+                                 float* dgate, moe_stream_t stream);
+
+/* moe_expert_down_backward: per group g, dh = dy W2_g ([rows, d] x [d, inter])
+ * and the SwiGLU backward with the saved ac: da = dh * c * silu'(a),
+ * dc = dh * silu(a), written as dac [rows, 2*inter] in ac's column order. */
+MOE_API int moe_expert_down_backward(const void* dy, const void* ac, const int32_t* group_offsets,
+                                     int G, int rows, int d, int inter, const void* w2, void* dac,
+                                     moe_stream_t stream);
+
+/* moe_expert_up_backward: per group g, dx = dac W13_g ([rows, 2*inter] x
+ * [2*inter, d], the packed w13 of the forward), dx [rows, d] bf16. */
+MOE_API int moe_expert_up_backward(const void* dac, const int32_t* group_offsets, int G,
+                                   int rows, int d, int inter, const void* w13, void* dx,
+                                   moe_stream_t stream);
+
+/* moe_expert_wgrad: per group g, dw[g] = a[rows of g]^T b[rows of g], the
+ * contraction over the group's rows; a [rows, m], b [rows, n] bf16, dw
+ * [G, m, n] bf16 (overwritten; zero for a group without rows). m % 128 == 0,
+ * n % 128 == 0. dW2 = moe_expert_wgrad(dy, h, m = d, n = inter); the packed
+ * dW13 = moe_expert_wgrad(dac, x, m = 2*inter, n = d). Rows of a and b
+ * outside every group but below `rows` must hold finite values. */
+MOE_API int moe_expert_wgrad(const void* a, const void* b, const int32_t* group_offsets, int G,
+                             int rows, int m, int n, void* dw, moe_stream_t stream);
+
+/* moe_gate_backward: dL/dz of each selected logit z_{t,idx} = u_t . e_idx
+ * from dgate. Sigmoid gate (g_k = S s_k / sum_j s_j, s = Sigmoid(z)
+ * recomputed here from u and the centroids): dz_k = S/sum (dg_k - sum_j dg_j
+ * s_j / sum) s_k (1 - s_k). Softmax gate (g = S softmax of the selected z):
+ * dz_k = g_k (dg_k - sum_j g_j dg_j / S). dz fp32 [T, top_k]; dz_perm fp32
+ * [T*top_k] receives dz[t,k] at row pos[t,k]. */
+MOE_API int moe_gate_backward(const void* u, const void* centroids, const int32_t* topk_idx,
+                              const float* topk_gate, const float* dgate, const int32_t* pos,
+                              int T, int d, int n_routed, int top_k, moe_gate_kind kind,
+                              float routed_scale, float* dz, float* dz_perm,
+                              moe_stream_t stream);
+
+/* moe_combine_dx: du_t = dout_t (residual; dout may be NULL for the form
+ * without it) + dx_shared_t (may be NULL) + sum_k dx_perm[pos[t,k]]
+ * + sum_k dz[t,k] e_{topk_idx[t,k]}, bf16 [T, d]. */
+MOE_API int moe_combine_dx(const void* dout, const void* dx_perm, const int32_t* pos,
+                           const void* dx_shared, const float* dz, const int32_t* topk_idx,
+                           const void* centroids, int T, int d, int top_k, void* du,
+                           moe_stream_t stream);
+
+/* moe_centroid_grad: de_i = sum over the rows r of expert i of dz_perm[r] *
+ * x_perm[r] (x_perm row r = u of the token routed there), bf16 [n_routed, d]. */
+MOE_API int moe_centroid_grad(const void* x_perm, const float* dz_perm,
+                              const int32_t* expert_offsets, int n_routed, int rows, int d,
+                              void* de, moe_stream_t stream);
 
 /* ------------------------------------------------------------------ helpers
  * moe_pack_w13: build the interleaved w13 [G, 2*inter, d] from w1 and w3

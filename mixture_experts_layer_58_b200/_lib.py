@@ -70,6 +70,15 @@ _SIGS = {
     "moe_get_device_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i]),
     "moe_version": (_i, []),
     "moe_selftest_wait_timeout": (_i, [_i, _vp]),
+    "moe_expert_up_swiglu_train": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_combine_backward": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_expert_down_backward": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_expert_up_backward": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_expert_wgrad": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
+    "moe_gate_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp,
+                               _vp]),
+    "moe_combine_dx": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_centroid_grad": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
 }
 
 _LIB = None
@@ -243,6 +252,54 @@ def moe_get_device_status(clear: bool = True) -> int:
 
 def moe_selftest_wait_timeout(limit_ms: int, stream=None):
     _check(_L().moe_selftest_wait_timeout(limit_ms, _stream(stream)), "moe_selftest_wait_timeout")
+
+
+def moe_expert_up_swiglu_train(x, group_offsets, G, rows, d, inter, w13, h, ac, stream=None):
+    _check(_L().moe_expert_up_swiglu_train(_p(x), _p(group_offsets), G, rows, d, inter, _p(w13),
+                                           _p(h), _p(ac), _stream(stream)),
+           "moe_expert_up_swiglu_train")
+
+
+def moe_combine_backward(dout, y_perm, pos, topk_gate, T, d, top_k, dy_perm, dgate, stream=None):
+    _check(_L().moe_combine_backward(_p(dout), _p(y_perm), _p(pos), _p(topk_gate), T, d, top_k,
+                                     _p(dy_perm), _p(dgate), _stream(stream)),
+           "moe_combine_backward")
+
+
+def moe_expert_down_backward(dy, ac, group_offsets, G, rows, d, inter, w2, dac, stream=None):
+    _check(_L().moe_expert_down_backward(_p(dy), _p(ac), _p(group_offsets), G, rows, d, inter,
+                                         _p(w2), _p(dac), _stream(stream)),
+           "moe_expert_down_backward")
+
+
+def moe_expert_up_backward(dac, group_offsets, G, rows, d, inter, w13, dx, stream=None):
+    _check(_L().moe_expert_up_backward(_p(dac), _p(group_offsets), G, rows, d, inter, _p(w13),
+                                       _p(dx), _stream(stream)), "moe_expert_up_backward")
+
+
+def moe_expert_wgrad(a, b, group_offsets, G, rows, m, n, dw, stream=None):
+    _check(_L().moe_expert_wgrad(_p(a), _p(b), _p(group_offsets), G, rows, m, n, _p(dw),
+                                 _stream(stream)), "moe_expert_wgrad")
+
+
+def moe_gate_backward(u, centroids, topk_idx, topk_gate, dgate, pos, T, d, n_routed, top_k, kind,
+                      routed_scale, dz, dz_perm, stream=None):
+    k = GATE_KINDS.get(kind, kind)
+    _check(_L().moe_gate_backward(_p(u), _p(centroids), _p(topk_idx), _p(topk_gate), _p(dgate),
+                                  _p(pos), T, d, n_routed, top_k, k, float(routed_scale), _p(dz),
+                                  _p(dz_perm), _stream(stream)), "moe_gate_backward")
+
+
+def moe_combine_dx(dout, dx_perm, pos, dx_shared, dz, topk_idx, centroids, T, d, top_k, du,
+                   stream=None):
+    _check(_L().moe_combine_dx(_p(dout), _p(dx_perm), _p(pos), _p(dx_shared), _p(dz),
+                               _p(topk_idx), _p(centroids), T, d, top_k, _p(du), _stream(stream)),
+           "moe_combine_dx")
+
+
+def moe_centroid_grad(x_perm, dz_perm, expert_offsets, n_routed, rows, d, de, stream=None):
+    _check(_L().moe_centroid_grad(_p(x_perm), _p(dz_perm), _p(expert_offsets), n_routed, rows, d,
+                                  _p(de), _stream(stream)), "moe_centroid_grad")
 
 
 def moe_strerror(status: int) -> str:

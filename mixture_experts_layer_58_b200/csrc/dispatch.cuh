@@ -218,8 +218,11 @@ __global__ void bias_update_kernel(const int32_t* __restrict__ counts, float* __
 }
 
 // ---------------------------------------------------------------- w13 packing
-// w13[g][256*c + r]       = w1[g][128*c + r]   (r < 128)
-// w13[g][256*c + 128 + r] = w3[g][128*c + r]
+// w13[g][32*c + r]      = w1[g][16*c + r]   (r < 16)
+// w13[g][32*c + 16 + r] = w3[g][16*c + r]
+// 16-row chunks: a 32-column slice of a GEMM accumulator then holds the gate
+// and up products of the same 16 h columns, and so do the 32 TMEM lanes of one
+// warp when the weights are the MMA's M side.
 __global__ void pack_w13_kernel(const __nv_bfloat16* __restrict__ w1,
                                 const __nv_bfloat16* __restrict__ w3, int G, int inter, int d,
                                 __nv_bfloat16* __restrict__ w13) {
@@ -231,10 +234,10 @@ __global__ void pack_w13_kernel(const __nv_bfloat16* __restrict__ w1,
     const size_t r = i / nvec_row;
     const size_t g = r / (2 * static_cast<size_t>(inter));
     const int row13 = static_cast<int>(r - g * 2 * inter);
-    const int c = row13 >> 8;
-    const int within = row13 & 255;
-    const __nv_bfloat16* srcm = within < 128 ? w1 : w3;
-    const size_t srow = g * inter + c * 128 + (within & 127);
+    const int c = row13 >> 5;
+    const int within = row13 & 31;
+    const __nv_bfloat16* srcm = within < 16 ? w1 : w3;
+    const size_t srow = g * inter + c * 16 + (within & 15);
     reinterpret_cast<uint4*>(w13)[i] = __ldg(reinterpret_cast<const uint4*>(srcm + srow * d) + v);
   }
 }

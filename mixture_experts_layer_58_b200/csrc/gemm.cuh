@@ -71,7 +71,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
                          const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
                          int rows, __nv_bfloat16* __restrict__ out, int ldo,
-                         unsigned int* status) {
+                         __nv_bfloat16* __restrict__ ac, unsigned int* status) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -230,26 +230,44 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       const bool valid = grow < row_end;
       const uint32_t taddr = tmem_base + acc * BN + lane_addr;
       if constexpr (EPI == EPI_SWIGLU) {
-        // accumulator columns [0,128) = x.W1 rows, [128,256) = x.W3 rows of the
-        // same 128 h columns
-        static_assert(BN == 256, "SwiGLU epilogue pairs 128 gate with 128 up columns");
+        // W1/W3 rows interleaved in 16-row chunks: accumulator columns
+        // [32q, 32q+16) = x.W1 and [32q+16, 32q+32) = x.W3 of h columns
+        // n_blk*128 + 16q + [0, 16)
+        static_assert(BN == 256, "SwiGLU epilogue: 256 accumulator columns -> 128 h columns");
         __nv_bfloat16* dst_row = out + static_cast<size_t>(grow) * ldo + n_blk * 128;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t ga[32], up[32];
-          tmem_ld_32cols(taddr + c, ga);
-          tmem_ld_32cols(taddr + 128 + c, up);
+        for (int c = 0; c < BN; c += 64) {
+          uint32_t x0[32], x1[32];
+          tmem_ld_32cols(taddr + c, x0);
+          tmem_ld_32cols(taddr + c + 32, x1);
           tmem_ld_wait();
+          if (valid && ac != nullptr) {
+            // training: keep the 64 pre-activations [rows, 2 * ldo], packed W13 order
+            uint32_t raw[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              raw[i] = pack_bf16x2(__uint_as_float(x0[2 * i]), __uint_as_float(x0[2 * i + 1]));
+              raw[16 + i] =
+                  pack_bf16x2(__uint_as_float(x1[2 * i]), __uint_as_float(x1[2 * i + 1]));
+            }
+            uint4* dst = reinterpret_cast<uint4*>(ac + static_cast<size_t>(grow) * (2 * ldo) +
+                                                  n_blk * BN + c);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_uint4(raw[4 * v], raw[4 * v + 1], raw[4 * v + 2], raw[4 * v + 3]);
+          }
           if (valid) {
             uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f32(__uint_as_float(ga[2 * i])) * __uint_as_float(up[2 * i]);
-              const float h1 =
-                  silu_f32(__uint_as_float(ga[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
-              pk[i] = pack_bf16x2(h0, h1);
+            for (int i = 0; i < 8; ++i) {
+              pk[i] = pack_bf16x2(
+                  silu_f32(__uint_as_float(x0[2 * i])) * __uint_as_float(x0[16 + 2 * i]),
+                  silu_f32(__uint_as_float(x0[2 * i + 1])) * __uint_as_float(x0[17 + 2 * i]));
+              pk[8 + i] = pack_bf16x2(
+                  silu_f32(__uint_as_float(x1[2 * i])) * __uint_as_float(x1[16 + 2 * i]),
+                  silu_f32(__uint_as_float(x1[2 * i + 1])) * __uint_as_float(x1[17 + 2 * i]));
             }
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c / 2);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);

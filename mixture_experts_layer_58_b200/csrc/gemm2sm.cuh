@@ -1,14 +1,28 @@
-// Grouped bf16 GEMM on CTA pairs: tcgen05.mma.cta_group::2, 256 x 256 tiles.
+// Grouped bf16 GEMM on CTA pairs: tcgen05.mma.cta_group::2 with the weights as
+// the MMA's M side (256 weight rows) and a group's token rows as its N side.
 //
 // The 1-CTA kernel (gemm.cuh) moves 48 KB from L2 into one SM per 128 x 256 x 64
 // step, and the L2->SM crossbar, not the tensor cores, sets its speed. Here two
-// CTAs of a cluster share one M = 256, N = 256 MMA: CTA r (r = 0 leader, 1 peer)
-// loads rows [128r, 128r+128) of the A tile and rows [128r, 128r+128) of the
-// B (weight) tile into its own shared memory, the leader issues the MMA, and
-// the hardware reads A and B halves from both CTAs. Each SM so loads 32 KB per
-// step for the same flops (a third less crossbar traffic) and the ring holds
-// 6 stages. Each CTA's TMEM receives its own 128 rows x 256 columns of the
-// accumulator (double-buffered: 2 x 256 columns).
+// CTAs of a cluster share one M = 256 MMA: CTA r (r = 0 leader, 1 peer) loads
+// weight rows [128r, 128r+128) of the tile's 256 and half of its token rows
+// into its own shared memory, the leader issues the MMA, and the hardware reads
+// both halves from both CTAs. Each SM so loads 32 KB per step for the flops of
+// a 128 x 256 x 64 step (a third less crossbar traffic) and the ring holds 6
+// stages.
+//
+// Why weights as M: a group's rows come in tiles of 256, and its last tile
+// holds 1..256 of them. With tokens as N that tile's MMA is N = its row count
+// rounded up to 32, and a narrow MMA costs less tensor time than a full one
+// (measured: about 107 clocks at N = 128 against 171 at N = 256 per K = 16
+// step and SM), so a ragged tail no longer costs a full 256-row tile.
+//
+// TMEM: each CTA receives its 128 weight rows (lanes) x N token columns of the
+// accumulator, double-buffered (2 x 256 columns). The epilogue transposes
+// through shared memory: 32 token columns at a time, each warp's 32 lanes are
+// written into a [32 tokens][features] bf16 tile, then the 4 epilogue warps
+// store whole token rows with 16-byte vectors. With W1/W3 interleaved in
+// 16-row chunks, lanes l and l+16 of a warp hold the gate and up products of
+// the same h column, paired with one shuffle.
 //
 // Synchronisation (all waits bounded; no TMA multicast):
 //   full[s]   leader only. Expects 64 KB per phase: the leader's arrive.expect_tx
@@ -17,9 +31,10 @@
 //             peer's (mapa address) when the stage has been read.
 //   tfull[a]  both CTAs; committed like empty at the end of a tile.
 //   tempty[a] leader only; lane 0 of each of the 8 epilogue warps (both CTAs)
-//             arrives once it has drained its TMEM rows (release.cluster).
-// Tiles are (group, 256-row block, 256-column block); a group's last block
-// may hold fewer than 256 valid rows (stores are masked).
+//             arrives once it has drained its TMEM columns (release.cluster).
+// Tiles are (group, 256-token block, 256-weight-row block); token columns past
+// the group's end are computed on whatever rows the loads fetched and never
+// stored.
 #pragma once
 #include "gemm.cuh"
 
@@ -29,15 +44,24 @@ constexpr int kStages2 = 6;
 constexpr int kBM2 = 256;        // rows per CTA-pair tile (128 per CTA)
 
 struct Gemm2smCfg {
-  static constexpr int kABytes = 128 * kBK * 2;   // this CTA's 128 rows of A
-  static constexpr int kBBytes = 128 * kBK * 2;   // this CTA's 128 rows of B
+  static constexpr int kABytes = 128 * kBK * 2;   // token rows (up to 128 of this CTA's half)
+  static constexpr int kBBytes = 128 * kBK * 2;   // this CTA's 128 weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kXBytes = 2 * 32 * 128 * 2;   // epilogue transpose, double-buffered
   static constexpr int kBarBytes = 256;
   static size_t smem_bytes(int G) {
-    return 1024 + static_cast<size_t>(kStages2) * kStageBytes + kBarBytes +
+    return 1024 + static_cast<size_t>(kStages2) * kStageBytes + kXBytes + kBarBytes +
            3 * static_cast<size_t>(G + 1) * sizeof(int);
   }
 };
+
+// Token columns of a pair tile whose first row leaves `rows_left` (> 0) rows
+// in its group: at most 256, rounded up to a multiple of 32 (the MMA's N; each
+// CTA supplies half).
+__device__ __forceinline__ int pair_tile_cols(int rows_left) {
+  const int n = rows_left < kBM2 ? rows_left : kBM2;
+  return (n + 31) & ~31;
+}
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -147,6 +171,55 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+// Dynamic tile order. The leader's producer takes the next tile index from a
+// global counter (zeroed before the launch) and publishes it, through a ring
+// of kTileQ slots, to the 10 other roles that walk the same tiles: the peer's
+// producer, the leader's MMA thread and the 4 epilogue warps of each CTA.
+// Tiles cost different amounts (a group's last tile is a narrower MMA), so a
+// fixed round-robin split would leave some pairs idle while others still work
+// through full tiles; taking tiles in index order also keeps the pairs that
+// share a weight tile close together in time, while it is still in L2.
+constexpr int kTileQ = 4;
+constexpr int kTileQConsumers = 10;
+
+__device__ __forceinline__ void st_shared_cluster_s32(uint32_t addr, int v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Leader producer: wait until slot i % kTileQ is free, then publish t in both CTAs.
+__device__ __forceinline__ bool tile_q_push(int i, int t, int* tq, uint64_t* tq_full,
+                                            uint64_t* tq_empty, unsigned int* status) {
+  const int j = i & (kTileQ - 1);
+  if (!mbar_wait_cluster(&tq_empty[j], ((i / kTileQ) & 1) ^ 1u, status, kStatusTimeoutProducer))
+    return false;
+  tq[j] = t;
+  st_shared_cluster_s32(mapa_shared(smem_u32(&tq[j]), 1), t);
+  mbar_arrive(&tq_full[j]);
+  mbar_arrive_cluster(mapa_shared(smem_u32(&tq_full[j]), 1));
+  return true;
+}
+
+// Any other role (one thread): the i-th published tile index of this CTA's ring.
+__device__ __forceinline__ bool tile_q_pop(int i, const int* tq, uint64_t* tq_full,
+                                           uint64_t* tq_empty, int& t, unsigned int* status,
+                                           unsigned int code) {
+  const int j = i & (kTileQ - 1);
+  if (!mbar_wait_cluster(&tq_full[j], (i / kTileQ) & 1, status, code)) return false;
+  t = *reinterpret_cast<const volatile int*>(&tq[j]);
+  mbar_arrive_cluster(mapa_shared(smem_u32(&tq_empty[j]), 0));
+  return true;
+}
+
+// The 4 epilogue warps of a CTA meet between writing and reading a transpose
+// buffer: lane 0 of each arrives once its warp's writes are done (the
+// mbarrier's release/acquire orders them), and every lane waits, bounded.
+__device__ __forceinline__ bool xfer_sync(uint64_t* bar, uint32_t parity, int lane,
+                                          unsigned int* status) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  return mbar_wait(bar, parity, status, kStatusTimeoutEpilogue);
+}
+
 // tile index -> (group, 256-row block, n block); row blocks fastest in a group.
 __device__ __forceinline__ void decode_tile_pair(int t, const int* s_tstart, const int* s_off,
                                                  const int* s_end, int G, int& g, int& m_blk,
@@ -172,19 +245,26 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                               const __grid_constant__ CUtensorMap tmB,
                               const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
                               int rows, __nv_bfloat16* __restrict__ out, int ldo,
-                              const int32_t* __restrict__ src_rows, unsigned int* status) {
+                              __nv_bfloat16* __restrict__ ac,
+                              const int32_t* __restrict__ src_rows, int* tile_counter,
+                              unsigned int* status) {
   constexpr int BN = 256;
   using C = Gemm2smCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages2 * C::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages2 * C::kBBytes);
+  __nv_bfloat16* sX = reinterpret_cast<__nv_bfloat16*>(sB + kStages2 * C::kBBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sX) + C::kXBytes);
   uint64_t* empty = full + kStages2;
   uint64_t* tfull = empty + kStages2;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* xready = mma_done + 1;   // [2]: the 4 epilogue warps filled sX half i
+  uint64_t* tq_full = xready + 2;    // [kTileQ]
+  uint64_t* tq_empty = tq_full + kTileQ;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kTileQ);
+  int* tq = reinterpret_cast<int*>(tmem_slot + 1);   // [kTileQ] tile indices
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_tstart = s_off + (G + 1);
   int* s_end = s_tstart + (G + 1);
@@ -192,8 +272,6 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1;
-  const int npairs = gridDim.x >> 1;
   const int n_blocks_n = n_per_group / BN;
   const int num_kb = K / kBK;
 
@@ -208,6 +286,12 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         mbar_init(&tempty[a], 8);
       }
       mbar_init(mma_done, 1);
+      mbar_init(&xready[0], 4);
+      mbar_init(&xready[1], 4);
+      for (int j = 0; j < kTileQ; ++j) {
+        mbar_init(&tq_full[j], 1);
+        mbar_init(&tq_empty[j], kTileQConsumers);
+      }
       fence_mbar_init();
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
@@ -257,10 +341,29 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t phase = 0;
     uint32_t issued = 0, issued_par = 0;
     bool ok = true;
-    for (int t = pair; t < total_tiles && ok; t += npairs) {
+    int t_next = 0;
+    if (rank == 0 && lane == 0) t_next = atomicAdd(tile_counter, 1);
+    for (int i = 0; ok; ++i) {
+      int t = total_tiles;
+      if (lane == 0) {
+        if (rank == 0) {
+          t = min(t_next, total_tiles);
+          ok = tile_q_push(i, t, tq, tq_full, tq_empty, status);
+          if (ok && t < total_tiles) t_next = atomicAdd(tile_counter, 1);
+        } else {
+          ok = tile_q_pop(i, tq, tq_full, tq_empty, t, status, kStatusTimeoutProducer);
+        }
+      }
+      if constexpr (GATHER) {
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        t = __shfl_sync(0xffffffffu, t, 0);
+      }
+      if (!ok || t >= total_tiles) break;
       int g, m_blk, n_blk;
       decode_tile_pair(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
-      const int a_row = s_off[g] + m_blk * kBM2 + static_cast<int>(rank) * 128;
+      const int row0 = s_off[g] + m_blk * kBM2;
+      const int ncols = pair_tile_cols(s_end[g] - row0);
+      const int a_row = row0 + static_cast<int>(rank) * (ncols >> 1);
       const int b_row = g * n_per_group + n_blk * BN + static_cast<int>(rank) * 128;
       int src[4] = {0, 0, 0, 0};
       if constexpr (GATHER) {
@@ -306,12 +409,18 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           mbar_wait(&full[s], (issued_par >> s) & 1u, status, kStatusTimeoutProducer);
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------------ MMA issuer (leader)
-    constexpr uint32_t idesc = idesc_bf16_f32(kBM2, BN);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    int local = 0;
-    for (int t = pair; t < total_tiles && ok; t += npairs, ++local) {
+    for (int local = 0; ok; ++local) {
+      int t;
+      if (!tile_q_pop(local, tq, tq_full, tq_empty, t, status, kStatusTimeoutMma) ||
+          t >= total_tiles)
+        break;
+      int g, m_blk, n_blk;
+      decode_tile_pair(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
+      const int ncols = pair_tile_cols(s_end[g] - (s_off[g] + m_blk * kBM2));
+      const uint32_t idesc = idesc_bf16_f32(kBM2, ncols);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       if (!mbar_wait_cluster(&tempty[acc], acc_par ^ 1u, status, kStatusTimeoutMma)) break;
@@ -323,11 +432,12 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           break;
         }
         tc_fence_after();
-        const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * C::kABytes));
-        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * C::kBBytes));
+        // MMA A operand = the weight rows (sB), B operand = the token rows (sA)
+        const uint64_t wdesc = sw128_kmajor_desc(smem_u32(sB + stage * C::kBBytes));
+        const uint64_t xdesc = sw128_kmajor_desc(smem_u32(sA + stage * C::kABytes));
 #pragma unroll
         for (int k = 0; k < kBK / kUmmaK; ++k)
-          umma_bf16_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+          umma_bf16_pair(d_tmem, wdesc + 2u * k, xdesc + 2u * k, idesc, (kb | k) != 0);
         const uint32_t e = smem_u32(&empty[stage]);
         umma_commit_pair(mapa_shared(e, 0));
         umma_commit_pair(mapa_shared(e, 1));
@@ -347,64 +457,96 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;
-    const int row_in_half = quarter * 32 + lane;
+    const int et = (warp - 2) * 32 + lane;   // 0..127 across the 4 epilogue warps
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-    int local = 0;
-    for (int t = pair; t < total_tiles; t += npairs, ++local) {
+    int chunk = 0;   // running count of 32-column chunks: selects the sX half
+    for (int local = 0;; ++local) {
+      int t = total_tiles;
+      bool got = true;
+      if (lane == 0)
+        got = tile_q_pop(local, tq, tq_full, tq_empty, t, status, kStatusTimeoutEpilogue);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (!got || t >= total_tiles) break;
       int g, m_blk, n_blk;
       decode_tile_pair(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
+      const int row0 = s_off[g] + m_blk * kBM2;
+      const int ncols = pair_tile_cols(s_end[g] - row0);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_par, status, kStatusTimeoutEpilogue)) break;
       tc_fence_after();
-      const int grow = s_off[g] + m_blk * kBM2 + static_cast<int>(rank) * 128 + row_in_half;
       const int row_end = min(s_end[g], rows);
-      const bool valid = grow >= 0 && grow < row_end;
       const uint32_t taddr = tmem_base + acc * BN + lane_addr;
-      if constexpr (EPI == EPI_SWIGLU) {
-        __nv_bfloat16* dst_row = out + static_cast<size_t>(grow) * ldo + n_blk * 128;
+      bool ok = true;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t ga[32], up[32];
-          tmem_ld_32cols(taddr + c, ga);
-          tmem_ld_32cols(taddr + 128 + c, up);
-          tmem_ld_wait();
-          if (valid) {
-            uint32_t pk[16];
+      for (int j0 = 0; j0 < ncols; j0 += 32, ++chunk) {
+        ok = false;
+        uint32_t v[32];
+        tmem_ld_32cols(taddr + j0, v);
+        tmem_ld_wait();
+        __nv_bfloat16* X = sX + (chunk & 1) * (32 * 128);
+        if constexpr (EPI == EPI_SWIGLU) {
+          // lane l < 16: gate product of h column (l & 15) of this warp's 16;
+          // lane l + 16: its up product. Lanes < 16 finish tokens 0..15 of the
+          // chunk, lanes >= 16 tokens 16..31. X = [32 tokens][64 h columns].
+          if (ac != nullptr) {
+            // training: keep the pre-activations, [rows, 2 * ldo] in the
+            // packed W13 column order (this lane's weight row = its column)
+            __nv_bfloat16* acol =
+                ac + n_blk * BN + static_cast<int>(rank) * 128 + quarter * 32 + lane;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f32(__uint_as_float(ga[2 * i])) * __uint_as_float(up[2 * i]);
-              const float h1 =
-                  silu_f32(__uint_as_float(ga[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
-              pk[i] = pack_bf16x2(h0, h1);
+            for (int i = 0; i < 32; ++i) {
+              const int grow = row0 + j0 + i;
+              if (grow < row_end)
+                acol[static_cast<size_t>(grow) * (2 * ldo)] =
+                    __float2bfloat16_rn(__uint_as_float(v[i]));
             }
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
+          }
+          const bool lo = lane < 16;
+          const int hc = quarter * 16 + (lane & 15);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t own = lo ? v[i] : v[i + 16];
+            const uint32_t send = lo ? v[i + 16] : v[i];
+            const uint32_t other = __shfl_xor_sync(0xffffffffu, send, 16);
+            const float a = __uint_as_float(lo ? own : other);
+            const float b = __uint_as_float(lo ? other : own);
+            X[(i + (lo ? 0 : 16)) * 64 + hc] = __float2bfloat16_rn(silu_f32(a) * b);
+          }
+          if (!xfer_sync(&xready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
+          __nv_bfloat16* dst0 = out + n_blk * 128 + static_cast<int>(rank) * 64;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int idx = et + 128 * k;
+            const int r = idx >> 3, seg = idx & 7;
+            const int grow = row0 + j0 + r;
+            if (grow < row_end)
+              *reinterpret_cast<uint4*>(dst0 + static_cast<size_t>(grow) * ldo + seg * 8) =
+                  *reinterpret_cast<const uint4*>(X + r * 64 + seg * 8);
+          }
+        } else {
+          // X = [32 tokens][128 output features of this CTA]
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            X[i * 128 + quarter * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+          if (!xfer_sync(&xready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
+          __nv_bfloat16* dst0 = out + n_blk * BN + static_cast<int>(rank) * 128;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int idx = et + 128 * k;
+            const int r = idx >> 4, seg = idx & 15;
+            const int grow = row0 + j0 + r;
+            if (grow < row_end)
+              *reinterpret_cast<uint4*>(dst0 + static_cast<size_t>(grow) * ldo + seg * 8) =
+                  *reinterpret_cast<const uint4*>(X + r * 128 + seg * 8);
           }
         }
-      } else {
-        __nv_bfloat16* dst_row = out + static_cast<size_t>(grow) * ldo + n_blk * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32cols(taddr + c, r);
-          tmem_ld_wait();
-          if (valid) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          }
-        }
+        ok = true;
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);

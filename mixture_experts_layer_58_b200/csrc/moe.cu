@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "moe.h"
@@ -18,12 +19,19 @@
 #include "gemm2sm.cuh"
 #include "gemm_fp8.cuh"
 #include "route.cuh"
+#include "bwd.cuh"
+#include "gemm_bwd.cuh"
 
 namespace {
 
 using namespace moe;
 
 __device__ unsigned int g_status;   // per-device status word (see moe_get_device_status)
+
+// Tile counters of the CTA-pair GEMM's dynamic schedule; each launch takes the
+// next slot (round robin) and zeroes it on its stream first.
+constexpr int kTileCounters = 256;
+__device__ int g_tile_counters[kTileCounters];
 
 thread_local int t_last_cuda_error = 0;
 
@@ -33,6 +41,8 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   unsigned int* status = nullptr;
+  int* tile_counters = nullptr;
+  std::atomic<unsigned> next_counter{0};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -66,6 +76,8 @@ int device_info(DeviceInfo** out) {
       void* p = nullptr;
       MOE_CUDA(cudaGetSymbolAddress(&p, g_status));
       di.status = static_cast<unsigned int*>(p);
+      MOE_CUDA(cudaGetSymbolAddress(&p, g_tile_counters));
+      di.tile_counters = static_cast<int*>(p);
       di.ready = true;
     }
   }
@@ -110,6 +122,25 @@ int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
   return MOE_OK;
 }
 
+// 2-D bf16 tensor map for TMA stores of 32 x 32 blocks (no swizzle) into a
+// row-major [rows, cols] matrix.
+int make_tmap_bf16_store32(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
+  int rc = get_encoder();
+  if (rc != MOE_OK) return rc;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 template <typename K>
 int set_smem(K kernel, size_t bytes) {
   MOE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -122,7 +153,8 @@ inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStre
 // ------------------------------------------------------------------ GEMM launch
 template <int BN, int EPI>
 int launch_grouped_gemm(const void* A, int rows, int K, const void* B, int G, int n_per_group,
-                        const int32_t* offsets, void* out, int ldo, cudaStream_t st) {
+                        const int32_t* offsets, void* out, int ldo, cudaStream_t st,
+                        void* ac = nullptr) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
@@ -137,7 +169,8 @@ int launch_grouped_gemm(const void* A, int rows, int K, const void* B, int G, in
       (static_cast<long long>(rows) / kBM + G) * static_cast<long long>(n_per_group / BN);
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
   kern<<<grid, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
-                                         static_cast<__nv_bfloat16*>(out), ldo, di->status);
+                                         static_cast<__nv_bfloat16*>(out), ldo,
+                                         static_cast<__nv_bfloat16*>(ac), di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -195,7 +228,7 @@ template <int EPI>
 int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int G,
                              int n_per_group, const int32_t* offsets, void* out, int ldo,
                              cudaStream_t st, const int32_t* src_rows = nullptr,
-                             int a_rows = 0) {
+                             int a_rows = 0, void* ac = nullptr) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
@@ -211,19 +244,68 @@ int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int 
   const long long max_tiles =
       (static_cast<long long>(rows) / kBM2 + G) * static_cast<long long>(n_per_group / 256);
   const int pairs = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms / 2, max_tiles)));
+  int* counter = di->tile_counters + (di->next_counter.fetch_add(1) % kTileCounters);
+  MOE_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   if (src_rows) {
     auto kern = grouped_gemm_bf16_pair_kernel<EPI, true>;
     if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
     kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
-                                                 static_cast<__nv_bfloat16*>(out), ldo, src_rows,
-                                                 di->status);
+                                                 static_cast<__nv_bfloat16*>(out), ldo,
+                                                 static_cast<__nv_bfloat16*>(ac), src_rows,
+                                                 counter, di->status);
   } else {
     auto kern = grouped_gemm_bf16_pair_kernel<EPI, false>;
     if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
     kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
-                                                 static_cast<__nv_bfloat16*>(out), ldo, nullptr,
-                                                 di->status);
+                                                 static_cast<__nv_bfloat16*>(out), ldo,
+                                                 static_cast<__nv_bfloat16*>(ac), nullptr,
+                                                 counter, di->status);
   }
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// dgrad: out[rows of g] = A[rows of g] (K-major, [rows, K]) * W_g ([K, N] row-major).
+template <int EPI>
+int launch_dgrad(const void* A, int rows, int K, const void* W, int G, int N,
+                 const int32_t* offsets, void* out, int ldo, const void* ac, cudaStream_t st) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  CUtensorMap tmA, tmW;
+  if ((rc = make_tmap_bf16(&tmA, A, K, rows, kBM)) != MOE_OK) return rc;
+  if ((rc = make_tmap_bf16(&tmW, W, N, static_cast<uint64_t>(G) * K, 64)) != MOE_OK) return rc;
+  const size_t smem = BwdCfg::smem_bytes(G);
+  auto kern = grouped_dgrad_bf16_kernel<EPI>;
+  if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
+  const long long max_tiles = (static_cast<long long>(rows) / kBM + G) *
+                              static_cast<long long>((N + BwdCfg::kBN - 1) / BwdCfg::kBN);
+  const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
+  kern<<<grid, kGemmThreads, smem, st>>>(tmA, tmW, offsets, G, K, N, rows,
+                                         static_cast<__nv_bfloat16*>(out), ldo,
+                                         static_cast<const __nv_bfloat16*>(ac), di->status);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// wgrad: dw[g] = A[rows of g]^T B[rows of g]; A [rows, M], B [rows, N], dw [G, M, N].
+int launch_wgrad(const void* A, const void* B, int rows, int M, int N, int G,
+                 const int32_t* offsets, void* dw, cudaStream_t st) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  CUtensorMap tmA, tmB, tmD;
+  if ((rc = make_tmap_bf16(&tmA, A, M, rows, 64)) != MOE_OK) return rc;
+  if ((rc = make_tmap_bf16(&tmB, B, N, rows, 64)) != MOE_OK) return rc;
+  if ((rc = make_tmap_bf16_store32(&tmD, dw, N, static_cast<uint64_t>(G) * M)) != MOE_OK)
+    return rc;
+  const size_t smem = BwdCfg::wgrad_smem_bytes(G);
+  if ((rc = set_smem(grouped_wgrad_bf16_kernel, smem)) != MOE_OK) return rc;
+  const long long tiles = static_cast<long long>(G) * (M / kBM) *
+                          ((N + BwdCfg::kBN - 1) / BwdCfg::kBN);
+  const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, tiles)));
+  grouped_wgrad_bf16_kernel<<<grid, kGemmThreads, smem, st>>>(tmA, tmB, tmD, offsets, G, M, N,
+                                                               rows, di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -660,6 +742,174 @@ int moe_bias_update(const int32_t* expert_counts, float* bias, int n_routed, lon
   if (!(gamma == gamma)) return MOE_ERR_INVALID_ARG;
   bias_update_kernel<<<(n_routed + 255) / 256, 256, 0, as_stream(stream)>>>(
       expert_counts, bias, n_routed, T * top_k, gamma);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ backward
+int moe_expert_up_swiglu_train(const void* x, const int32_t* group_offsets, int G, int rows,
+                               int d, int inter, const void* w13, void* h, void* ac,
+                               moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!x || !group_offsets || !w13 || !h || !ac || !aligned16(x) || !aligned16(w13) ||
+      !aligned16(h) || !aligned16(ac))
+    return MOE_ERR_INVALID_ARG;
+  if (use_pair_tiles(rows, G))
+    return launch_grouped_gemm_pair<EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
+                                                inter, as_stream(stream), nullptr, 0, ac);
+  return launch_grouped_gemm<256, EPI_SWIGLU>(x, rows, d, w13, G, 2 * inter, group_offsets, h,
+                                              inter, as_stream(stream), ac);
+}
+
+int moe_combine_backward(const void* dout, const void* y_perm, const int32_t* pos,
+                         const float* topk_gate, int T, int d, int top_k, void* dy_perm,
+                         float* dgate, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!dout || !y_perm || !pos || !topk_gate || !dy_perm || !dgate || !aligned16(dout) ||
+      !aligned16(y_perm) || !aligned16(dy_perm))
+    return MOE_ERR_INVALID_ARG;
+  const int blocks = (T + kBwdTokensPerBlock - 1) / kBwdTokensPerBlock;
+  const auto* o = static_cast<const __nv_bfloat16*>(dout);
+  const auto* y = static_cast<const __nv_bfloat16*>(y_perm);
+  auto* dy = static_cast<__nv_bfloat16*>(dy_perm);
+  cudaStream_t st = as_stream(stream);
+#define MOE_CB_CASE(KK)                                                                       \
+  case KK:                                                                                    \
+    combine_backward_kernel<KK><<<blocks, 32 * kBwdTokensPerBlock, 0, st>>>(o, y, pos,        \
+                                                                           topk_gate, T, d,   \
+                                                                           dy, dgate);        \
+    break;
+  switch (top_k) {
+    MOE_CB_CASE(1) MOE_CB_CASE(2) MOE_CB_CASE(3) MOE_CB_CASE(4)
+    MOE_CB_CASE(5) MOE_CB_CASE(6) MOE_CB_CASE(7) MOE_CB_CASE(8)
+    default: return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+#undef MOE_CB_CASE
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_expert_down_backward(const void* dy, const void* ac, const int32_t* group_offsets, int G,
+                             int rows, int d, int inter, const void* w2, void* dac,
+                             moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!dy || !ac || !group_offsets || !w2 || !dac || !aligned16(dy) || !aligned16(ac) ||
+      !aligned16(w2) || !aligned16(dac))
+    return MOE_ERR_INVALID_ARG;
+  return launch_dgrad<EPI_DG_SWIGLU_BWD>(dy, rows, d, w2, G, inter, group_offsets, dac,
+                                         2 * inter, ac, as_stream(stream));
+}
+
+int moe_expert_up_backward(const void* dac, const int32_t* group_offsets, int G, int rows, int d,
+                           int inter, const void* w13, void* dx, moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!dac || !group_offsets || !w13 || !dx || !aligned16(dac) || !aligned16(w13) ||
+      !aligned16(dx))
+    return MOE_ERR_INVALID_ARG;
+  return launch_dgrad<EPI_DG_STORE>(dac, rows, 2 * inter, w13, G, d, group_offsets, dx, d,
+                                    nullptr, as_stream(stream));
+}
+
+int moe_expert_wgrad(const void* a, const void* b, const int32_t* group_offsets, int G, int rows,
+                     int m, int n, void* dw, moe_stream_t stream) {
+  if (G < 1 || rows < 0 || m <= 0 || n <= 0) return MOE_ERR_INVALID_ARG;
+  if (G > kMaxGroups || m % 128 != 0 || n % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!group_offsets || !dw || !aligned16(dw)) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && (!a || !b || !aligned16(a) || !aligned16(b))) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) {
+    MOE_CUDA(cudaMemsetAsync(dw, 0, static_cast<size_t>(G) * m * n * 2, as_stream(stream)));
+    return MOE_OK;
+  }
+  return launch_wgrad(a, b, rows, m, n, G, group_offsets, dw, as_stream(stream));
+}
+
+int moe_gate_backward(const void* u, const void* centroids, const int32_t* topk_idx,
+                      const float* topk_gate, const float* dgate, const int32_t* pos, int T,
+                      int d, int n_routed, int top_k, moe_gate_kind kind, float routed_scale,
+                      float* dz, float* dz_perm, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (kind != MOE_GATE_SIGMOID_BIAS && kind != MOE_GATE_SOFTMAX_TOPK) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!(routed_scale == routed_scale) || routed_scale == 0.0f) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!u || !centroids || !topk_idx || !topk_gate || !dgate || !pos || !dz || !dz_perm ||
+      !aligned16(u) || !aligned16(centroids))
+    return MOE_ERR_INVALID_ARG;
+  const int blocks = (T + kBwdTokensPerBlock - 1) / kBwdTokensPerBlock;
+  const auto* uu = static_cast<const __nv_bfloat16*>(u);
+  const auto* ee = static_cast<const __nv_bfloat16*>(centroids);
+  cudaStream_t st = as_stream(stream);
+#define MOE_GB_CASE(KK)                                                                        \
+  case KK:                                                                                     \
+    if (kind == MOE_GATE_SIGMOID_BIAS)                                                         \
+      gate_backward_kernel<KK, 0><<<blocks, 32 * kBwdTokensPerBlock, 0, st>>>(                 \
+          uu, ee, topk_idx, topk_gate, dgate, pos, T, d, routed_scale, dz, dz_perm);           \
+    else                                                                                       \
+      gate_backward_kernel<KK, 1><<<blocks, 32 * kBwdTokensPerBlock, 0, st>>>(                 \
+          uu, ee, topk_idx, topk_gate, dgate, pos, T, d, routed_scale, dz, dz_perm);           \
+    break;
+  switch (top_k) {
+    MOE_GB_CASE(1) MOE_GB_CASE(2) MOE_GB_CASE(3) MOE_GB_CASE(4)
+    MOE_GB_CASE(5) MOE_GB_CASE(6) MOE_GB_CASE(7) MOE_GB_CASE(8)
+    default: return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+#undef MOE_GB_CASE
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_combine_dx(const void* dout, const void* dx_perm, const int32_t* pos,
+                   const void* dx_shared, const float* dz, const int32_t* topk_idx,
+                   const void* centroids, int T, int d, int top_k, void* du,
+                   moe_stream_t stream) {
+  if (T < 0 || d <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!dx_perm || !pos || !dz || !topk_idx || !centroids || !du || !aligned16(dx_perm) ||
+      !aligned16(centroids) || !aligned16(du))
+    return MOE_ERR_INVALID_ARG;
+  if ((dout && !aligned16(dout)) || (dx_shared && !aligned16(dx_shared)))
+    return MOE_ERR_INVALID_ARG;
+  const int blocks = (T + kBwdTokensPerBlock - 1) / kBwdTokensPerBlock;
+  const auto* o = static_cast<const __nv_bfloat16*>(dout);
+  const auto* dxp = static_cast<const __nv_bfloat16*>(dx_perm);
+  const auto* dxs = static_cast<const __nv_bfloat16*>(dx_shared);
+  const auto* ee = static_cast<const __nv_bfloat16*>(centroids);
+  auto* out = static_cast<__nv_bfloat16*>(du);
+  cudaStream_t st = as_stream(stream);
+#define MOE_DX_CASE(KK)                                                                        \
+  case KK:                                                                                     \
+    combine_dx_kernel<KK><<<blocks, 32 * kBwdTokensPerBlock, 0, st>>>(o, dxp, pos, dxs, dz,    \
+                                                                      topk_idx, ee, T, d, out); \
+    break;
+  switch (top_k) {
+    MOE_DX_CASE(1) MOE_DX_CASE(2) MOE_DX_CASE(3) MOE_DX_CASE(4)
+    MOE_DX_CASE(5) MOE_DX_CASE(6) MOE_DX_CASE(7) MOE_DX_CASE(8)
+    default: return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+#undef MOE_DX_CASE
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_centroid_grad(const void* x_perm, const float* dz_perm, const int32_t* expert_offsets,
+                      int n_routed, int rows, int d, void* de, moe_stream_t stream) {
+  if (n_routed <= 0 || rows < 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!expert_offsets || !de || !aligned16(de)) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && (!x_perm || !dz_perm || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  dim3 grid(n_routed, (d + kCentroidCols - 1) / kCentroidCols);
+  centroid_grad_kernel<<<grid, kCentroidCols / 8, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x_perm), dz_perm, expert_offsets, d,
+      static_cast<__nv_bfloat16*>(de));
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

@@ -8,12 +8,45 @@ in libmoe.so's kernels:
     moe_grouped_ffn  routed experts (G = N_r) then the shared expert (G = 1)
     moe_combine      h' = u + shared + sum_k g * y
     moe_bias_update  b -= / += gamma from the loads (end of the step)
+
+Training (bf16): forward(u, train=True) also keeps the SwiGLU pre-activations;
+backward(dout) then runs the backward calls (combine, expert dgrad and
+wgrad, gate, du, centroid gradient) and leaves the weight gradients on the
+layer (grad_w13 in the packed W13 layout, grad_w2, grad_ws13, grad_ws2,
+grad_centroids).
 """
 from __future__ import annotations
 
 import torch
 
 from . import _lib as L
+
+
+class _Timed:
+    """Context manager factory: CUDA events around a call when timers is a dict."""
+
+    def __init__(self, timers):
+        self.timers = timers
+
+    def __call__(self, name):
+        return _TimedCall(self.timers, name)
+
+
+class _TimedCall:
+    def __init__(self, timers, name):
+        self.timers, self.name = timers, name
+
+    def __enter__(self):
+        if self.timers is not None:
+            self.e0 = torch.cuda.Event(enable_timing=True)
+            self.e0.record()
+
+    def __exit__(self, *exc):
+        if self.timers is not None:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record()
+            self.timers.setdefault(self.name, []).append((self.e0, e1))
+        return False
 
 
 class MoELayer:
@@ -189,21 +222,128 @@ class MoELayer:
                       u if residual else None, T, self.d, self.top_k,
                       self.out if out is None else out)
 
-    def forward(self, u, residual: bool = True, out=None):
+    def forward(self, u, residual: bool = True, out=None, train: bool = False):
         """h' for the bf16 batch u [T, d] (device), written to `out` ([T, d]
-        bf16, device) or to the layer's own output buffer, which is returned."""
+        bf16, device) or to the layer's own output buffer, which is returned.
+        train=True (bf16, copy-based dispatch) keeps what backward() needs."""
         assert u.dtype == torch.bfloat16 and u.is_contiguous() and u.device.type == "cuda"
         T = u.shape[0]
         self.allocate(T)
         dst = self.out if out is None else out
         assert dst.shape == (T, self.d) and dst.dtype == torch.bfloat16 and dst.is_contiguous()
+        if train:
+            if self.fp8 or self.fused_gather:
+                raise ValueError("training runs on the bf16 layer with the copy-based dispatch")
+            self._allocate_train(T)
+        self._train_state = (u, residual) if train else None
         self.route(u)
         if T > 0:
             self.permute(u)
-            self.routed_ffn(T, u)
-            self.shared_ffn(u)
+            if train:
+                self._routed_ffn_train(T)
+                self._shared_ffn_train(u)
+            else:
+                self.routed_ffn(T, u)
+                self.shared_ffn(u)
             self.combine(u, residual, dst)
         return dst
+
+    # ------------------------------------------------------------------ training
+    def _allocate_train(self, T: int) -> None:
+        if getattr(self, "_train_T", -1) == T:
+            return
+        dev, K, d, I = self.device, self.top_k, self.d, self.inter
+        rows = T * K
+        bf, f32 = torch.bfloat16, torch.float32
+        self.h = torch.empty((rows, I), dtype=bf, device=dev)
+        self.ac = torch.empty((rows, 2 * I), dtype=bf, device=dev)
+        self.dy_perm = torch.empty((rows, d), dtype=bf, device=dev)
+        self.dac = torch.empty((rows, 2 * I), dtype=bf, device=dev)
+        self.dx_perm = torch.empty((rows, d), dtype=bf, device=dev)
+        self.dgate = torch.empty((T, K), dtype=f32, device=dev)
+        self.dz = torch.empty((T, K), dtype=f32, device=dev)
+        self.dz_perm = torch.empty(rows, dtype=f32, device=dev)
+        self.du = torch.empty((T, d), dtype=bf, device=dev)
+        if self.ws13 is not None:
+            Is = self.shared_inter
+            self.h_s = torch.empty((T, Is), dtype=bf, device=dev)
+            self.ac_s = torch.empty((T, 2 * Is), dtype=bf, device=dev)
+            self.dac_s = torch.empty((T, 2 * Is), dtype=bf, device=dev)
+            self.dx_s = torch.empty((T, d), dtype=bf, device=dev)
+        if getattr(self, "grad_w13", None) is None:
+            self.grad_w13 = torch.empty_like(self.w13)
+            self.grad_w2 = torch.empty_like(self.w2)
+            self.grad_centroids = torch.empty_like(self.centroids)
+            if self.ws13 is not None:
+                self.grad_ws13 = torch.empty_like(self.ws13)
+                self.grad_ws2 = torch.empty_like(self.ws2)
+        self._train_T = T
+
+    def _routed_ffn_train(self, T):
+        rows = T * self.top_k
+        L.moe_expert_up_swiglu_train(self.x_perm, self.offsets, self.n_routed, rows, self.d,
+                                     self.inter, self.w13, self.h, self.ac)
+        L.moe_expert_down(self.h, self.offsets, self.n_routed, rows, self.inter, self.d, self.w2,
+                          self.y_perm)
+
+    def _shared_ffn_train(self, u):
+        if self.ws13 is None:
+            return
+        T = u.shape[0]
+        L.moe_expert_up_swiglu_train(u, self.shared_offsets, 1, T, self.d, self.shared_inter,
+                                     self.ws13, self.h_s, self.ac_s)
+        L.moe_expert_down(self.h_s, self.shared_offsets, 1, T, self.shared_inter, self.d, self.ws2,
+                          self.shared_out)
+
+    def backward(self, dout, timers=None):
+        """Gradients of the last forward(..., train=True) for dL/dh' = dout
+        ([T, d] bf16, device). Returns du [T, d] bf16 (the layer's buffer);
+        the weight gradients are left in grad_w13 (packed like w13), grad_w2,
+        grad_ws13, grad_ws2 and grad_centroids. The bias gets none.
+        timers: optional dict; the routed up-projection dgrad ("dx") and the
+        routed W13 weight gradient ("dw13") each get a (start, end) pair of
+        CUDA events appended to timers[name] on the current stream."""
+        if getattr(self, "_train_state", None) is None:
+            raise RuntimeError("backward() needs a preceding forward(..., train=True)")
+        u, residual = self._train_state
+        T, K, d, I, G = u.shape[0], self.top_k, self.d, self.inter, self.n_routed
+        assert dout.shape == (T, d) and dout.dtype == torch.bfloat16 and dout.is_contiguous()
+        rows = T * K
+        if T == 0:
+            return self.du
+        L.moe_combine_backward(dout, self.y_perm, self.pos, self.topk_gate, T, d, K,
+                               self.dy_perm, self.dgate)
+        L.moe_expert_down_backward(self.dy_perm, self.ac, self.offsets, G, rows, d, I, self.w2,
+                                   self.dac)
+        ev = _Timed(timers)
+        with ev("dx"):
+            L.moe_expert_up_backward(self.dac, self.offsets, G, rows, d, I, self.w13,
+                                     self.dx_perm)
+        L.moe_expert_wgrad(self.dy_perm, self.h, self.offsets, G, rows, d, I, self.grad_w2)
+        with ev("dw13"):
+            L.moe_expert_wgrad(self.dac, self.x_perm, self.offsets, G, rows, 2 * I, d,
+                               self.grad_w13)
+        dx_s = None
+        if self.ws13 is not None:
+            Is = self.shared_inter
+            so = self.shared_offsets
+            L.moe_expert_down_backward(dout, self.ac_s, so, 1, T, d, Is, self.ws2, self.dac_s)
+            L.moe_expert_up_backward(self.dac_s, so, 1, T, d, Is, self.ws13, self.dx_s)
+            L.moe_expert_wgrad(dout, self.h_s, so, 1, T, d, Is, self.grad_ws2)
+            L.moe_expert_wgrad(self.dac_s, u, so, 1, T, 2 * Is, d, self.grad_ws13)
+            dx_s = self.dx_s
+        L.moe_gate_backward(u, self.centroids, self.topk_idx, self.topk_gate, self.dgate, self.pos,
+                            T, d, G, K, self.gate_kind, self.routed_scale, self.dz, self.dz_perm)
+        L.moe_combine_dx(dout if residual else None, self.dx_perm, self.pos, dx_s, self.dz,
+                         self.topk_idx, self.centroids, T, d, K, self.du)
+        L.moe_centroid_grad(self.x_perm, self.dz_perm, self.offsets, G, rows, d,
+                            self.grad_centroids)
+        return self.du
+
+    def launches_per_backward(self) -> int:
+        # combine bwd, down dgrad, up dgrad, 2 wgrad; shared: 4 more; gate bwd,
+        # du, centroid grad
+        return 5 + (4 if self.ws13 is not None else 0) + 3
 
     def update_bias(self, counts=None, T=None):
         """End-of-step bias update from this batch's loads (or from counts

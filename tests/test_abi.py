@@ -187,3 +187,42 @@ def test_fused_gather_entry_points_reject_bad_arguments(lib):
 def test_selftest_rejects_bad_limit(lib):
     assert lib.moe_selftest_wait_timeout(0, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_wait_timeout(20000, None) == L.MOE_ERR_INVALID_ARG
+
+
+def test_backward_entry_points_reject_bad_arguments(lib):
+    E = L.MOE_ERR_INVALID_ARG
+    U = L.MOE_ERR_UNSUPPORTED_SHAPE
+    # training forward: ac is required and aligned
+    assert lib.moe_expert_up_swiglu_train(A, A, 4, 256, 256, 128, A, A, None, None) == E
+    assert lib.moe_expert_up_swiglu_train(A, A, 4, 256, 256, 128, A, A, MIS, None) == E
+    assert lib.moe_expert_up_swiglu_train(A, A, 4, 256, 256, 100, A, A, A, None) == U
+    # combine backward
+    assert lib.moe_combine_backward(A, A, A, A, -1, 256, 4, A, A, None) == E
+    assert lib.moe_combine_backward(A, A, A, A, 64, 256, 9, A, A, None) == U
+    assert lib.moe_combine_backward(A, A, A, A, 64, 256, 4, MIS, A, None) == E
+    assert lib.moe_combine_backward(A, A, A, A, 64, 256, 4, A, None, None) == E
+    # expert dgrad
+    assert lib.moe_expert_down_backward(A, None, A, 4, 256, 256, 128, A, A, None) == E
+    assert lib.moe_expert_down_backward(A, A, A, 4, 256, 200, 128, A, A, None) == U
+    assert lib.moe_expert_up_backward(A, A, 4, 256, 256, 128, A, MIS, None) == E
+    assert lib.moe_expert_up_backward(A, A, 0, 256, 256, 128, A, A, None) == E
+    # expert wgrad
+    assert lib.moe_expert_wgrad(A, A, A, 4, 256, 100, 256, A, None) == U
+    assert lib.moe_expert_wgrad(A, A, A, 4, 256, 128, 200, A, None) == U
+    assert lib.moe_expert_wgrad(A, None, A, 4, 256, 128, 256, A, None) == E
+    assert lib.moe_expert_wgrad(A, A, None, 4, 256, 128, 256, A, None) == E
+    # gate backward
+    assert lib.moe_gate_backward(A, A, A, A, A, A, 64, 256, 16, 4, 2, ctypes.c_float(1.0), A, A,
+                                 None) == E
+    assert lib.moe_gate_backward(A, A, A, A, A, A, 64, 256, 16, 17, 0, ctypes.c_float(1.0), A, A,
+                                 None) == U
+    assert lib.moe_gate_backward(A, A, A, A, A, A, 64, 256, 16, 4, 0, ctypes.c_float(0.0), A, A,
+                                 None) == E
+    assert lib.moe_gate_backward(A, A, A, A, None, A, 64, 256, 16, 4, 0, ctypes.c_float(1.0), A,
+                                 A, None) == E
+    # du combine, centroid gradient
+    assert lib.moe_combine_dx(A, A, A, A, A, A, A, 64, 256, 9, A, None) == U
+    assert lib.moe_combine_dx(MIS, A, A, A, A, A, A, 64, 256, 4, A, None) == E
+    assert lib.moe_combine_dx(A, A, A, A, None, A, A, 64, 256, 4, A, None) == E
+    assert lib.moe_centroid_grad(A, A, A, 16, 256, 250, A, None) == U
+    assert lib.moe_centroid_grad(A, None, A, 16, 256, 256, A, None) == E

@@ -226,33 +226,37 @@ def test_grouped_ffn_single_group_vs_torch_matmul():
                 what="h")
 
 
-@pytest.mark.parametrize("extra", [0, 600])
+@pytest.mark.parametrize("extra", [0, 256, 600])
 def test_grouped_ffn_tile_paths_by_group_size(extra):
     """Group sizes that hit every tile path of both grouped-GEMM forms: empty
     groups, ragged last tiles of every size, full tiles. Each group against fp32
     torch matmuls of the same bf16 operands, h rounded to bf16 as the kernel
-    does."""
+    does; rows past the last group stay untouched."""
     # extra = 0: groups average < 256 rows -> single-CTA 128-row tiles;
-    # extra = 600: larger groups -> CTA-pair 256-row tiles. Either way the
-    # last tile of a group is ragged in every way (1..255 valid rows).
+    # extra = 256, 600: larger groups -> CTA-pair tiles of 256 rows, the last
+    # one an MMA of N = its rows rounded up to 32 (1..256 valid rows: 257,
+    # 271, ... leave 1, 15, 16, 17, 31, 32, 33, ... rows in the last tile).
     sizes = [1, 15, 0, 16, 17, 31, 32, 33, 100, 127, 128, 129, 255, 256, 0, 300, 384, 385, 513]
     sizes = [s + extra if s else 0 for s in sizes]
     G, d, inter = len(sizes), 256, 256
     rows = sum(sizes)
+    pad = 64                                   # rows after the last group
     g = torch.Generator(device="cuda").manual_seed(12)
-    x = torch.randn(rows, d, generator=g, device="cuda").bfloat16()
+    x = torch.randn(rows + pad, d, generator=g, device="cuda").bfloat16()
     w1 = (0.05 * torch.randn(G, inter, d, generator=g, device="cuda")).bfloat16()
     w3 = (0.05 * torch.randn(G, inter, d, generator=g, device="cuda")).bfloat16()
     w2 = (0.05 * torch.randn(G, d, inter, generator=g, device="cuda")).bfloat16()
     w13 = torch.empty(G, 2 * inter, d, dtype=torch.bfloat16, device="cuda")
     L.moe_pack_w13(w1, w3, G, inter, d, w13)
     off = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32, device="cuda")
-    y = torch.full((rows, d), 3.0, dtype=torch.bfloat16, device="cuda")
-    wsb = L.moe_grouped_ffn_workspace_size(rows, inter)
+    y = torch.full((rows + pad, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    wsb = L.moe_grouped_ffn_workspace_size(rows + pad, inter)
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
-    L.moe_grouped_ffn(x, None, off, G, rows, d, inter, w13, None, w2, None, L.MOE_BF16, y, ws, wsb)
+    L.moe_grouped_ffn(x, None, off, G, rows + pad, d, inter, w13, None, w2, None, L.MOE_BF16, y,
+                      ws, wsb)
     torch.cuda.synchronize()
     assert L.moe_get_device_status() == 0
+    assert bool((y[rows:] == 3.0).all())
     o = off.cpu().tolist()
     for i in range(G):
         a, b = o[i], o[i + 1]
