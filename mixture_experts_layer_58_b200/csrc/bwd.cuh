@@ -198,26 +198,61 @@ combine_dx_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
 }
 
 // de_i = sum over the rows r of group i of dz_perm[r] x_perm[r]. Block
-// (group i, 2048-column chunk); each thread owns 8 columns of the chunk.
-constexpr int kCentroidCols = 2048;
-__global__ void __launch_bounds__(kCentroidCols / 8)
+// (group i, 256 columns): warp w sums rows w, w+8, ... of the group (each lane
+// 8 columns, four rows in flight), then the 8 partial sums are added in a
+// fixed order through shared memory (no atomics: the result is reproducible).
+constexpr int kCentroidCols = 256;
+constexpr int kCentroidWarps = 8;
+__global__ void __launch_bounds__(32 * kCentroidWarps)
 centroid_grad_kernel(const __nv_bfloat16* __restrict__ x_perm, const float* __restrict__ dz_perm,
                      const int32_t* __restrict__ offsets, int d,
                      __nv_bfloat16* __restrict__ de) {
+  __shared__ float part[kCentroidWarps][kCentroidCols + 4];
   const int i = blockIdx.x;
-  const int col = blockIdx.y * kCentroidCols + threadIdx.x * 8;
-  if (col >= d) return;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int col = blockIdx.y * kCentroidCols + lane * 8;
   const int r0 = __ldg(offsets + i);
   const int r1 = __ldg(offsets + i + 1);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int r = r0; r < r1; ++r) {
-    const float w = __ldg(dz_perm + r);
-    float x[8];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x_perm + static_cast<size_t>(r) * d + col)), x);
+  if (col < d) {
+    int r = r0 + warp;
+    for (; r + 3 * kCentroidWarps < r1; r += 4 * kCentroidWarps) {
+      uint4 q[4];
+      float w[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] = fmaf(w, x[k], acc[k]);
+      for (int j = 0; j < 4; ++j) {
+        const int rr = r + j * kCentroidWarps;
+        q[j] = __ldg(reinterpret_cast<const uint4*>(x_perm + static_cast<size_t>(rr) * d + col));
+        w[j] = __ldg(dz_perm + rr);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float x[8];
+        bf16x8_to_f32(q[j], x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = fmaf(w[j], x[k], acc[k]);
+      }
+    }
+    for (; r < r1; r += kCentroidWarps) {
+      float x[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x_perm + static_cast<size_t>(r) * d + col)), x);
+      const float w = __ldg(dz_perm + r);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] = fmaf(w, x[k], acc[k]);
+    }
   }
-  *reinterpret_cast<uint4*>(de + static_cast<size_t>(i) * d + col) = f32_to_bf16x8(acc);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) part[warp][lane * 8 + k] = acc[k];
+  __syncthreads();
+  // thread t finishes column t of the block: sum of the 8 warps in order
+  const int c = blockIdx.y * kCentroidCols + threadIdx.x;
+  if (threadIdx.x < kCentroidCols && c < d) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCentroidWarps; ++w) s += part[w][threadIdx.x];
+    de[static_cast<size_t>(i) * d + c] = __float2bfloat16_rn(s);
+  }
 }
 
 }  // namespace moe

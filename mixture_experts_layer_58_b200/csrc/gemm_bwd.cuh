@@ -17,10 +17,12 @@
 //
 // Both kernels keep the forward kernel's shape: one persistent CTA per SM,
 // warp 0 TMA producer, warp 1 MMA issuer, warps 2-5 epilogue, a 4-stage ring
-// of 48 KB and a double-buffered 2 x 256-column TMEM accumulator; all waits
-// bounded, no TMA multicast.
+// of 48 KB and a double-buffered 2 x 256-column TMEM accumulator; tiles in
+// index order from a global counter (tileq.cuh); all waits bounded, no TMA
+// multicast.
 #pragma once
 #include "gemm.cuh"
+#include "tileq.cuh"
 
 namespace moe {
 
@@ -92,7 +94,8 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmW,
                           const int32_t* __restrict__ offsets, int G, int K, int N, int rows,
                           __nv_bfloat16* __restrict__ out, int ldo,
-                          const __nv_bfloat16* __restrict__ ac, unsigned int* status) {
+                          const __nv_bfloat16* __restrict__ ac, int* tile_counter,
+                          unsigned int* status) {
   using C = BwdCfg;
   constexpr int BN = C::kBN;
   extern __shared__ uint8_t smem_raw[];
@@ -104,7 +107,10 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* tq_full = mma_done + 1;
+  uint64_t* tq_empty = tq_full + kCtaTileQ;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kCtaTileQ);
+  int* tq = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_tstart = s_off + (G + 1);
   int* s_end = s_tstart + (G + 1);
@@ -125,6 +131,10 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         mbar_init(&tempty[a], 128);
       }
       mbar_init(mma_done, 1);
+      for (int j = 0; j < kCtaTileQ; ++j) {
+        mbar_init(&tq_full[j], 1);
+        mbar_init(&tq_empty[j], 5);   // MMA role + 4 epilogue warps
+      }
       fence_mbar_init();
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmW);
@@ -147,7 +157,11 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t phase = 0;
     uint32_t issued = 0, issued_par = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    int t_next = atomicAdd(tile_counter, 1);
+    for (int i = 0; ok; ++i) {
+      const int t = min(t_next, total_tiles);
+      if (!cta_tile_push(i, t, tq, tq_full, tq_empty, status) || t >= total_tiles) break;
+      t_next = atomicAdd(tile_counter, 1);
       int g, m_blk, n_blk;
       decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int a_row = s_off[g] + m_blk * kBM;
@@ -180,8 +194,11 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    int local = 0;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+    for (int local = 0; ok; ++local) {
+      int t;
+      if (!cta_tile_pop(local, tq, tq_full, tq_empty, t, status, kStatusTimeoutMma) ||
+          t >= total_tiles)
+        break;
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       if (!mbar_wait(&tempty[acc], acc_par ^ 1u, status, kStatusTimeoutMma)) break;
@@ -214,8 +231,14 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    int local = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+    for (int local = 0;; ++local) {
+      int t = total_tiles;
+      bool got = true;
+      if (lane == 0)
+        got = cta_tile_pop(local, tq, tq_full, tq_empty, t, status, kStatusTimeoutEpilogue);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (!got || t >= total_tiles) break;
       int g, m_blk, n_blk;
       decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int acc = local & 1;
@@ -299,7 +322,7 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmD,
                           const int32_t* __restrict__ offsets, int G, int M, int N, int rows,
-                          unsigned int* status) {
+                          int* tile_counter, unsigned int* status) {
   using C = BwdCfg;
   constexpr int BN = C::kBN;
   extern __shared__ uint8_t smem_raw[];
@@ -312,7 +335,10 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* tq_full = mma_done + 1;
+  uint64_t* tq_empty = tq_full + kCtaTileQ;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kCtaTileQ);
+  int* tq = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_end = s_off + (G + 1);
 
@@ -334,6 +360,10 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
         mbar_init(&tempty[a], 128);
       }
       mbar_init(mma_done, 1);
+      for (int j = 0; j < kCtaTileQ; ++j) {
+        mbar_init(&tq_full[j], 1);
+        mbar_init(&tq_empty[j], 5);   // MMA role + 4 epilogue warps
+      }
       fence_mbar_init();
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
@@ -361,7 +391,11 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t phase = 0;
     uint32_t issued = 0, issued_par = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    int t_next = atomicAdd(tile_counter, 1);
+    for (int i = 0; ok; ++i) {
+      const int t = min(t_next, total_tiles);
+      if (!cta_tile_push(i, t, tq, tq_full, tq_empty, status) || t >= total_tiles) break;
+      t_next = atomicAdd(tile_counter, 1);
       const int g = t / per_group;
       const int rem = t - g * per_group;
       const int n_blk = rem / mb;
@@ -402,8 +436,14 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    int local = 0;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++local) {
+    for (int local = 0; ok; ++local) {
+      int t = total_tiles;
+      bool popped = true;
+      if (lane == 0)
+        popped = cta_tile_pop(local, tq, tq_full, tq_empty, t, status, kStatusTimeoutMma);
+      popped = __shfl_sync(0xffffffffu, popped ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (!popped || t >= total_tiles) break;
       const int g = t / per_group;
       const int r0 = s_off[g];
       const int m_rows = s_end[g] - r0;
@@ -464,12 +504,22 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     // single lane stores the block with TMA (dW tiles are whole, and the
     // tensor map clips a last half block at N), so the global writes are
     // full rows of 64 B instead of one 16-B piece per row per instruction.
+    // The buffer uses the 64-byte swizzle of the tensor map: 16-B chunk q of
+    // row r sits at chunk q ^ ((r >> 1) & 3), so the 8 rows one phase of a
+    // 16-B shared store touches fall in 8 different bank groups.
     const int quarter = warp & 3;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     uint8_t* obuf = sOut + (warp - 2) * 2 * C::kOutBufBytes;
-    int local = 0;
+    const int sw = (lane >> 1) & 3;
     int chunk = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++local) {
+    for (int local = 0;; ++local) {
+      int t = total_tiles;
+      bool got = true;
+      if (lane == 0)
+        got = cta_tile_pop(local, tq, tq_full, tq_empty, t, status, kStatusTimeoutEpilogue);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (!got || t >= total_tiles) break;
       const int g = t / per_group;
       const int rem = t - g * per_group;
       const int n_blk = rem / mb;
@@ -481,30 +531,35 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * BN + lane_addr;
       const int y = g * M + m_blk * kBM + quarter * 32;
-      const int ncols = min(BN, N - n_blk * BN);
+      const int ncols = min(BN, N - n_blk * BN);   // 128 or 256
 #pragma unroll 1
-      for (int c = 0; c < ncols; c += 32, ++chunk) {
-        uint32_t r[32];
-        tmem_ld_32cols(taddr + c, r);
+      for (int c = 0; c < ncols; c += 64) {
+        uint32_t r[2][32];
+        tmem_ld_32cols(taddr + c, r[0]);
+        tmem_ld_32cols(taddr + c + 32, r[1]);
         tmem_ld_wait();
-        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = empty_group ? 0u
-                              : pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-        uint8_t* buf = obuf + (chunk & 1) * C::kOutBufBytes;
-        // the store issued from this buffer two chunks ago must have read it
-        if (lane == 0) bulk_wait_group_read<1>();
-        __syncwarp();
-        uint4* row = reinterpret_cast<uint4*>(buf + lane * 64);
+        for (int h = 0; h < 2; ++h, ++chunk) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          row[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmD, buf, n_blk * BN + c, y);
-          bulk_commit_group();
+          for (int i = 0; i < 16; ++i)
+            pk[i] = empty_group ? 0u
+                                : pack_bf16x2(__uint_as_float(r[h][2 * i]),
+                                              __uint_as_float(r[h][2 * i + 1]));
+          uint8_t* buf = obuf + (chunk & 1) * C::kOutBufBytes;
+          // the store issued from this buffer two chunks ago must have read it
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          uint4* row = reinterpret_cast<uint4*>(buf + lane * 64);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            row[v ^ sw] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmD, buf, n_blk * BN + c + 32 * h, y);
+            bulk_commit_group();
+          }
         }
       }
       tc_fence_before();

@@ -16,7 +16,8 @@
 //
 // 10 warps, one persistent CTA per SM, 128 x 128 tiles:
 //   warp 0      TMA producer: A [128 rows x 128 B] + B [128 rows x 128 B] per stage,
-//               6 stages.
+//               6 stages; takes the tiles in index order from a global counter
+//               and hands each index to the other roles (tileq.cuh).
 //   warp 1      MMA issuer: one K block (4 x K=32) per P buffer, two buffers of
 //               128 TMEM columns.
 //   warps 2-9   promotion + epilogue. Warp w reads TMEM lane quarter w % 4;
@@ -31,6 +32,7 @@
 #pragma once
 #include "fp8.cuh"
 #include "gemm.cuh"
+#include "tileq.cuh"
 
 namespace moe {
 
@@ -78,7 +80,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                         const float* __restrict__ a_scales, const float* __restrict__ b_scales,
                         const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
                         int rows, __nv_bfloat16* __restrict__ out, int ldo,
-                        unsigned int* status) {
+                        int* tile_counter, unsigned int* status) {
   using C = GemmF8Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -89,7 +91,10 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* pfull = empty + kF8Stages;
   uint64_t* pempty = pfull + 2;
   uint64_t* mma_done = pempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* tq_full = mma_done + 1;
+  uint64_t* tq_empty = tq_full + kCtaTileQ;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kCtaTileQ);
+  int* tq = reinterpret_cast<int*>(tmem_slot + 1);
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);
   int* s_tstart = s_off + (G + 1);
   int* s_end = s_tstart + (G + 1);
@@ -110,6 +115,10 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         mbar_init(&pempty[b], kF8EpiThreads);
       }
       mbar_init(mma_done, 1);
+      for (int j = 0; j < kCtaTileQ; ++j) {
+        mbar_init(&tq_full[j], 1);
+        mbar_init(&tq_empty[j], 1 + kF8EpiThreads / 32);   // MMA thread + epilogue warps
+      }
       fence_mbar_init();
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
@@ -156,7 +165,11 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t phase = 0;
     uint32_t issued = 0, issued_par = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    int t_next = atomicAdd(tile_counter, 1);
+    for (int i = 0; ok; ++i) {
+      const int t = min(t_next, total_tiles);
+      if (!cta_tile_push(i, t, tq, tq_full, tq_empty, status) || t >= total_tiles) break;
+      t_next = atomicAdd(tile_counter, 1);
       int g, m_blk, n_blk;
       decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int a_row = s_off[g] + m_blk * kBM;
@@ -187,7 +200,11 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t phase = 0;
     uint32_t kcount = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    for (int i = 0; ok; ++i) {
+      int t;
+      if (!cta_tile_pop(i, tq, tq_full, tq_empty, t, status, kStatusTimeoutMma) ||
+          t >= total_tiles)
+        break;
       for (int kb = 0; kb < num_kb; ++kb, ++kcount) {
         const uint32_t pb = kcount & 1u;
         const uint32_t ppar = (kcount >> 1) & 1u;
@@ -225,7 +242,14 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     const int ksb = num_kb;                   // scale blocks along K
     uint32_t kcount = 0;
     bool broken = false;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+    for (int i = 0;; ++i) {
+      int t = total_tiles;
+      bool got = true;
+      if (lane == 0)
+        got = cta_tile_pop(i, tq, tq_full, tq_empty, t, status, kStatusTimeoutEpilogue);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (!got || t >= total_tiles) break;
       int g, m_blk, n_blk;
       decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int row0 = s_off[g] + m_blk * kBM;

@@ -122,8 +122,8 @@ int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
   return MOE_OK;
 }
 
-// 2-D bf16 tensor map for TMA stores of 32 x 32 blocks (no swizzle) into a
-// row-major [rows, cols] matrix.
+// 2-D bf16 tensor map for TMA stores of 32 x 32 blocks into a row-major
+// [rows, cols] matrix; the shared-memory block uses the 64-byte swizzle.
 int make_tmap_bf16_store32(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
   int rc = get_encoder();
   if (rc != MOE_OK) return rc;
@@ -132,7 +132,7 @@ int make_tmap_bf16_store32(CUtensorMap* map, void* base, uint64_t cols, uint64_t
   cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     t_last_cuda_error = static_cast<int>(r);
@@ -213,8 +213,11 @@ int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int 
   const long long max_tiles =
       (static_cast<long long>(rows) / kBM + G) * static_cast<long long>(n_per_group / kF8BN);
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
+  int* counter = di->tile_counters + (di->next_counter.fetch_add(1) % kTileCounters);
+  MOE_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   kern<<<grid, kF8Threads, smem, st>>>(tmA, tmB, a_scales, b_scales, offsets, G, K, n_per_group,
-                                       rows, static_cast<__nv_bfloat16*>(out), ldo, di->status);
+                                       rows, static_cast<__nv_bfloat16*>(out), ldo, counter,
+                                       di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -281,9 +284,12 @@ int launch_dgrad(const void* A, int rows, int K, const void* W, int G, int N,
   const long long max_tiles = (static_cast<long long>(rows) / kBM + G) *
                               static_cast<long long>((N + BwdCfg::kBN - 1) / BwdCfg::kBN);
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
+  int* counter = di->tile_counters + (di->next_counter.fetch_add(1) % kTileCounters);
+  MOE_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   kern<<<grid, kGemmThreads, smem, st>>>(tmA, tmW, offsets, G, K, N, rows,
                                          static_cast<__nv_bfloat16*>(out), ldo,
-                                         static_cast<const __nv_bfloat16*>(ac), di->status);
+                                         static_cast<const __nv_bfloat16*>(ac), counter,
+                                         di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -304,8 +310,10 @@ int launch_wgrad(const void* A, const void* B, int rows, int M, int N, int G,
   const long long tiles = static_cast<long long>(G) * (M / kBM) *
                           ((N + BwdCfg::kBN - 1) / BwdCfg::kBN);
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, tiles)));
+  int* counter = di->tile_counters + (di->next_counter.fetch_add(1) % kTileCounters);
+  MOE_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   grouped_wgrad_bf16_kernel<<<grid, kGemmThreads, smem, st>>>(tmA, tmB, tmD, offsets, G, M, N,
-                                                               rows, di->status);
+                                                               rows, counter, di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -907,7 +915,7 @@ int moe_centroid_grad(const void* x_perm, const float* dz_perm, const int32_t* e
   if (!expert_offsets || !de || !aligned16(de)) return MOE_ERR_INVALID_ARG;
   if (rows > 0 && (!x_perm || !dz_perm || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
   dim3 grid(n_routed, (d + kCentroidCols - 1) / kCentroidCols);
-  centroid_grad_kernel<<<grid, kCentroidCols / 8, 0, as_stream(stream)>>>(
+  centroid_grad_kernel<<<grid, 32 * kCentroidWarps, 0, as_stream(stream)>>>(
       static_cast<const __nv_bfloat16*>(x_perm), dz_perm, expert_offsets, d,
       static_cast<__nv_bfloat16*>(de));
   MOE_CUDA(cudaGetLastError());
