@@ -361,6 +361,8 @@ def main():
                          "fused: the up-projection gathers the token rows itself (bf16; measured "
                          "slower: the TMA gathers are request-rate bound); train: forward with "
                          "saved pre-activations + backward + bias update (bf16)")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="run the shared expert after the routed experts on one stream")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -402,7 +404,8 @@ def main():
     shared = synth.shared_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
     lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
                    routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
-                   fp8=cfg.fp8, fused_gather=(args.mode == "fused"), device=dev)
+                   fp8=cfg.fp8, fused_gather=(args.mode == "fused"),
+                   overlap_shared=not args.no_overlap, device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
     torch.cuda.empty_cache()
@@ -410,37 +413,11 @@ def main():
     u = u_host.to(dev)
     lay.allocate(T)
     stream = torch.cuda.current_stream()
-    up_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
 
-    def step(i=None):
-        lay.route(u)
-        lay.permute(u)
-        if i is not None:
-            up_ev[i][0].record(stream)
-        if lay.fused_gather:
-            L.moe_expert_up_swiglu_gather(u, T, lay.src, lay.offsets, cfg.n_routed, T * K, d, I,
-                                          lay.w13, lay.ffn_ws)
-        elif cfg.fp8:
-            hb = lay.ffn_ws
-            h8 = lay.ffn_ws[(T * K * I * 2 + 255) // 256 * 256:]
-            hs = h8[(T * K * I + 255) // 256 * 256:]
-            L.moe_expert_up_swiglu_fp8(lay.x8, lay.x_s, lay.offsets, cfg.n_routed, T * K, d, I,
-                                       lay.w13, lay.w13_s, hb)
-        else:
-            L.moe_expert_up_swiglu(lay.x_perm, lay.offsets, cfg.n_routed, T * K, d, I, lay.w13,
-                                   lay.ffn_ws)
-        if i is not None:
-            up_ev[i][1].record(stream)
-        if cfg.fp8:
-            L.moe_quant_act_fp8(hb, T * K, I, h8, hs)
-            L.moe_expert_down_fp8(h8, hs, lay.offsets, cfg.n_routed, T * K, I, d, lay.w2,
-                                  lay.w2_s, lay.y_perm)
-        else:
-            L.moe_expert_down(lay.ffn_ws, lay.offsets, cfg.n_routed, T * K, I, d, lay.w2,
-                              lay.y_perm)
-        lay.shared_ffn(u)
-        lay.combine(u)
+    up_timers = {}
+
+    def step(timed=False):
+        lay.forward(u, timers=up_timers if timed else None)
         if cfg.gate_kind == "sigmoid":
             if world > 1:
                 lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
@@ -462,13 +439,13 @@ def main():
         barrier()
         torch.cuda.synchronize()
         t_start.record(stream)
-        for i in range(args.steps):
-            step(i)
+        for _ in range(args.steps):
+            step(timed=True)
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
     ms = t_start.elapsed_time(t_end)
-    up_ms = sum(a.elapsed_time(b) for a, b in up_ev) / args.steps
+    up_ms = sum(a.elapsed_time(b) for a, b in up_timers["up"]) / args.steps
     if world > 1:
         tt = torch.tensor([ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -573,6 +550,8 @@ def main():
                    "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
                    "gate": cfg.gate_kind, "global_batch_tokens": T * world,
                    "mode": "fused gather" if lay.fused_gather else "five-call",
+                   "shared_expert": "side stream, overlapped" if lay.overlap_shared
+                   else "after the routed experts",
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (22.6 GB of expert weights streamed per step)"
                    if cfg.weights_on_gpu else "L2 not flushed: small workload",

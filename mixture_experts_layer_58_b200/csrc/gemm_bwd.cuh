@@ -243,15 +243,37 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       decode_tile(t, s_tstart, s_off, s_end, G, g, m_blk, n_blk);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], acc_par, status, kStatusTimeoutEpilogue)) break;
-      tc_fence_after();
       const int grow = s_off[g] + m_blk * kBM + row_in_tile;
       const bool valid = grow < min(s_end[g], rows);
-      const uint32_t taddr = tmem_base + acc * BN + lane_addr;
       const int ncols = min(BN, N - n_blk * BN);
+      // SwiGLU backward: the saved [a|c] of this row, one 128-byte piece per
+      // 32 h columns, loaded a chunk ahead (the first while the MMAs of the
+      // tile still run) so its latency overlaps the work
+      const uint4* ac_row = nullptr;
+      uint4 in_next[8];
+      if constexpr (EPI == EPI_DG_SWIGLU_BWD) {
+        ac_row = reinterpret_cast<const uint4*>(ac + static_cast<size_t>(valid ? grow : 0) * ldo +
+                                                2 * (n_blk * BN));
+        if (valid) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) in_next[v] = __ldg(ac_row + v);
+        }
+      }
+      if (!mbar_wait(&tfull[acc], acc_par, status, kStatusTimeoutEpilogue)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + acc * BN + lane_addr;
 #pragma unroll 1
       for (int c = 0; c < ncols; c += 32) {
         uint32_t r[32];
+        uint4 in[8];
+        if constexpr (EPI == EPI_DG_SWIGLU_BWD) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) in[v] = in_next[v];
+          if (valid && c + 32 < ncols) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) in_next[v] = __ldg(ac_row + (c + 32) / 4 + v);
+          }
+        }
         tmem_ld_32cols(taddr + c, r);
         tmem_ld_wait();
         if (!valid) continue;
@@ -269,11 +291,6 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           // h columns j0 + [0, 32) <-> ac / dac columns 2*j0 + [0, 64):
           // [a 0..15 | c 0..15 | a 16..31 | c 16..31]
           const int j0 = n_blk * BN + c;
-          const uint4* src =
-              reinterpret_cast<const uint4*>(ac + static_cast<size_t>(grow) * ldo + 2 * j0);
-          uint4 in[8];
-#pragma unroll
-          for (int v = 0; v < 8; ++v) in[v] = __ldg(src + v);
           const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(in);
           uint32_t pk[32];
 #pragma unroll

@@ -305,13 +305,13 @@ int launch_wgrad(const void* A, const void* B, int rows, int M, int N, int G,
   if ((rc = make_tmap_bf16(&tmB, B, N, rows, 64)) != MOE_OK) return rc;
   if ((rc = make_tmap_bf16_store32(&tmD, dw, N, static_cast<uint64_t>(G) * M)) != MOE_OK)
     return rc;
+  int* counter = di->tile_counters + (di->next_counter.fetch_add(1) % kTileCounters);
+  MOE_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   const size_t smem = BwdCfg::wgrad_smem_bytes(G);
   if ((rc = set_smem(grouped_wgrad_bf16_kernel, smem)) != MOE_OK) return rc;
   const long long tiles = static_cast<long long>(G) * (M / kBM) *
                           ((N + BwdCfg::kBN - 1) / BwdCfg::kBN);
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, tiles)));
-  int* counter = di->tile_counters + (di->next_counter.fetch_add(1) % kTileCounters);
-  MOE_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   grouped_wgrad_bf16_kernel<<<grid, kGemmThreads, smem, st>>>(tmA, tmB, tmD, offsets, G, M, N,
                                                                rows, counter, di->status);
   MOE_CUDA(cudaGetLastError());

@@ -60,7 +60,8 @@ class MoELayer:
 
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
-                 fp8: bool = False, fused_gather: bool = False, device="cuda"):
+                 fp8: bool = False, fused_gather: bool = False, overlap_shared: bool = True,
+                 device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -75,6 +76,8 @@ class MoELayer:
         # fused gather (bf16): the up-projection reads the token rows of u
         # itself, so the dispatch only computes row indices (no x_perm copy)
         self.fused_gather = bool(fused_gather) and not self.fp8
+        # bf16: run the shared expert on a side stream next to the routed path
+        self.overlap_shared = bool(overlap_shared) and not self.fp8
         self.centroids = centroids.to(dev, bf).contiguous()
         self.bias = (bias.to(dev, torch.float32).contiguous() if bias is not None
                      else torch.zeros(self.n_routed, dtype=torch.float32, device=dev))
@@ -158,6 +161,11 @@ class MoELayer:
         self.ffn_ws = torch.empty(ffn_ws, dtype=torch.uint8, device=dev)
         self.shared_out = (torch.empty((T, d), dtype=torch.bfloat16, device=dev)
                            if self.ws13 is not None else None)
+        # the shared expert runs on a side stream next to the routed path
+        # (bf16), so it gets its own workspace
+        self.shared_ws_bytes = L.moe_grouped_ffn_workspace_size(T, max(self.shared_inter, 128), dt)
+        self.shared_ws = (torch.empty(self.shared_ws_bytes, dtype=torch.uint8, device=dev)
+                          if self.ws13 is not None else None)
         self.shared_offsets = torch.tensor([0, T], dtype=i32, device=dev)
         self.out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
         self._T = T
@@ -186,6 +194,39 @@ class MoELayer:
                       self.x_perm, self.offsets, self.pos, self.src, self.perm_ws,
                       self.perm_ws_bytes)
 
+    def _routed_up(self, T, u):
+        rows = T * self.top_k
+        if self.fused_gather:
+            L.moe_expert_up_swiglu_gather(u, T, self.src, self.offsets, self.n_routed, rows, self.d,
+                                          self.inter, self.w13, self.ffn_ws)
+        elif self.fp8:
+            hb, h8, hs = self._fp8_h()
+            L.moe_expert_up_swiglu_fp8(self.x8, self.x_s, self.offsets, self.n_routed, rows,
+                                       self.d, self.inter, self.w13, self.w13_s, hb)
+        else:
+            L.moe_expert_up_swiglu(self.x_perm, self.offsets, self.n_routed, rows, self.d,
+                                   self.inter, self.w13, self.ffn_ws)
+
+    def _routed_down(self, T):
+        rows = T * self.top_k
+        if self.fp8:
+            hb, h8, hs = self._fp8_h()
+            L.moe_quant_act_fp8(hb, rows, self.inter, h8, hs)
+            L.moe_expert_down_fp8(h8, hs, self.offsets, self.n_routed, rows, self.inter, self.d,
+                                  self.w2, self.w2_s, self.y_perm)
+        else:
+            L.moe_expert_down(self.ffn_ws, self.offsets, self.n_routed, rows, self.inter, self.d,
+                              self.w2, self.y_perm)
+
+    def _fp8_h(self):
+        """Views of the FP8 FFN workspace: bf16 h, its E4M3 codes, their scales
+        (the layout moe_grouped_ffn uses)."""
+        rows = self._T * self.top_k
+        hb = self.ffn_ws
+        h8 = self.ffn_ws[(rows * self.inter * 2 + 255) // 256 * 256:]
+        hs = h8[(rows * self.inter + 255) // 256 * 256:]
+        return hb, h8, hs
+
     def routed_ffn(self, T, u=None):
         if self.fused_gather:
             rows = T * self.top_k
@@ -213,8 +254,8 @@ class MoELayer:
                               L.MOE_FP8_E4M3, self.shared_out, self.ffn_ws, self.ffn_ws_bytes)
             return
         L.moe_grouped_ffn(u, None, self.shared_offsets, 1, T, self.d, self.shared_inter, self.ws13,
-                          None, self.ws2, None, L.MOE_BF16, self.shared_out, self.ffn_ws,
-                          self.ffn_ws_bytes)
+                          None, self.ws2, None, L.MOE_BF16, self.shared_out, self.shared_ws,
+                          self.shared_ws_bytes)
 
     def combine(self, u, residual: bool = True, out=None):
         T = u.shape[0]
@@ -222,10 +263,15 @@ class MoELayer:
                       u if residual else None, T, self.d, self.top_k,
                       self.out if out is None else out)
 
-    def forward(self, u, residual: bool = True, out=None, train: bool = False):
+    def forward(self, u, residual: bool = True, out=None, train: bool = False, timers=None):
         """h' for the bf16 batch u [T, d] (device), written to `out` ([T, d]
         bf16, device) or to the layer's own output buffer, which is returned.
-        train=True (bf16, copy-based dispatch) keeps what backward() needs."""
+        train=True (bf16, copy-based dispatch) keeps what backward() needs.
+        The bf16 shared expert depends on u alone: it runs on a side stream
+        while the current stream routes and dispatches (and, for decode-sized
+        groups, runs the routed experts); the current stream waits for it
+        before the routed GEMMs (large groups) or before the combine. timers: optional dict; the
+        routed up-projection gets a (start, end) event pair under "up"."""
         assert u.dtype == torch.bfloat16 and u.is_contiguous() and u.device.type == "cuda"
         T = u.shape[0]
         self.allocate(T)
@@ -236,17 +282,54 @@ class MoELayer:
                 raise ValueError("training runs on the bf16 layer with the copy-based dispatch")
             self._allocate_train(T)
         self._train_state = (u, residual) if train else None
+        side = None
+        if T > 0 and self.ws13 is not None and self.overlap_shared:
+            side = self._fork()
+            u.record_stream(side)
+            with torch.cuda.stream(side):
+                if train:
+                    self._shared_ffn_train(u)
+                else:
+                    self.shared_ffn(u)
+            self._join_event.record(side)
         self.route(u)
+        # Where the shared expert rejoins: the routed GEMMs of large groups
+        # (CTA-pair form) are compute-bound like the shared expert itself, so
+        # the shared expert overlaps only the HBM-bound route and dispatch and
+        # the routed GEMMs run alone; decode-sized groups stream their weights
+        # from HBM, and the shared expert runs next to them too.
+        join_early = side is not None and T * self.top_k >= 256 * self.n_routed
         if T > 0:
             self.permute(u)
+            if join_early:
+                torch.cuda.current_stream().wait_event(self._join_event)
+            with _Timed(timers)("up"):
+                if train:
+                    self._routed_up_train(T)
+                else:
+                    self._routed_up(T, u)
             if train:
-                self._routed_ffn_train(T)
-                self._shared_ffn_train(u)
+                self._routed_down_train(T)
             else:
-                self.routed_ffn(T, u)
+                self._routed_down(T)
+            if side is None:
                 self.shared_ffn(u)
+            elif not join_early:
+                torch.cuda.current_stream().wait_event(self._join_event)
             self.combine(u, residual, dst)
         return dst
+
+    def _fork(self):
+        """Side stream for the shared expert, ordered after everything already
+        on the current stream (the previous step's combine included)."""
+        cur = torch.cuda.current_stream()
+        if getattr(self, "_side", None) is None:
+            self._side = torch.cuda.Stream(device=self.device)
+            self._fork_event = torch.cuda.Event()
+            self._join_event = torch.cuda.Event()
+        self._fork_event.record(cur)
+        self._side.wait_event(self._fork_event)
+        return self._side
 
     # ------------------------------------------------------------------ training
     def _allocate_train(self, T: int) -> None:
@@ -279,10 +362,13 @@ class MoELayer:
                 self.grad_ws2 = torch.empty_like(self.ws2)
         self._train_T = T
 
-    def _routed_ffn_train(self, T):
+    def _routed_up_train(self, T):
         rows = T * self.top_k
         L.moe_expert_up_swiglu_train(self.x_perm, self.offsets, self.n_routed, rows, self.d,
                                      self.inter, self.w13, self.h, self.ac)
+
+    def _routed_down_train(self, T):
+        rows = T * self.top_k
         L.moe_expert_down(self.h, self.offsets, self.n_routed, rows, self.inter, self.d, self.w2,
                           self.y_perm)
 

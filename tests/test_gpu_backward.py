@@ -178,3 +178,65 @@ def test_layer_backward_matches_oracle(name, T, cuda_ok):
         check_close(f64(g3[0]), s3, max_tol=GRAD_MAX, mean_tol=GRAD_MEAN, what="shared dW3")
         check_close(f64(lay.grad_ws2), s2, max_tol=GRAD_MAX, mean_tol=GRAD_MEAN,
                     what="shared dW2")
+
+
+def test_v3p_backward_sampled(cuda_ok):
+    """The training step at the full V3 prefill shape, in the launch
+    configuration `bench.py --mode train` times: du on sampled tokens (those
+    of the hottest and the least-loaded expert and random ones), the complete
+    weight gradients of the least-loaded expert, and sampled columns of the
+    centroid gradient, each against the fp64 backward oracle computed for
+    exactly those entries."""
+    from mixture_experts_layer_58_b200 import build
+    from oracle import moe_oracle as om
+    build.build()
+    cfg = synth.CONFIGS["v3p"]
+    inp = Inputs(cfg)
+    lay = inp.layer
+    lay.forward(inp.u_dev, train=True)
+    g = torch.Generator().manual_seed(99)
+    dout = (0.05 * torch.randn(cfg.T, cfg.d, generator=g)).bfloat16()
+    du = lay.backward(dout.cuda())
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+
+    idx = lay.topk_idx.cpu().numpy().astype(np.int64)
+    counts = np.bincount(idx.ravel(), minlength=cfg.n_routed)
+    hot = int(np.argmax(counts))
+    cold = int(np.argmin(np.where(counts > 0, counts, counts.max() + 1)))
+    rng = np.random.default_rng(4)
+    t_hot = np.nonzero((idx == hot).any(1))[0][:3]
+    t_cold = np.nonzero((idx == cold).any(1))[0]
+    tokens = np.unique(np.concatenate([t_hot, t_cold, rng.choice(cfg.T, 4, replace=False)]))
+    S = cfg.routed_scale
+    shared = inp.shared_list()
+
+    # du and dgate of the sampled tokens: the oracle backward of those tokens
+    # alone is exact (tokens are independent given the selection)
+    ref = mb.layer_backward(inp.u[torch.from_numpy(tokens)], inp.e, idx[tokens], S, inp.expert,
+                            shared, dout[torch.from_numpy(tokens)], cfg.gate_kind)
+    check_close(f64(du)[tokens], ref.du, max_tol=GRAD_MAX, mean_tol=GRAD_MEAN, what="du (sampled)")
+    check_close(f64(lay.dgate)[tokens], ref.dgate, max_tol=GRAD_MAX, mean_tol=GRAD_MEAN,
+                what="dgate (sampled)")
+
+    # complete dW1/dW3/dW2 of the least-loaded expert: its rows are all of t_cold
+    k_cold = np.nonzero(idx[t_cold] == cold)[1]
+    gate = om.gates_for_indices(inp.u[torch.from_numpy(t_cold)], inp.e, idx[t_cold], S,
+                                cfg.gate_kind)
+    w1, w3, w2 = inp.expert(cold)
+    dy = gate[np.arange(len(t_cold)), k_cold][:, None] * f64(dout)[t_cold]
+    _, rw1, rw3, rw2 = mb.ffn_backward(f64(inp.u)[t_cold], w1, w3, w2, dy)
+    dw1, dw3 = _unpack_w13(lay.grad_w13[cold:cold + 1])
+    check_close(f64(dw1[0]), rw1, max_tol=GRAD_MAX, mean_tol=GRAD_MEAN, what=f"dW1 expert {cold}")
+    check_close(f64(dw3[0]), rw3, max_tol=GRAD_MAX, mean_tol=GRAD_MEAN, what=f"dW3 expert {cold}")
+    check_close(f64(lay.grad_w2[cold]), rw2, max_tol=GRAD_MAX, mean_tol=GRAD_MEAN,
+                what=f"dW2 expert {cold}")
+
+    # centroid gradient of the least-loaded expert: sum over its tokens of dz u
+    full_cold = mb.layer_backward(inp.u[torch.from_numpy(t_cold)], inp.e, idx[t_cold], S,
+                                  inp.expert, shared, dout[torch.from_numpy(t_cold)],
+                                  cfg.gate_kind)
+    check_close(f64(lay.grad_centroids[cold]), full_cold.de[cold], max_tol=DE_MAX,
+                mean_tol=DE_MEAN, what=f"de expert {cold}")
+    del inp
+    torch.cuda.empty_cache()
