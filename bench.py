@@ -250,6 +250,10 @@ def run_train(args, cfg, rank, world, local, dev):
     def step(timers=None):
         lay.forward(u, train=True)
         lay.backward(dout, timers)
+        if world > 1:
+            # data parallel: average the weight gradients over the ranks
+            dp.allreduce_grads([lay.grad_w13, lay.grad_w2, lay.grad_centroids,
+                                getattr(lay, "grad_ws13", None), getattr(lay, "grad_ws2", None)])
         if cfg.gate_kind == "sigmoid":
             if world > 1:
                 lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
