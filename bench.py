@@ -537,6 +537,18 @@ def main():
                 "kernel": kname, "kernel_ms": up_ms,
                 "peak_source": f"{pk['_source']} bf16_tflops_sustained"
                                + (" x 2 (nominal fp8/bf16)" if cfg.fp8 else "")}
+    if T * K < 256 * cfg.n_routed:
+        # decode-sized groups: the up-projection streams the W13 slabs of every
+        # expert the batch touches from HBM; its roofline is the copy bandwidth
+        touched = int((counts > 0).sum())
+        wbytes = (1 if cfg.fp8 else 2) * 2 * I * d
+        up_bytes = touched * wbytes + T * K * d * (1 if cfg.fp8 else 2) + T * K * I * 2
+        gbs = up_bytes / (up_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / pk["hbm_gbs"], "traffic": None, "kernel": kname,
+                    "kernel_ms": up_ms, "bytes_per_launch": up_bytes,
+                    "experts_touched": touched,
+                    "peak_source": f"{pk['_source']} hbm_gbs"}
     if cfg.fp8:
         try:
             roofline["cublas_fp8_tflops_live"] = cublas_fp8_tflops(dev)

@@ -5,7 +5,9 @@ in libmoe.so's kernels:
 
     moe_route        gate GEMM + sigmoid + biased top-K + gates + counts
     moe_permute      expert-contiguous copy of the token rows
-    moe_grouped_ffn  routed experts (G = N_r) then the shared expert (G = 1)
+    moe_expert_up_swiglu, moe_expert_down
+                     the routed experts' grouped FFN (G = N_r)
+    moe_grouped_ffn  the shared expert (G = 1), on a side stream
     moe_combine      h' = u + shared + sum_k g * y
     moe_bias_update  b -= / += gamma from the loads (end of the step)
 
@@ -226,23 +228,6 @@ class MoELayer:
         h8 = self.ffn_ws[(rows * self.inter * 2 + 255) // 256 * 256:]
         hs = h8[(rows * self.inter + 255) // 256 * 256:]
         return hb, h8, hs
-
-    def routed_ffn(self, T, u=None):
-        if self.fused_gather:
-            rows = T * self.top_k
-            L.moe_expert_up_swiglu_gather(u, T, self.src, self.offsets, self.n_routed, rows, self.d,
-                                          self.inter, self.w13, self.ffn_ws)
-            L.moe_expert_down(self.ffn_ws, self.offsets, self.n_routed, rows, self.inter, self.d,
-                              self.w2, self.y_perm)
-            return
-        if self.fp8:
-            L.moe_grouped_ffn(self.x8, self.x_s, self.offsets, self.n_routed, T * self.top_k,
-                              self.d, self.inter, self.w13, self.w13_s, self.w2, self.w2_s,
-                              L.MOE_FP8_E4M3, self.y_perm, self.ffn_ws, self.ffn_ws_bytes)
-            return
-        L.moe_grouped_ffn(self.x_perm, None, self.offsets, self.n_routed, T * self.top_k, self.d,
-                          self.inter, self.w13, None, self.w2, None, L.MOE_BF16, self.y_perm,
-                          self.ffn_ws, self.ffn_ws_bytes)
 
     def shared_ffn(self, u):
         if self.ws13 is None:
