@@ -450,6 +450,7 @@ def main():
         barrier()
     ms = t_start.elapsed_time(t_end)
     up_ms = sum(a.elapsed_time(b) for a, b in up_timers["up"]) / args.steps
+    stage_ms = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in up_timers.items()}
     if world > 1:
         tt = torch.tensor([ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -579,6 +580,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2, "api": "MoELayer.forward",
                 "copies": "pinned host, own stream, overlapped with neighbouring steps"},
+        "stage_ms": stage_ms,
         "gpu_launches": args.steps * lay.launches_per_step(),
         "clocks": clk.summary(),
     }

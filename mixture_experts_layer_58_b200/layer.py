@@ -255,8 +255,10 @@ class MoELayer:
         The bf16 shared expert depends on u alone: it runs on a side stream
         while the current stream routes and dispatches (and, for decode-sized
         groups, runs the routed experts); the current stream waits for it
-        before the routed GEMMs (large groups) or before the combine. timers: optional dict; the
-        routed up-projection gets a (start, end) event pair under "up"."""
+        before the routed GEMMs (large groups) or before the combine.
+        timers: optional dict; each stage ("route", "permute", "up", "down",
+        "shared", "combine") gets a (start, end) CUDA event pair, recorded on
+        the stream the stage runs on."""
         assert u.dtype == torch.bfloat16 and u.is_contiguous() and u.device.type == "cuda"
         T = u.shape[0]
         self.allocate(T)
@@ -267,17 +269,20 @@ class MoELayer:
                 raise ValueError("training runs on the bf16 layer with the copy-based dispatch")
             self._allocate_train(T)
         self._train_state = (u, residual) if train else None
+        ev = _Timed(timers)
         side = None
         if T > 0 and self.ws13 is not None and self.overlap_shared:
             side = self._fork()
             u.record_stream(side)
             with torch.cuda.stream(side):
-                if train:
-                    self._shared_ffn_train(u)
-                else:
-                    self.shared_ffn(u)
+                with ev("shared"):
+                    if train:
+                        self._shared_ffn_train(u)
+                    else:
+                        self.shared_ffn(u)
             self._join_event.record(side)
-        self.route(u)
+        with ev("route"):
+            self.route(u)
         # Where the shared expert rejoins: the routed GEMMs of large groups
         # (CTA-pair form) are compute-bound like the shared expert itself, so
         # the shared expert overlaps only the HBM-bound route and dispatch and
@@ -285,23 +290,27 @@ class MoELayer:
         # from HBM, and the shared expert runs next to them too.
         join_early = side is not None and T * self.top_k >= 256 * self.n_routed
         if T > 0:
-            self.permute(u)
+            with ev("permute"):
+                self.permute(u)
             if join_early:
                 torch.cuda.current_stream().wait_event(self._join_event)
-            with _Timed(timers)("up"):
+            with ev("up"):
                 if train:
                     self._routed_up_train(T)
                 else:
                     self._routed_up(T, u)
-            if train:
-                self._routed_down_train(T)
-            else:
-                self._routed_down(T)
+            with ev("down"):
+                if train:
+                    self._routed_down_train(T)
+                else:
+                    self._routed_down(T)
             if side is None:
-                self.shared_ffn(u)
+                with ev("shared"):
+                    self.shared_ffn(u)
             elif not join_early:
                 torch.cuda.current_stream().wait_event(self._join_event)
-            self.combine(u, residual, dst)
+            with ev("combine"):
+                self.combine(u, residual, dst)
         return dst
 
     def _fork(self):

@@ -311,3 +311,20 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert L.moe_get_device_status() == 0
     inp = Inputs(synth.CONFIGS["tiny"])
     _full_check(inp)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_shared_expert_in_line_matches_overlapped(name):
+    """The shared expert on its side stream (default) and run in line after
+    the routed experts give the same layer output bit for bit, and both match
+    the oracle (Mid joins the side stream before the routed GEMMs, Tiny
+    before the combine)."""
+    cfg = synth.CONFIGS[name]
+    inp = Inputs(cfg)
+    lay = inp.layer
+    assert lay.overlap_shared
+    _full_check(inp)
+    overlapped = lay.out.clone()
+    lay.overlap_shared = False
+    _full_check(inp)
+    assert torch.equal(lay.out, overlapped)
