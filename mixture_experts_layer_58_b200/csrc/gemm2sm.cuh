@@ -242,6 +242,7 @@ __device__ __forceinline__ void decode_tile_pair(int t, const int* s_tstart, con
 template <int EPI, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                              const __grid_constant__ CUtensorMap tmA32,
                               const __grid_constant__ CUtensorMap tmB,
                               const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
                               int rows, __nv_bfloat16* __restrict__ out, int ldo,
@@ -294,6 +295,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       fence_mbar_init();
       tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmA32);
       tma_prefetch_desc(&tmB);
     }
     __syncwarp();
@@ -365,6 +367,13 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const int ncols = pair_tile_cols(s_end[g] - row0);
       const int a_row = row0 + static_cast<int>(rank) * (ncols >> 1);
       const int b_row = g * n_per_group + n_blk * BN + static_cast<int>(rank) * 128;
+      // bytes landing on the leader's barrier per stage, from both CTAs: the
+      // weight half-tiles, and the token rows (a full tile or the gather form:
+      // 128 rows in one box or 32 gathers; a ragged tail tile: its ncols/2
+      // rows rounded up to boxes of 32, not a full 128-row box per K step)
+      const int nbox = GATHER ? 4 : ((ncols >> 1) + 31) >> 5;
+      const uint32_t stage_tx =
+          2u * static_cast<uint32_t>(C::kBBytes + nbox * 32 * 128);
       int src[4] = {0, 0, 0, 0};
       if constexpr (GATHER) {
         // rows past the group's end load any row of the group (masked later)
@@ -384,13 +393,18 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           ok = false;
           break;
         }
-        if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+        if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&full[stage], stage_tx);
         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
         if constexpr (GATHER) {
           tma_gather4_pair(sA + stage * C::kABytes + lane * 4 * 128, &tmA, bar, kb * kBK, src[0],
                            src[1], src[2], src[3]);
-        } else {
+        } else if (nbox == 4) {
           tma_load_2d_pair(sA + stage * C::kABytes, &tmA, bar, kb * kBK, a_row);
+        } else {
+          // a ragged tail tile: only the token rows it uses, in boxes of 32
+          for (int j = 0; j < nbox; ++j)
+            tma_load_2d_pair(sA + stage * C::kABytes + j * (32 * 128), &tmA32, bar, kb * kBK,
+                             a_row + 32 * j);
         }
         if (lane == 0) tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, bar, kb * kBK, b_row);
         issued |= 1u << stage;

@@ -235,11 +235,14 @@ int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int 
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmA32, tmB;
   if (src_rows) {
     if ((rc = make_tmap_bf16(&tmA, A, K, a_rows, 1)) != MOE_OK) return rc;
-  } else if ((rc = make_tmap_bf16(&tmA, A, K, rows, 128)) != MOE_OK) {
-    return rc;
+    tmA32 = tmA;
+  } else {
+    // token rows: 128 per box for full tiles, 32 per box for ragged tails
+    if ((rc = make_tmap_bf16(&tmA, A, K, rows, 128)) != MOE_OK) return rc;
+    if ((rc = make_tmap_bf16(&tmA32, A, K, rows, 32)) != MOE_OK) return rc;
   }
   if ((rc = make_tmap_bf16(&tmB, B, K, static_cast<uint64_t>(G) * n_per_group, 128)) != MOE_OK)
     return rc;
@@ -252,14 +255,14 @@ int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int 
   if (src_rows) {
     auto kern = grouped_gemm_bf16_pair_kernel<EPI, true>;
     if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
-    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
+    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
                                                  static_cast<__nv_bfloat16*>(out), ldo,
                                                  static_cast<__nv_bfloat16*>(ac), src_rows,
                                                  counter, di->status);
   } else {
     auto kern = grouped_gemm_bf16_pair_kernel<EPI, false>;
     if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
-    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
+    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
                                                  static_cast<__nv_bfloat16*>(out), ldo,
                                                  static_cast<__nv_bfloat16*>(ac), nullptr,
                                                  counter, di->status);
