@@ -18,6 +18,7 @@ page, deepseekmodel.com, MTP listing: hidden size 7168):
   v3p_fp8      v3p inputs; FP8 E4M3 expert weights (128x128 blocks) and
                activations (1x128 tiles)
   v3p_small    profiling-size case with the V3 expert shapes: T=4096, 32 experts
+  v3p_small_fp8  the same in the FP8 variant
 
 Distributions: u ~ N(0,1); centroids and all expert / shared weights
 ~ N(0, 0.02^2) (0.02 is the standard deviation); every float tensor is drawn
@@ -105,6 +106,10 @@ CONFIGS = {
     "v3p_fp8": MoEConfig("v3p_fp8", T=16384, d=7168, n_routed=256, top_k=8, n_shared=1,
                          inter=2048, routed_scale=2.5, bias_lo=-0.05, bias_hi=0.05, zipf_s=1.1,
                          zipf_alpha=V3P_ZIPF_ALPHA, fp8=True, weights_on_gpu=True),
+    # profiling-size case of the FP8 variant
+    "v3p_small_fp8": MoEConfig("v3p_small_fp8", T=4096, d=7168, n_routed=32, top_k=8,
+                               n_shared=1, inter=2048, routed_scale=2.5, bias_lo=-0.05,
+                               bias_hi=0.05, fp8=True, weights_on_gpu=True),
 }
 
 # Per-tensor seed streams (added to 1000 * cfg.seed).
