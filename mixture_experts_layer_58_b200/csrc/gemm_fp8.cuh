@@ -18,8 +18,9 @@
 //   warp 0      TMA producer: A [128 rows x 128 B] + B [128 rows x 128 B] per stage,
 //               6 stages; takes the tiles in index order from a global counter
 //               and hands each index to the other roles (tileq.cuh).
-//   warp 1      MMA issuer: one K block (4 x K=32) per P buffer, two buffers of
-//               128 TMEM columns.
+//   warp 1      MMA issuer: one K block (4 x K=32) per P buffer, four buffers of
+//               128 TMEM columns (the MMA runs up to three blocks ahead of the
+//               promotion).
 //   warps 2-9   promotion + epilogue. Warp w reads TMEM lane quarter w % 4;
 //               half = (w - 2) / 4 picks its 64 columns: for the up-projection
 //               the gate columns [32*half, +32) and the up columns
@@ -49,7 +50,8 @@ struct GemmF8Cfg {
   static constexpr int kABytes = kBM * kF8BK;
   static constexpr int kBBytes = kF8BN * kF8BK;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTmemCols = 2 * kF8BN;
+  static constexpr int kPBufs = 4;                // P buffers of 128 TMEM columns
+  static constexpr int kTmemCols = kPBufs * kF8BN;
   static constexpr int kBarBytes = 256;
   static size_t smem_bytes(int G) {
     return 1024 + static_cast<size_t>(kF8Stages) * kStageBytes + kBarBytes +
@@ -89,8 +91,8 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + kF8Stages * C::kBBytes);
   uint64_t* empty = full + kF8Stages;
   uint64_t* pfull = empty + kF8Stages;
-  uint64_t* pempty = pfull + 2;
-  uint64_t* mma_done = pempty + 2;
+  uint64_t* pempty = pfull + C::kPBufs;
+  uint64_t* mma_done = pempty + C::kPBufs;
   uint64_t* tq_full = mma_done + 1;
   uint64_t* tq_empty = tq_full + kCtaTileQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kCtaTileQ);
@@ -110,7 +112,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         mbar_init(&full[s], 1);
         mbar_init(&empty[s], 1);
       }
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < C::kPBufs; ++b) {
         mbar_init(&pfull[b], 1);
         mbar_init(&pempty[b], kF8EpiThreads);
       }
@@ -206,8 +208,8 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
           t >= total_tiles)
         break;
       for (int kb = 0; kb < num_kb; ++kb, ++kcount) {
-        const uint32_t pb = kcount & 1u;
-        const uint32_t ppar = (kcount >> 1) & 1u;
+        const uint32_t pb = kcount % C::kPBufs;
+        const uint32_t ppar = (kcount / C::kPBufs) & 1u;
         if (!mbar_wait(&pempty[pb], ppar ^ 1u, status, kStatusTimeoutMma) ||
             !mbar_wait(&full[stage], phase, status, kStatusTimeoutMma)) {
           ok = false;
@@ -289,8 +291,8 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
           w0_n = __ldg(sw0 + kb + 1);
           w1_n = __ldg(sw1 + kb + 1);
         }
-        const uint32_t pb = kcount & 1u;
-        const uint32_t ppar = (kcount >> 1) & 1u;
+        const uint32_t pb = kcount % C::kPBufs;
+        const uint32_t ppar = (kcount / C::kPBufs) & 1u;
         if (!broken && !mbar_wait(&pfull[pb], ppar, status, kStatusTimeoutEpilogue)) broken = true;
         tc_fence_after();
         const uint32_t taddr = tmem_base + pb * kF8BN + lane_addr;
