@@ -201,7 +201,7 @@ MOE_API int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, in
  * logical row r of x is row src_token[r] of u [T, d] (bf16, 16-B aligned),
  * read by the kernel itself (TMA gather, four rows per load). src_token,
  * group_offsets: from moe_permute_index. Removes the expert-contiguous copy
- * of the dispatch (the "fused gather" of the build plan). */
+ * of the dispatch: the dispatch then moves no token rows. */
 MOE_API int moe_expert_up_swiglu_gather(const void* u, int T, const int32_t* src_token,
                                         const int32_t* group_offsets, int G, int rows, int d,
                                         int inter, const void* w13, void* h,
