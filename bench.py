@@ -367,6 +367,10 @@ def main():
                          "saved pre-activations + backward + bias update (bf16)")
     ap.add_argument("--no-overlap", action="store_true",
                     help="run the shared expert after the routed experts on one stream")
+    ap.add_argument("--parallel", default="dp", choices=["dp", "ep"],
+                    help="dp: every rank holds all experts, its own batch; ep: the routed "
+                         "experts split over the ranks, token rows exchanged by NCCL "
+                         "all-to-all (bf16 forward, five-call mode)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -387,8 +391,20 @@ def main():
     import torch.distributed as dist
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
+    ep_mode = args.parallel == "ep"
+    if ep_mode and (cfg.fp8 or args.mode != "five-call"):
+        raise SystemExit("--parallel ep runs the bf16 five-call forward")
+    if world > 1 or ep_mode:
         from datetime import timedelta
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            if "MASTER_PORT" not in os.environ:
+                import socket
+                with socket.socket() as sk:          # a free port for the one-rank group
+                    sk.bind(("127.0.0.1", 0))
+                    os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     from mixture_experts_layer_58_b200 import _lib as L
@@ -406,10 +422,17 @@ def main():
     e_host, b_host = synth.centroids(cfg), synth.bias(cfg)
     W1, W3, W2 = synth.all_expert_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
     shared = synth.shared_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
-    lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
-                   routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
-                   fp8=cfg.fp8, fused_gather=(args.mode == "fused"),
-                   overlap_shared=not args.no_overlap, device=dev)
+    if ep_mode:
+        from mixture_experts_layer_58_b200.ep import ExpertParallelMoELayer
+        lay = ExpertParallelMoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
+                                     routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
+                                     gamma=cfg.gamma, overlap_shared=not args.no_overlap,
+                                     device=dev)
+    else:
+        lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
+                       routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
+                       fp8=cfg.fp8, fused_gather=(args.mode == "fused"),
+                       overlap_shared=not args.no_overlap, device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
     torch.cuda.empty_cache()
@@ -419,11 +442,14 @@ def main():
     stream = torch.cuda.current_stream()
 
     up_timers = {}
+    recv_rows = []        # rows this rank's experts received, per timed step (ep)
 
     def step(timed=False):
         lay.forward(u, timers=up_timers if timed else None)
+        if ep_mode and timed:
+            recv_rows.append(lay.last_plan.n_recv)
         if cfg.gate_kind == "sigmoid":
-            if world > 1:
+            if world > 1 or ep_mode:
                 lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
             else:
                 lay.update_bias()
@@ -451,7 +477,7 @@ def main():
     ms = t_start.elapsed_time(t_end)
     up_ms = sum(a.elapsed_time(b) for a, b in up_timers["up"]) / args.steps
     stage_ms = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in up_timers.items()}
-    if world > 1:
+    if world > 1 or ep_mode:
         tt = torch.tensor([ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
@@ -494,7 +520,7 @@ def main():
             stream.wait_event(down_done[b])       # o_buf[b] downloaded
             lay.forward(u_buf[b], out=o_buf[b])
             if cfg.gate_kind == "sigmoid":
-                if world > 1:
+                if world > 1 or ep_mode:
                     lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
                 else:
                     lay.update_bias()
@@ -515,7 +541,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
+    if world > 1 or ep_mode:
         tt = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_ms = float(tt.item())
@@ -523,14 +549,17 @@ def main():
 
     # ---- roofline of the dominant kernel (routed up-projection + SwiGLU)
     pk = peaks()
-    up_flops = 2.0 * T * K * d * 2 * I
+    # the routed rows this rank's up-projection processes: its own T*K rows,
+    # or under expert parallelism the rows its experts received
+    up_rows = sum(recv_rows) / len(recv_rows) if recv_rows else T * K
+    up_flops = 2.0 * up_rows * d * 2 * I
     achieved = up_flops / (up_ms * 1e-3) / 1e12
     # an FP8 contraction takes the measured bf16 peak x the nominal fp8/bf16 ratio (2)
     ratio = 2.0 if cfg.fp8 else 1.0
     peak = (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * ratio
     kname = ("grouped_gemm_fp8_kernel<SwiGLU> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
              "grouped_gemm_bf16_pair_kernel<SwiGLU, gather> (moe_expert_up_swiglu_gather)"
-             if lay.fused_gather else
+             if (lay.fused_gather or ep_mode) else
              "grouped_gemm bf16 <SwiGLU>, CTA-pair or 1-CTA tiles by group size "
              "(moe_expert_up_swiglu)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -566,10 +595,13 @@ def main():
         "config": {"workload": cfg.name, "T": T, "d": d, "n_routed": cfg.n_routed, "top_k": K,
                    "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
                    "gate": cfg.gate_kind, "global_batch_tokens": T * world,
-                   "mode": "fused gather" if lay.fused_gather else "five-call",
+                   "mode": ("expert-parallel: NCCL all-to-all dispatch/return, gathered "
+                            "up-projection" if ep_mode else
+                            "fused gather" if lay.fused_gather else "five-call"),
                    "shared_expert": "side stream, overlapped" if lay.overlap_shared
                    else "after the routed experts",
-                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "parallelism": (f"ep{world}" if ep_mode else
+                                   f"dp{world}" if world > 1 else "single"),
                    "l2": "inputs larger than L2 (22.6 GB of expert weights streamed per step)"
                    if cfg.weights_on_gpu else "L2 not flushed: small workload",
                    "max_expert_load": int(counts.max()), "mean_expert_load": T * K / cfg.n_routed},
@@ -578,7 +610,7 @@ def main():
         "layer_frac_of_tensor_peak": layer_tflops / (pk["bf16_tflops"] * ratio),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
-                "d2h_bytes_per_step": T * d * 2, "api": "MoELayer.forward",
+                "d2h_bytes_per_step": T * d * 2, "api": type(lay).__name__ + ".forward",
                 "copies": "pinned host, own stream, overlapped with neighbouring steps"},
         "stage_ms": stage_ms,
         "gpu_launches": args.steps * lay.launches_per_step(),
@@ -600,7 +632,7 @@ def main():
 
     if rank == 0:
         print(json.dumps(result), flush=True)
-    if world > 1:
+    if world > 1 or ep_mode:
         dist.barrier()
         dist.destroy_process_group()
 

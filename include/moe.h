@@ -378,6 +378,55 @@ MOE_API int moe_centroid_grad(const void* x_perm, const float* dz_perm,
                               const int32_t* expert_offsets, int n_routed, int rows, int d,
                               void* de, moe_stream_t stream);
 
+/* ------------------------------------------------------------------ expert parallelism
+ * The routed experts split evenly over W ranks: rank p holds experts
+ * [p*n_local, (p+1)*n_local), n_routed = W*n_local; the centroids, the bias
+ * and the shared expert are replicated. Token rows travel by all-to-all
+ * exchanges (DeepSeek-V3 technical report summary: "Problem setting and
+ * motivation", the all-to-all cost of fine-grained routing; "Main ideas",
+ * DualPipe bullet). One forward on each rank:
+ *   moe_route, moe_permute (local tokens, all n_routed experts)
+ *   counts exchange: rank p receives, from every rank q, the counts of q's
+ *     rows for p's n_local experts -> recv_counts [W, n_local]
+ *   moe_ep_plan (host)
+ *   dispatch exchange: x_perm rows [offsets[p*n_local], offsets[(p+1)*n_local])
+ *     go to rank p (send_splits[p] rows); recv_splits[q] rows arrive from q
+ *   moe_expert_up_swiglu_gather(x_recv, n_recv, regroup, group_offsets,
+ *     n_local, ...), moe_expert_down(..., y_exp)
+ *   moe_gather_rows(y_exp, n_recv, ungroup, n_recv, d, y_src)
+ *   return exchange: y_src back with the splits swapped -> y_perm
+ *   moe_combine (local tokens), as for one GPU.
+ * The collectives are the caller's (NCCL in the binding).
+ *
+ * moe_ep_plan: HOST function on host arrays; launches nothing, touches no
+ * device, may be called without a GPU.
+ *   local_counts [W*n_local] int32: this rank's rows per expert (its
+ *     moe_route counts).
+ *   recv_counts [W, n_local] int32: recv_counts[q*n_local + e] = rows that
+ *     rank q routes to this rank's local expert e.
+ *   Out: send_splits[W], recv_splits[W] (rows to / from each rank);
+ *     group_offsets [n_local+1] int32: expert-major offsets of the received
+ *     rows; *n_recv = their number R. regroup [R] int32: for expert-major row
+ *     j (expert e's rows from rank 0, then rank 1, ...; each rank's rows in
+ *     its token order), its row in the received (source-major) buffer;
+ *     ungroup [R] int32: the inverse. regroup/ungroup may be NULL (splits,
+ *     offsets and R only); otherwise R must be <= recv_capacity.
+ *   Errors: MOE_ERR_INVALID_ARG for a NULL required pointer, W or n_local
+ *   < 1, a negative count, or R > recv_capacity with regroup/ungroup given;
+ *   MOE_ERR_UNSUPPORTED_SHAPE for R >= 2^31. Nothing is written on error.
+ *
+ * moe_gather_rows: dst[i, :] = src[index[i], :] for i < n (bf16 rows of d
+ *   elements; src [n_src, d], dst [n, d], 16-B aligned, d % 8 == 0; index
+ *   [n] int32 device). An index outside [0, n_src) yields a zero row (src is
+ *   never read out of bounds). HBM-bound: reads and writes n*d*2 bytes.
+ */
+MOE_API int moe_ep_plan(const int32_t* local_counts, const int32_t* recv_counts, int world,
+                        int n_local, long long recv_capacity, long long* send_splits,
+                        long long* recv_splits, int32_t* group_offsets, int32_t* regroup,
+                        int32_t* ungroup, long long* n_recv);
+MOE_API int moe_gather_rows(const void* src, int n_src, const int32_t* index, int n, int d,
+                            void* dst, moe_stream_t stream);
+
 /* ------------------------------------------------------------------ helpers
  * moe_pack_w13: build the interleaved w13 [G, 2*inter, d] from w1 and w3
  * [G, inter, d] (all bf16, 16-B aligned; layout described at moe_grouped_ffn).

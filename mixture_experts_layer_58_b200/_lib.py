@@ -79,6 +79,9 @@ _SIGS = {
                                _vp]),
     "moe_combine_dx": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_centroid_grad": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_ep_plan": (_i, [_vp, _vp, _i, _i, _ll, _vp, _vp, _vp, _vp, _vp,
+                         ctypes.POINTER(ctypes.c_longlong)]),
+    "moe_gather_rows": (_i, [_vp, _i, _vp, _i, _i, _vp, _vp]),
 }
 
 _LIB = None
@@ -240,6 +243,39 @@ def moe_bias_update(expert_counts, bias, n_routed, T, top_k, gamma, stream=None)
 def moe_pack_w13(w1, w3, G, inter, d, w13, stream=None):
     _check(_L().moe_pack_w13(_p(w1), _p(w3), G, inter, d, _p(w13), _stream(stream)),
            "moe_pack_w13")
+
+
+def _host(t, dtype_name, where):
+    """Host pointer of a CPU tensor (None -> NULL); moe_ep_plan reads and
+    writes host memory, so a device tensor here is a caller error."""
+    if t is None:
+        return None
+    if t.device.type != "cpu" or not t.is_contiguous() or str(t.dtype) != dtype_name:
+        raise ValueError(f"{where}: expected a contiguous CPU {dtype_name} tensor, got "
+                         f"{t.dtype} on {t.device}")
+    return t.data_ptr()
+
+
+def moe_ep_plan(local_counts, recv_counts, world, n_local, recv_capacity, send_splits,
+                recv_splits, group_offsets, regroup=None, ungroup=None) -> int:
+    """Host plan of one expert-parallel exchange (all arguments CPU tensors:
+    counts int32, splits int64, offsets/regroup/ungroup int32). Returns the
+    number of received rows."""
+    w = "moe_ep_plan"
+    n = ctypes.c_longlong(0)
+    _check(_L().moe_ep_plan(_host(local_counts, "torch.int32", w),
+                            _host(recv_counts, "torch.int32", w), int(world), int(n_local),
+                            int(recv_capacity), _host(send_splits, "torch.int64", w),
+                            _host(recv_splits, "torch.int64", w),
+                            _host(group_offsets, "torch.int32", w),
+                            _host(regroup, "torch.int32", w), _host(ungroup, "torch.int32", w),
+                            ctypes.byref(n)), w)
+    return int(n.value)
+
+
+def moe_gather_rows(src, n_src, index, n, d, dst, stream=None):
+    _check(_L().moe_gather_rows(_p(src), n_src, _p(index), n, d, _p(dst), _stream(stream)),
+           "moe_gather_rows")
 
 
 def moe_get_device_status(clear: bool = True) -> int:

@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["moe.cu"]
 HEADERS = ["ptx.cuh", "gemm.cuh", "route.cuh", "dispatch.cuh", "fp8.cuh", "gemm_fp8.cuh", "gemm2sm.cuh",
-           "gemm_bwd.cuh", "bwd.cuh", "tileq.cuh"]
+           "gemm_bwd.cuh", "bwd.cuh", "tileq.cuh", "ep.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -21,6 +21,7 @@
 #include "route.cuh"
 #include "bwd.cuh"
 #include "gemm_bwd.cuh"
+#include "ep.cuh"
 
 namespace {
 
@@ -742,6 +743,47 @@ int moe_combine(const void* y_perm, const int32_t* pos, const float* topk_gate,
       static_cast<const __nv_bfloat16*>(y_perm), pos, topk_gate,
       static_cast<const __nv_bfloat16*>(shared_out), static_cast<const __nv_bfloat16*>(residual),
       T, d, top_k, static_cast<__nv_bfloat16*>(out));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ expert parallelism
+int moe_ep_plan(const int32_t* local_counts, const int32_t* recv_counts, int world, int n_local,
+                long long recv_capacity, long long* send_splits, long long* recv_splits,
+                int32_t* group_offsets, int32_t* regroup, int32_t* ungroup, long long* n_recv) {
+  if (!local_counts || !recv_counts || !send_splits || !recv_splits || !group_offsets || !n_recv)
+    return MOE_ERR_INVALID_ARG;
+  if (world < 1 || n_local < 1 || static_cast<long long>(world) * n_local > (1LL << 24))
+    return MOE_ERR_INVALID_ARG;
+  if ((regroup || ungroup) && recv_capacity < 0) return MOE_ERR_INVALID_ARG;
+  // validate and size first, so that nothing is written on error
+  long long total = 0;
+  for (long long i = 0; i < static_cast<long long>(world) * n_local; ++i) {
+    if (recv_counts[i] < 0 || local_counts[i] < 0) return MOE_ERR_INVALID_ARG;
+    total += recv_counts[i];
+  }
+  if (total > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((regroup || ungroup) && total > recv_capacity) return MOE_ERR_INVALID_ARG;
+  const long long r = ep_plan_host(local_counts, recv_counts, world, n_local, recv_capacity,
+                                   send_splits, recv_splits, group_offsets, regroup, ungroup);
+  if (r < 0) return MOE_ERR_INVALID_ARG;
+  *n_recv = r;
+  return MOE_OK;
+}
+
+int moe_gather_rows(const void* src, int n_src, const int32_t* index, int n, int d, void* dst,
+                    moe_stream_t stream) {
+  if (n < 0 || n_src < 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return MOE_OK;
+  if (!src || !index || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int blocks = std::max(1, std::min((n + 7) / 8, di->num_sms * 8));
+  gather_rows_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(src), n_src, index, n, d,
+      static_cast<__nv_bfloat16*>(dst));
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

@@ -1,0 +1,265 @@
+"""Expert parallelism of the DeepSeekMoE layer: W ranks, one per GPU.
+
+Rank p holds the routed experts [p*n_local, (p+1)*n_local) (n_routed =
+W*n_local); the centroids, the bias and the shared expert are replicated.
+Fine-grained routing sends each token to up to K experts on other GPUs, and
+the token rows travel by all-to-all exchanges (DeepSeek-V3 technical report
+summary: "Problem setting and motivation", the all-to-all cost of
+fine-grained routing; "Main ideas", DualPipe bullet; "Limitations", the SMs
+given to the all-to-all).
+
+One forward on every rank, over its own batch of tokens:
+
+    moe_route, moe_permute      its tokens, all n_routed experts
+    counts exchange             all-to-all of the n_routed loads
+                                -> recv_counts [W, n_local]
+    moe_ep_plan (host)          split sizes, expert-major grouping of the
+                                received rows and its inverse
+    dispatch exchange           all-to-all of the x_perm rows
+    up-projection               reads the received rows expert-major through
+                                the plan's regroup index (no copy)
+    down-projection
+    moe_gather_rows             back to the received order
+    return exchange             all-to-all back -> y_perm in x_perm order
+    moe_combine                 its tokens, as on one GPU
+
+The shared expert runs on a side stream on the rank's own tokens. The bias
+update needs the loads of the whole step: the counts are summed over the ranks
+(dp.sync_load) before every rank applies the same update.
+
+The exchanges are NCCL collectives (torch.distributed) between the library's
+kernels; the host plan needs the split sizes, so a step reads 2*n_routed
+int32 back to the host once. The stage methods (begin, plan, experts,
+finish) let a caller put its own transport between them.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+import torch.distributed as dist
+
+from . import _lib as L
+from . import dp
+from .layer import MoELayer, _Timed
+
+
+@dataclass
+class ExchangePlan:
+    """Host plan of one exchange, seen from one rank (moe_ep_plan's outputs)."""
+    send_splits: list      # rows to each rank (x_perm blocks, rank order)
+    recv_splits: list      # rows from each rank
+    n_recv: int            # rows received
+    group_offsets: torch.Tensor  # [n_local + 1] int32 (CPU): expert-major offsets
+    regroup: torch.Tensor  # [n_recv] int32 (CPU): expert-major row -> received row
+    ungroup: torch.Tensor  # [n_recv] int32 (CPU): received row -> expert-major row
+
+
+def plan_exchange(local_counts: torch.Tensor, recv_counts: torch.Tensor, world: int,
+                  n_local: int) -> ExchangePlan:
+    """The plan of one exchange from this rank's loads (local_counts
+    [world*n_local] int32) and the loads every rank routes to this rank's
+    experts (recv_counts [world, n_local] int32); both CPU tensors."""
+    local_counts = local_counts.to(torch.int32).contiguous()
+    recv_counts = recv_counts.to(torch.int32).contiguous()
+    n = int(recv_counts.sum())
+    ss = torch.empty(world, dtype=torch.int64)
+    rs = torch.empty(world, dtype=torch.int64)
+    go = torch.empty(n_local + 1, dtype=torch.int32)
+    rg = torch.empty(max(n, 1), dtype=torch.int32)
+    ug = torch.empty(max(n, 1), dtype=torch.int32)
+    got = L.moe_ep_plan(local_counts, recv_counts, world, n_local, n, ss, rs, go, rg, ug)
+    assert got == n
+    return ExchangePlan(ss.tolist(), rs.tolist(), n, go, rg[:n], ug[:n])
+
+
+def exchange_counts(counts: torch.Tensor, group=None) -> torch.Tensor:
+    """All-to-all of the per-expert loads [world*n_local] int32: chunk p of
+    this rank's counts goes to rank p; chunk q of the result is what rank q
+    routes to this rank's experts."""
+    out = torch.empty_like(counts)
+    dist.all_to_all_single(out, counts, group=group)
+    return out
+
+
+def dispatch_rows(x_perm: torch.Tensor, plan: ExchangePlan, out: torch.Tensor,
+                  group=None) -> torch.Tensor:
+    """All-to-all of the expert-contiguous token rows: x_perm's block of rows
+    for rank p's experts goes to rank p; the rows received land in
+    out[:n_recv], source-major."""
+    rows = sum(plan.send_splits)
+    dst = out[:plan.n_recv]
+    dist.all_to_all_single(dst, x_perm[:rows], output_split_sizes=plan.recv_splits,
+                           input_split_sizes=plan.send_splits, group=group)
+    return dst
+
+
+def return_rows(y_src: torch.Tensor, plan: ExchangePlan, out: torch.Tensor,
+                group=None) -> torch.Tensor:
+    """All-to-all back: the expert outputs of the rows received from rank q
+    (in the order received) return to rank q, landing in x_perm order."""
+    rows = sum(plan.send_splits)
+    dst = out[:rows]
+    dist.all_to_all_single(dst, y_src[:plan.n_recv], output_split_sizes=plan.send_splits,
+                           input_split_sizes=plan.recv_splits, group=group)
+    return dst
+
+
+class ExpertParallelMoELayer(MoELayer):
+    """A DeepSeekMoE layer whose routed experts are split over the ranks of
+    `group` (bf16 forward). w1, w3 [·, I, d] and w2 [·, d, I] are either all
+    n_routed experts (this rank keeps its slice) or only this rank's n_local.
+    world/rank default to the group's; give them explicitly to build one
+    rank's layer without a process group (the ranks then exchange through the
+    caller's own transport between the stage methods)."""
+
+    def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
+                 routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
+                 group=None, world: int | None = None, rank: int | None = None,
+                 overlap_shared: bool = True, device="cuda"):
+        self.group = group
+        self.world = dist.get_world_size(group) if world is None else int(world)
+        self.rank = dist.get_rank(group) if rank is None else int(rank)
+        n_routed = centroids.shape[0]
+        if n_routed % self.world:
+            raise ValueError(f"{n_routed} routed experts do not split over {self.world} ranks")
+        self.n_local = n_routed // self.world
+        self.expert_lo = self.rank * self.n_local
+        if w1.shape[0] == n_routed and self.n_local != n_routed:
+            sl = slice(self.expert_lo, self.expert_lo + self.n_local)
+            w1, w3, w2 = w1[sl], w3[sl], w2[sl]
+        if w1.shape[0] != self.n_local:
+            raise ValueError(f"expected {self.n_local} or {n_routed} experts, got {w1.shape[0]}")
+        super().__init__(centroids, bias, w1, w3, w2, shared, top_k=top_k,
+                         routed_scale=routed_scale, gate_kind=gate_kind, gamma=gamma,
+                         overlap_shared=overlap_shared, device=device)
+        self._cap = -1
+
+    # ------------------------------------------------------------------ buffers
+    def _ensure_recv(self, n: int) -> None:
+        """Grow-only buffers for n received rows (rounded up to 256 rows)."""
+        if n <= self._cap:
+            return
+        cap = max(256, (n + 255) // 256 * 256)
+        dev, bf, d = self.device, torch.bfloat16, self.d
+        self.x_recv = torch.empty((cap, d), dtype=bf, device=dev)
+        self.h_recv = torch.empty((cap, self.inter), dtype=bf, device=dev)
+        self.y_exp = torch.empty((cap, d), dtype=bf, device=dev)
+        self.y_src = torch.empty((cap, d), dtype=bf, device=dev)
+        # group offsets, regroup, ungroup: one pinned host block, one copy
+        self._idx_host = torch.empty(self.n_local + 1 + 2 * cap, dtype=torch.int32,
+                                     pin_memory=True)
+        self._idx_dev = torch.empty(self.n_local + 1 + 2 * cap, dtype=torch.int32, device=dev)
+        self._cap = cap
+
+    # ------------------------------------------------------------------ stages
+    def begin(self, u, timers=None):
+        """Route and dispatch-copy this rank's tokens (and start the shared
+        expert on the side stream). Leaves the loads in self.counts."""
+        assert u.dtype == torch.bfloat16 and u.is_contiguous() and u.device.type == "cuda"
+        T = u.shape[0]
+        self.allocate(T)
+        ev = _Timed(timers)
+        self._side_used = False
+        if T > 0 and self.ws13 is not None and self.overlap_shared:
+            side = self._fork()
+            u.record_stream(side)
+            with torch.cuda.stream(side):
+                with ev("shared"):
+                    self.shared_ffn(u)
+            self._join_event.record(side)
+            self._side_used = True
+        with ev("route"):
+            self.route(u)
+        if T > 0:
+            with ev("permute"):
+                self.permute(u)
+
+    def plan(self, local_counts: torch.Tensor, recv_counts: torch.Tensor) -> ExchangePlan:
+        """Host plan from CPU loads; uploads its indices (one copy on the
+        current stream) and sizes the receive buffers."""
+        p = plan_exchange(local_counts, recv_counts.view(self.world, self.n_local), self.world,
+                          self.n_local)
+        self._ensure_recv(p.n_recv)
+        nl, n = self.n_local, p.n_recv
+        h = self._idx_host
+        h[:nl + 1] = p.group_offsets
+        h[nl + 1:nl + 1 + n] = p.regroup
+        h[nl + 1 + n:nl + 1 + 2 * n] = p.ungroup
+        self._idx_dev[:nl + 1 + 2 * n].copy_(h[:nl + 1 + 2 * n], non_blocking=True)
+        self._goff = self._idx_dev[:nl + 1]
+        self._regroup = self._idx_dev[nl + 1:nl + 1 + n]
+        self._ungroup = self._idx_dev[nl + 1 + n:nl + 1 + 2 * n]
+        return p
+
+    def experts(self, plan: ExchangePlan, x_recv=None, timers=None) -> torch.Tensor:
+        """This rank's experts on the received rows (x_recv, default
+        self.x_recv); returns their outputs in the order received."""
+        n = plan.n_recv
+        x = self.x_recv if x_recv is None else x_recv
+        ev = _Timed(timers)
+        if n > 0:
+            with ev("up"):
+                L.moe_expert_up_swiglu_gather(x, n, self._regroup, self._goff, self.n_local, n,
+                                              self.d, self.inter, self.w13, self.h_recv)
+            with ev("down"):
+                L.moe_expert_down(self.h_recv, self._goff, self.n_local, n, self.inter, self.d,
+                                  self.w2, self.y_exp)
+            with ev("regather"):
+                L.moe_gather_rows(self.y_exp, n, self._ungroup, n, self.d, self.y_src)
+        return self.y_src[:n]
+
+    def finish(self, u, residual: bool = True, out=None, timers=None):
+        """Combine this rank's tokens from self.y_perm (x_perm order)."""
+        T = u.shape[0]
+        dst = self.out if out is None else out
+        assert dst.shape == (T, self.d) and dst.dtype == torch.bfloat16 and dst.is_contiguous()
+        ev = _Timed(timers)
+        if T > 0:
+            if self._side_used:
+                torch.cuda.current_stream().wait_event(self._join_event)
+            elif self.ws13 is not None:
+                with ev("shared"):
+                    self.shared_ffn(u)
+            with ev("combine"):
+                self.combine(u, residual, dst)
+        return dst
+
+    # ------------------------------------------------------------------ forward
+    def forward(self, u, residual: bool = True, out=None, train: bool = False, timers=None):
+        """h' for this rank's tokens u [T, d] (bf16, device). Every rank of
+        the group must call it (the exchanges are collectives), with any T."""
+        if train:
+            raise ValueError("the expert-parallel layer runs the forward only")
+        self.begin(u, timers)
+        ev = _Timed(timers)
+        with ev("exchange_counts"):
+            recv = exchange_counts(self.counts, self.group)
+        loads = torch.cat([self.counts, recv]).cpu()
+        p = self.plan(loads[:self.n_routed], loads[self.n_routed:])
+        with ev("dispatch"):
+            dispatch_rows(self.x_perm, p, self.x_recv, self.group)
+        y_src = self.experts(p, timers=timers)
+        with ev("return"):
+            return_rows(y_src, p, self.y_perm, self.group)
+        self.last_plan = p
+        return self.finish(u, residual, out, timers)
+
+    def step(self, u):
+        """forward, then the bias update from the loads summed over the ranks."""
+        out = self.forward(u)
+        if self.gate_kind == "sigmoid":
+            c = self.counts.clone()
+            T_all = dp.sync_load(c, u.shape[0], self.group)
+            self.update_bias(c, T_all)
+        return out
+
+    # route (1 + a memset), permute (3), up, down, regather, shared FFN (2),
+    # combine; the exchanges are NCCL's
+    def launches_per_step(self) -> int:
+        n = 1 + 3 + 3 + 1
+        if self.ws13 is not None:
+            n += 2
+        if self.gate_kind == "sigmoid":
+            n += 1
+        return n

@@ -184,6 +184,17 @@ def test_fused_gather_entry_points_reject_bad_arguments(lib):
         L.MOE_ERR_INVALID_ARG
 
 
+def test_gather_rows_rejects_bad_arguments(lib):
+    assert lib.moe_gather_rows(A, 10, A, -1, 256, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(A, -1, A, 4, 256, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(A, 10, A, 4, 0, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(A, 10, A, 4, 12, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_gather_rows(MIS, 10, A, 4, 256, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(A, 10, A, 4, 256, MIS, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(A, 10, None, 4, 256, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(A, 10, A, 0, 256, A, None) == L.MOE_OK     # nothing to do
+
+
 def test_selftest_rejects_bad_limit(lib):
     assert lib.moe_selftest_wait_timeout(0, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_wait_timeout(20000, None) == L.MOE_ERR_INVALID_ARG
