@@ -559,7 +559,7 @@ def main():
     peak = (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * ratio
     kname = ("grouped_gemm_fp8_kernel<SwiGLU> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
              "grouped_gemm_bf16_pair_kernel<SwiGLU, gather> (moe_expert_up_swiglu_gather)"
-             if (lay.fused_gather or ep_mode) else
+             if lay.fused_gather else
              "grouped_gemm bf16 <SwiGLU>, CTA-pair or 1-CTA tiles by group size "
              "(moe_expert_up_swiglu)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -595,8 +595,8 @@ def main():
         "config": {"workload": cfg.name, "T": T, "d": d, "n_routed": cfg.n_routed, "top_k": K,
                    "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
                    "gate": cfg.gate_kind, "global_batch_tokens": T * world,
-                   "mode": ("expert-parallel: NCCL all-to-all dispatch/return, gathered "
-                            "up-projection" if ep_mode else
+                   "mode": ("expert-parallel: NCCL all-to-all dispatch/return, rows "
+                            "regrouped by expert on the receiving rank" if ep_mode else
                             "fused gather" if lay.fused_gather else "five-call"),
                    "shared_expert": "side stream, overlapped" if lay.overlap_shared
                    else "after the routed experts",

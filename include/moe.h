@@ -391,8 +391,10 @@ MOE_API int moe_centroid_grad(const void* x_perm, const float* dz_perm,
  *   moe_ep_plan (host)
  *   dispatch exchange: x_perm rows [offsets[p*n_local], offsets[(p+1)*n_local])
  *     go to rank p (send_splits[p] rows); recv_splits[q] rows arrive from q
- *   moe_expert_up_swiglu_gather(x_recv, n_recv, regroup, group_offsets,
- *     n_local, ...), moe_expert_down(..., y_exp)
+ *   moe_gather_rows(x_recv, n_recv, regroup, n_recv, d, x_exp)
+ *   moe_expert_up_swiglu(x_exp, group_offsets, n_local, n_recv, ...),
+ *     moe_expert_down(..., y_exp)   (or moe_expert_up_swiglu_gather on
+ *     x_recv with regroup as src_token, which skips the copy but is slower)
  *   moe_gather_rows(y_exp, n_recv, ungroup, n_recv, d, y_src)
  *   return exchange: y_src back with the splits swapped -> y_perm
  *   moe_combine (local tokens), as for one GPU.

@@ -16,10 +16,9 @@ One forward on every rank, over its own batch of tokens:
     moe_ep_plan (host)          split sizes, expert-major grouping of the
                                 received rows and its inverse
     dispatch exchange           all-to-all of the x_perm rows
-    up-projection               reads the received rows expert-major through
-                                the plan's regroup index (no copy)
-    down-projection
-    moe_gather_rows             back to the received order
+    moe_gather_rows             the received rows, expert-major (regroup)
+    up-projection, down-projection
+    moe_gather_rows             back to the received order (ungroup)
     return exchange             all-to-all back -> y_perm in x_perm order
     moe_combine                 its tokens, as on one GPU
 
@@ -142,10 +141,13 @@ class ExpertParallelMoELayer(MoELayer):
             return
         cap = max(256, (n + 255) // 256 * 256)
         dev, bf, d = self.device, torch.bfloat16, self.d
+        # two row buffers, reused in stream order: x_recv holds the received
+        # rows, then the expert-major down-projection output; y_src holds the
+        # expert-major copy of the received rows, then the outputs in the
+        # order received
         self.x_recv = torch.empty((cap, d), dtype=bf, device=dev)
-        self.h_recv = torch.empty((cap, self.inter), dtype=bf, device=dev)
-        self.y_exp = torch.empty((cap, d), dtype=bf, device=dev)
         self.y_src = torch.empty((cap, d), dtype=bf, device=dev)
+        self.h_recv = torch.empty((cap, self.inter), dtype=bf, device=dev)
         # group offsets, regroup, ungroup: one pinned host block, one copy
         self._idx_host = torch.empty(self.n_local + 1 + 2 * cap, dtype=torch.int32,
                                      pin_memory=True)
@@ -199,14 +201,20 @@ class ExpertParallelMoELayer(MoELayer):
         x = self.x_recv if x_recv is None else x_recv
         ev = _Timed(timers)
         if n > 0:
+            # The rows are copied into expert-major order rather than read in
+            # place by the gathered up-projection: that form is bound by its
+            # TMA request rate, the copy by HBM bandwidth (far cheaper).
+            x_exp, y_exp = self.y_src, self.x_recv
+            with ev("regroup"):
+                L.moe_gather_rows(x, n, self._regroup, n, self.d, x_exp)
             with ev("up"):
-                L.moe_expert_up_swiglu_gather(x, n, self._regroup, self._goff, self.n_local, n,
-                                              self.d, self.inter, self.w13, self.h_recv)
+                L.moe_expert_up_swiglu(x_exp, self._goff, self.n_local, n, self.d, self.inter,
+                                       self.w13, self.h_recv)
             with ev("down"):
                 L.moe_expert_down(self.h_recv, self._goff, self.n_local, n, self.inter, self.d,
-                                  self.w2, self.y_exp)
-            with ev("regather"):
-                L.moe_gather_rows(self.y_exp, n, self._ungroup, n, self.d, self.y_src)
+                                  self.w2, y_exp)
+            with ev("ungroup"):
+                L.moe_gather_rows(y_exp, n, self._ungroup, n, self.d, self.y_src)
         return self.y_src[:n]
 
     def finish(self, u, residual: bool = True, out=None, timers=None):
@@ -254,10 +262,10 @@ class ExpertParallelMoELayer(MoELayer):
             self.update_bias(c, T_all)
         return out
 
-    # route (1 + a memset), permute (3), up, down, regather, shared FFN (2),
-    # combine; the exchanges are NCCL's
+    # route (1 + a memset), permute (3), regroup, up, down, ungroup, shared
+    # FFN (2), combine; the exchanges are NCCL's
     def launches_per_step(self) -> int:
-        n = 1 + 3 + 3 + 1
+        n = 1 + 3 + 4 + 1
         if self.ws13 is not None:
             n += 2
         if self.gate_kind == "sigmoid":
