@@ -147,3 +147,17 @@ def test_emulated_ranks_reproduce_the_single_process_layer(world, Ts):
     for u, r, out in zip(us, routes, outs):
         ref = om.layer_output(u, r.idx, r.gate, expert, shared)
         np.testing.assert_allclose(out, ref, rtol=1e-9, atol=1e-9)
+
+
+def test_layer_rejects_an_uneven_split_and_a_wrong_expert_count():
+    """Raised on the host before any device memory is touched."""
+    from mixture_experts_layer_58_b200.ep import ExpertParallelMoELayer
+    cfg = synth.CONFIGS["tiny"]                 # 16 routed experts
+    e, b = synth.centroids(cfg), synth.bias(cfg)
+    W1, W3, W2 = synth.all_expert_weights(cfg, "cpu")
+    with pytest.raises(ValueError, match="do not split"):
+        ExpertParallelMoELayer(e, b, W1, W3, W2, top_k=4, routed_scale=1.0, world=3, rank=0)
+    with pytest.raises(ValueError, match="expected 8 or 16 experts"):
+        ExpertParallelMoELayer(e, b, W1[:5], W3[:5], W2[:5], top_k=4, routed_scale=1.0,
+                               world=2, rank=1)
+
