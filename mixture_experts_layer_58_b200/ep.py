@@ -133,6 +133,7 @@ class ExpertParallelMoELayer(MoELayer):
                          routed_scale=routed_scale, gate_kind=gate_kind, gamma=gamma,
                          overlap_shared=overlap_shared, device=device)
         self._cap = -1
+        self._idx_copied = None   # event after the last upload of the plan's indices
 
     # ------------------------------------------------------------------ buffers
     def _ensure_recv(self, n: int) -> None:
@@ -182,6 +183,11 @@ class ExpertParallelMoELayer(MoELayer):
         current stream) and sizes the receive buffers."""
         p = plan_exchange(local_counts, recv_counts.view(self.world, self.n_local), self.world,
                           self.n_local)
+        if self._idx_copied is not None:
+            # the previous upload must have left the pinned block before it
+            # is rewritten (forward's host read already guarantees it; a
+            # caller driving the stages itself may not)
+            self._idx_copied.synchronize()
         self._ensure_recv(p.n_recv)
         nl, n = self.n_local, p.n_recv
         h = self._idx_host
@@ -189,6 +195,9 @@ class ExpertParallelMoELayer(MoELayer):
         h[nl + 1:nl + 1 + n] = p.regroup
         h[nl + 1 + n:nl + 1 + 2 * n] = p.ungroup
         self._idx_dev[:nl + 1 + 2 * n].copy_(h[:nl + 1 + 2 * n], non_blocking=True)
+        if self._idx_copied is None:
+            self._idx_copied = torch.cuda.Event()
+        self._idx_copied.record()
         self._goff = self._idx_dev[:nl + 1]
         self._regroup = self._idx_dev[nl + 1:nl + 1 + n]
         self._ungroup = self._idx_dev[nl + 1 + n:nl + 1 + 2 * n]
