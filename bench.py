@@ -563,7 +563,9 @@ def main():
              "grouped_gemm bf16 <SwiGLU>, CTA-pair or 1-CTA tiles by group size "
              "(moe_expert_up_swiglu)")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(cfg.name),
+                "frac": achieved / peak,
+                # the recorded counters are those of the single-GPU launch
+                "traffic": None if ep_mode else recorded_traffic(cfg.name),
                 "kernel": kname, "kernel_ms": up_ms,
                 "peak_source": f"{pk['_source']} bf16_tflops_sustained"
                                + (" x 2 (nominal fp8/bf16)" if cfg.fp8 else "")}
