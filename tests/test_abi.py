@@ -237,3 +237,22 @@ def test_backward_entry_points_reject_bad_arguments(lib):
     assert lib.moe_combine_dx(A, A, A, A, None, A, A, 64, 256, 4, A, None) == E
     assert lib.moe_centroid_grad(A, A, A, 16, 256, 250, A, None) == U
     assert lib.moe_centroid_grad(A, None, A, 16, 256, 256, A, None) == E
+
+
+def test_header_is_c99_and_the_library_links_from_c(lib, tmp_path):
+    """A plain C program includes moe.h, links libmoe.so and calls the entry
+    points that need no GPU (tests/c_abi_check.c)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "c_abi_check"
+    pkg = os.path.dirname(L.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe),
+                    "-L", pkg, "-l:libmoe.so", "-Wl,-rpath," + pkg], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
+
