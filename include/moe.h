@@ -162,7 +162,10 @@ MOE_API int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
  *
  * Group g owns rows [group_offsets[g], group_offsets[g+1]) of x and its own
  * weights. group_offsets is a DEVICE array of G+1 non-decreasing int32 with
- * group_offsets[G] <= rows (rows outside every group are not written).
+ * 0 <= group_offsets[0] and group_offsets[G] <= rows (rows outside every group
+ * are not written). Being on the device, it is not checked by the host:
+ * offsets outside that contract are undefined behaviour (moe_permute's
+ * expert_offsets always meet it).
  *
  *   x      [rows, d] bf16, 16-B aligned.
  *   w13    [G, 2*inter, d] bf16, 16-B aligned: W1 and W3 of each group,
