@@ -132,3 +132,62 @@ def test_round_bf16_matches_torch_cast():
     x32 = x.astype(np.float32)
     want = torch.from_numpy(x32).to(torch.bfloat16).float().numpy()
     assert np.array_equal(fp8.round_bf16(x32), want)
+
+
+def _torch_fp8_dequant(x32: torch.Tensor, rows_per_block: int) -> torch.Tensor:
+    """Quantise fp32 x [r, c] to E4M3 with torch's own float8_e4m3fn cast,
+    one scale max|x|/448 (fp32; 1 for an all-zero block) per
+    rows_per_block x 128 block, and return the dequantised values in fp64."""
+    r, c = x32.shape
+    b = x32.reshape(r // rows_per_block, rows_per_block, c // 128, 128)
+    amax = b.abs().amax(dim=(1, 3))
+    s = torch.where(amax == 0, torch.ones_like(amax), amax / 448.0)
+    q = (b / s[:, None, :, None]).to(torch.float8_e4m3fn)
+    return (q.to(torch.float64) * s.to(torch.float64)[:, None, :, None]).reshape(r, c)
+
+
+def _torch_ffn_fp8(x32, w1, w3, w2):
+    """The FP8 expert FFN restated with torch primitives: dequantised operands
+    (the promoted per-block sum equals their fp64 product), h in fp64, held
+    in bf16 (via fp32), quantised again per 1x128 tile for the second GEMM."""
+    xd = _torch_fp8_dequant(x32, 1)
+    w1d, w3d, w2d = (_torch_fp8_dequant(torch.from_numpy(w), 128) for w in (w1, w3, w2))
+    a, g = xd @ w1d.T, xd @ w3d.T
+    h = torch.nn.functional.silu(a) * g
+    hb = h.to(torch.float32).to(torch.bfloat16).to(torch.float32)
+    return _torch_fp8_dequant(hb, 1) @ w2d.T
+
+
+def test_fp8_ffn_and_layer_match_a_torch_restatement():
+    """The composition of the FP8 oracle (ffn_fp8, layer_output_fp8) against
+    an independent formulation: torch's E4M3 cast instead of the oracle's
+    encoder, dequantise-then-multiply instead of the promoted block sum.
+    A swapped W1/W3, a transposed scale grid or a missing bf16 rounding of h
+    fails it."""
+    from oracle import moe_oracle as om
+    rng = np.random.default_rng(11)
+    T, d, inter, n_r, K = 24, 256, 384, 4, 2
+    u = rng.standard_normal((T, d)).astype(np.float32)
+    u[3, :128] = 0.0                               # an all-zero tile: scale 1
+    experts = [tuple((0.02 * rng.standard_normal(shape)).astype(np.float32)
+                     for shape in ((inter, d), (inter, d), (d, inter))) for _ in range(n_r)]
+    shared = tuple((0.02 * rng.standard_normal(shape)).astype(np.float32)
+                   for shape in ((inter, d), (inter, d), (d, inter)))
+    u32 = torch.from_numpy(u)
+    # one expert alone
+    uq, us = fp8.quant_act_1x128(u)
+    y_or = fp8.ffn_fp8(uq, us, fp8.quant_expert(*experts[1]))
+    y_t = _torch_ffn_fp8(u32, *experts[1]).numpy()
+    assert np.abs(y_or - y_t).max() <= 1e-12 * np.abs(y_t).max()
+    # the layer: routing from the exact oracle, gates, shared expert, residual
+    e = (0.5 * rng.standard_normal((n_r, d))).astype(np.float32)
+    r = om.route(u, e, None, K, 2.5)
+    qexp = [fp8.quant_expert(*w) for w in experts]
+    out_or = fp8.layer_output_fp8(u, r.idx, r.gate, lambda i: qexp[i], [fp8.quant_expert(*shared)])
+    out_t = u.astype(np.float64) + _torch_ffn_fp8(u32, *shared).numpy()
+    for t in range(T):
+        for k in range(K):
+            i = int(r.idx[t, k])
+            out_t[t] += r.gate[t, k] * _torch_ffn_fp8(u32[t:t + 1], *experts[i]).numpy()[0]
+    assert np.abs(out_or - out_t).max() <= 1e-12 * np.abs(out_t).max()
+
