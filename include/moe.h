@@ -458,7 +458,9 @@ MOE_API int moe_get_device_status(unsigned int* status, int clear);
  * counterpart in the pages. */
 MOE_API int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream);
 
-/* Library version, major*10000 + minor*100 + patch. */
+/* Library version, major*10000 + minor*100 + patch. 0.2.0 (200) adds, over
+ * the forward's five calls of 0.1.0: the FP8 variant, the fused-gather
+ * up-projection, the backward and the expert-parallel entry points. */
 MOE_API int moe_version(void);
 
 #ifdef __cplusplus

@@ -382,7 +382,7 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, unsign
 
 extern "C" {
 
-int moe_version(void) { return 100; }
+int moe_version(void) { return 200; }
 
 int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream) {
   if (limit_ms <= 0 || limit_ms > 10000) return MOE_ERR_INVALID_ARG;
