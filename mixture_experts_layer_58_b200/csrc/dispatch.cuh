@@ -30,16 +30,24 @@ permute_hist_kernel(const int32_t* __restrict__ idx, int T, int K, int n_routed,
 }
 
 // Pass 2: expert offsets (exclusive scan of the counts), then for this chunk
-// the row of every (token, slot): thread e walks the chunk's pairs in token
-// order and hands expert e's rows out in that order (stable).
+// the row of every (token, slot) pair, handed out per expert in pair order
+// (token-major, so the order inside an expert is stable). The chunk's pairs
+// go in rounds of 256, one per thread: within a warp, __match_any_sync ranks
+// the lanes that share an expert; per-warp counts are scanned across the 8
+// warps in shared memory; a running per-expert row carries from round to
+// round, and the chunk's first row per expert comes from the earlier chunks'
+// histograms. Pairs whose expert is outside [0, n_routed) get pos = -1.
 __global__ void __launch_bounds__(256)
 permute_index_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                      const int32_t* __restrict__ hist, int T, int K, int n_routed,
                      int32_t* __restrict__ offsets, int32_t* __restrict__ pos,
                      int32_t* __restrict__ src_token) {
   __shared__ int s_scan[256];
-  __shared__ int s_idx[kPermChunk * kMaxTopK];
+  __shared__ int s_next[256];          // next row of each expert
+  __shared__ int s_wcnt[8][256];       // this round: rows per (warp, expert), then their first row
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
   const int chunk = blockIdx.x;
   const int t0 = chunk * kPermChunk;
   const int n = min(kPermChunk, T - t0) * K;
@@ -59,27 +67,60 @@ permute_index_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict_
     offsets[tid] = excl;
     if (tid == n_routed - 1) offsets[n_routed] = s_scan[tid];
   }
-  int base = excl;
-  if (tid < n_routed)
-    for (int cc = 0; cc < chunk; ++cc) base += hist[static_cast<size_t>(cc) * n_routed + tid];
-
-  int32_t* pos_c = pos + static_cast<size_t>(t0) * K;
-  for (int i = tid; i < n; i += 256) {
-    s_idx[i] = idx[static_cast<size_t>(t0) * K + i];
-    pos_c[i] = -1;
-  }
-  __syncthreads();
   if (tid < n_routed) {
-    int r = base;
-    for (int i = 0; i < n; ++i) {
-      if (s_idx[i] == tid) {
-        if (r >= 0 && r < total) {
-          pos_c[i] = r;
-          src_token[r] = t0 + i / K;
-        }
-        ++r;
-      }
+    // the histogram loads are independent: keep eight in flight
+    int base = excl;
+    int cc = 0;
+    for (; cc + 8 <= chunk; cc += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = hist[static_cast<size_t>(cc + j) * n_routed + tid];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) base += v[j];
     }
+    for (; cc < chunk; ++cc) base += hist[static_cast<size_t>(cc) * n_routed + tid];
+    s_next[tid] = base;
+  }
+
+  const int32_t* idx_c = idx + static_cast<size_t>(t0) * K;
+  int32_t* pos_c = pos + static_cast<size_t>(t0) * K;
+  const unsigned lanes_below = (1u << lane) - 1u;
+  for (int r0 = 0; r0 < n; r0 += 256) {          // same trip count in every thread
+    for (int j = tid; j < 8 * 256; j += 256) (&s_wcnt[0][0])[j] = 0;
+    __syncthreads();
+    const int i = r0 + tid;
+    int e = -1;
+    if (i < n) {
+      e = idx_c[i];
+      if (static_cast<unsigned>(e) >= static_cast<unsigned>(n_routed)) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int before = __popc(peers & lanes_below);
+    if (e >= 0 && before == 0) s_wcnt[warp][e] = __popc(peers);
+    __syncthreads();
+    if (tid < n_routed) {
+      int run = s_next[tid];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const int v = s_wcnt[w][tid];
+        s_wcnt[w][tid] = run;
+        run += v;
+      }
+      s_next[tid] = run;
+    }
+    __syncthreads();
+    if (i < n) {
+      int p = -1;
+      if (e >= 0) {
+        const int row = s_wcnt[warp][e] + before;
+        if (row >= 0 && row < total) {
+          p = row;
+          src_token[row] = t0 + i / K;
+        }
+      }
+      pos_c[i] = p;
+    }
+    __syncthreads();                              // s_wcnt is cleared next round
   }
 }
 
