@@ -68,7 +68,8 @@ def plan_exchange(local_counts: torch.Tensor, recv_counts: torch.Tensor, world: 
     rg = torch.empty(max(n, 1), dtype=torch.int32)
     ug = torch.empty(max(n, 1), dtype=torch.int32)
     got = L.moe_ep_plan(local_counts, recv_counts, world, n_local, n, ss, rs, go, rg, ug)
-    assert got == n
+    if got != n:
+        raise RuntimeError(f"moe_ep_plan counted {got} received rows, expected {n}")
     return ExchangePlan(ss.tolist(), rs.tolist(), n, go, rg[:n], ug[:n])
 
 
