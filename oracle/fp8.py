@@ -17,15 +17,16 @@ E4M3 itself (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
 subnormals, no infinities, S.1111.111 = NaN, largest finite 448) is written
 here from that definition.
 
-Readings (restated in the design doc): activations use 1x128 tiles ([V3]; the
-pseudocode's 128x128 activation blocks are read as garbled); a tile whose
-max is 0 gets scale 1; the scale and the division x/scale are evaluated in
-fp32, the precision the kernels use for that decision, and the fp32 quotient
-is rounded to E4M3 to nearest-even, saturating at +-448; dequantisation
-multiplies by BOTH the activation and the weight scale of each 128-wide K
-block ([V3]; the pseudocode's single scale is read as garbled); the
-intermediate h is held in bf16 between the two expert GEMMs and its codes are
-decided from that value. All other arithmetic is fp64.
+Readings where the pages are silent or garbled: activations use 1x128 tiles
+([V3]; the pseudocode's 128x128 activation blocks are read as garbled); a
+tile whose max is 0 gets scale 1; a value is rounded to fp32 before it is
+quantised, and the scale and the division x/scale are evaluated in fp32 (the
+scales are fp32 numbers), the fp32 quotient rounded to E4M3 to nearest-even,
+saturating at +-448; dequantisation multiplies by BOTH the activation and the
+weight scale of each 128-wide K block ([V3]; the pseudocode's single scale is
+read as garbled); the intermediate h of an expert FFN is quantised from its
+exact value (the pages give it no storage precision of its own). All other
+arithmetic is fp64.
 """
 from __future__ import annotations
 
@@ -93,9 +94,9 @@ def _scale_fp32(amax: np.ndarray) -> np.ndarray:
 def quant_act_1x128(x):
     """Tile-wise activation quantisation ([V3]: 1x128 tiles).
 
-    x [n, k] (k % 128 == 0, values exactly fp32) -> (codes uint8 [n,k],
-    scales fp32 [n, k/128]). Each 128-wide tile of a row: s = max|x|/448,
-    code = E4M3(x / s)."""
+    x [n, k] (k % 128 == 0; rounded to fp32 first, exact for bf16 or fp32
+    input) -> (codes uint8 [n,k], scales fp32 [n, k/128]). Each 128-wide tile
+    of a row: s = max|x|/448, code = E4M3(x / s)."""
     x32 = np.asarray(x, dtype=np.float32)
     n, k = x32.shape
     assert k % BLOCK == 0
@@ -156,24 +157,15 @@ def _as32(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float32)
 
 
-def round_bf16(x) -> np.ndarray:
-    """Round to the nearest bfloat16 (ties to even), via fp32, as fp32 values."""
-    f = np.asarray(x, dtype=np.float32)
-    bits = f.view(np.uint32).astype(np.uint64)
-    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
-    return bits.astype(np.uint32).view(np.float32)
-
-
 def ffn_fp8(xq, xs, qexpert) -> np.ndarray:
     """SwiGLU expert with FP8 operands: a = x W1^T, g = x W3^T (promoted FP8
-    GEMMs), h = silu(a) * g in fp64, h held in bf16 between the two GEMMs (as
-    in the bf16 path) and quantised per 1x128 tile from that value, then
-    y = h W2^T (promoted FP8 GEMM)."""
+    GEMMs), h = silu(a) * g in fp64, quantised per 1x128 tile from that
+    exact value, then y = h W2^T (promoted FP8 GEMM)."""
     (w1q, w1s), (w3q, w3s), (w2q, w2s) = qexpert
     a = fp8_gemm(xq, xs, w1q, w1s)
     g = fp8_gemm(xq, xs, w3q, w3s)
     h = a / (1.0 + np.exp(-a)) * g
-    hq, hs = quant_act_1x128(round_bf16(h))
+    hq, hs = quant_act_1x128(h)
     return fp8_gemm(hq, hs, w2q, w2s)
 
 

@@ -18,7 +18,7 @@ Every input float array is converted to fp64 (the exact value of the bf16 or
 fp32 number it holds) and all arithmetic below is fp64, with no intermediate
 rounding. The only rounding is the bias vector, which is state stored in fp32.
 
-Readings where the pages are silent (each restated in the design doc):
+Readings where the pages are silent:
   * the expert FFN is SwiGLU without biases, W2 (silu(W1 x) * (W3 x));
     the pages never define ExpertFFN  -> parity of the FFN itself is pinned
     only by the dense special case and library identities (tests);

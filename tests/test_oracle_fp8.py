@@ -125,15 +125,6 @@ def test_fp8_ffn_close_to_exact_ffn():
     assert np.abs(y8 - y).mean() <= 0.1 * np.abs(y).mean()
 
 
-def test_round_bf16_matches_torch_cast():
-    rng = np.random.default_rng(7)
-    x = np.concatenate([rng.standard_normal(100000) * 10, rng.standard_normal(1000) * 1e-30,
-                        np.array([1.0, -2.5, 0.0, 65504.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9])])
-    x32 = x.astype(np.float32)
-    want = torch.from_numpy(x32).to(torch.bfloat16).float().numpy()
-    assert np.array_equal(fp8.round_bf16(x32), want)
-
-
 def _torch_fp8_dequant(x32: torch.Tensor, rows_per_block: int) -> torch.Tensor:
     """Quantise fp32 x [r, c] to E4M3 with torch's own float8_e4m3fn cast,
     one scale max|x|/448 (fp32; 1 for an all-zero block) per
@@ -148,22 +139,22 @@ def _torch_fp8_dequant(x32: torch.Tensor, rows_per_block: int) -> torch.Tensor:
 
 def _torch_ffn_fp8(x32, w1, w3, w2):
     """The FP8 expert FFN restated with torch primitives: dequantised operands
-    (the promoted per-block sum equals their fp64 product), h in fp64, held
-    in bf16 (via fp32), quantised again per 1x128 tile for the second GEMM."""
+    (the promoted per-block sum equals their fp64 product), h in fp64,
+    quantised again per 1x128 tile (from its fp32 value: the scale and the
+    quotient are fp32) for the second GEMM."""
     xd = _torch_fp8_dequant(x32, 1)
     w1d, w3d, w2d = (_torch_fp8_dequant(torch.from_numpy(w), 128) for w in (w1, w3, w2))
     a, g = xd @ w1d.T, xd @ w3d.T
     h = torch.nn.functional.silu(a) * g
-    hb = h.to(torch.float32).to(torch.bfloat16).to(torch.float32)
-    return _torch_fp8_dequant(hb, 1) @ w2d.T
+    return _torch_fp8_dequant(h.to(torch.float32), 1) @ w2d.T
 
 
 def test_fp8_ffn_and_layer_match_a_torch_restatement():
     """The composition of the FP8 oracle (ffn_fp8, layer_output_fp8) against
     an independent formulation: torch's E4M3 cast instead of the oracle's
     encoder, dequantise-then-multiply instead of the promoted block sum.
-    A swapped W1/W3, a transposed scale grid or a missing bf16 rounding of h
-    fails it."""
+    A swapped W1/W3, a transposed scale grid or an extra rounding of h fails
+    it (the last is planted in the test below)."""
     from oracle import moe_oracle as om
     rng = np.random.default_rng(11)
     T, d, inter, n_r, K = 24, 256, 384, 4, 2
@@ -191,3 +182,29 @@ def test_fp8_ffn_and_layer_match_a_torch_restatement():
             out_t[t] += r.gate[t, k] * _torch_ffn_fp8(u32[t:t + 1], *experts[i]).numpy()[0]
     assert np.abs(out_or - out_t).max() <= 1e-12 * np.abs(out_t).max()
 
+
+
+def test_planted_bf16_hold_of_h_fails_the_restatement(monkeypatch):
+    """The FP8 oracle quantises h from its exact value (the pages give h no
+    storage precision). Plant the mistake of holding h in bf16 before its
+    1x128 quantisation (an implementation's storage choice) and check that
+    the torch restatement above catches it."""
+    rng = np.random.default_rng(12)
+    d, inter = 256, 384
+    x = rng.standard_normal((24, d)).astype(np.float32)
+    w = tuple((0.02 * rng.standard_normal(shape)).astype(np.float32)
+              for shape in ((inter, d), (inter, d), (d, inter)))
+    xq, xs = fp8.quant_act_1x128(x)
+    qe = fp8.quant_expert(*w)
+    y_t = _torch_ffn_fp8(torch.from_numpy(x), *w).numpy()
+    y_or = fp8.ffn_fp8(xq, xs, qe)
+    assert np.abs(y_or - y_t).max() <= 1e-12 * np.abs(y_t).max()
+    real = fp8.quant_act_1x128
+
+    def quant_of_bf16(v):
+        hb = torch.from_numpy(np.asarray(v, dtype=np.float32)).bfloat16().float().numpy()
+        return real(hb)
+
+    monkeypatch.setattr(fp8, "quant_act_1x128", quant_of_bf16)
+    y_planted = fp8.ffn_fp8(xq, xs, qe)
+    assert np.abs(y_planted - y_t).max() > 1e-6 * np.abs(y_t).max()
