@@ -161,11 +161,15 @@ MOE_API int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
  * biases, FFN(x) = W2 (silu(W1 x) * (W3 x)), is this library's reading).
  *
  * Group g owns rows [group_offsets[g], group_offsets[g+1]) of x and its own
- * weights. group_offsets is a DEVICE array of G+1 non-decreasing int32 with
- * 0 <= group_offsets[0] and group_offsets[G] <= rows (rows outside every group
- * are not written). Being on the device, it is not checked by the host:
- * offsets outside that contract are undefined behaviour (moe_permute's
- * expert_offsets always meet it).
+ * weights. group_offsets is a DEVICE array of G+1 int32, meant to be
+ * non-decreasing with 0 <= group_offsets[0] and group_offsets[G] <= rows
+ * (moe_permute's expert_offsets always are); rows outside every group are not
+ * written. Being on the device it is not checked by the host, but every
+ * kernel that reads it first clamps each entry into [0, rows] and raises it
+ * to the largest entry before it, so a malformed array yields empty or
+ * shortened groups and never a read or write outside x, y or the workspace.
+ * The same holds for the group offsets of every grouped call below (expert
+ * dgrad and wgrad, the FP8 GEMMs, the centroid gradient).
  *
  *   x      [rows, d] bf16, 16-B aligned.
  *   w13    [G, 2*inter, d] bf16, 16-B aligned: W1 and W3 of each group,

@@ -205,15 +205,17 @@ constexpr int kCentroidCols = 256;
 constexpr int kCentroidWarps = 8;
 __global__ void __launch_bounds__(32 * kCentroidWarps)
 centroid_grad_kernel(const __nv_bfloat16* __restrict__ x_perm, const float* __restrict__ dz_perm,
-                     const int32_t* __restrict__ offsets, int d,
+                     const int32_t* __restrict__ offsets, int rows, int d,
                      __nv_bfloat16* __restrict__ de) {
   __shared__ float part[kCentroidWarps][kCentroidCols + 4];
   const int i = blockIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int col = blockIdx.y * kCentroidCols + lane * 8;
-  const int r0 = __ldg(offsets + i);
-  const int r1 = __ldg(offsets + i + 1);
+  // the caller's offsets are clamped into [0, rows] (an empty range if they
+  // decrease), so x_perm is never read outside its rows
+  const int r0 = min(max(__ldg(offsets + i), 0), rows);
+  const int r1 = min(max(__ldg(offsets + i + 1), r0), rows);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (col < d) {
     int r = r0 + warp;

@@ -63,6 +63,59 @@ __device__ __forceinline__ void decode_tile(int t, const int* s_tstart, const in
   m_blk = local - n_blk * mt;
 }
 
+// Group table of a grouped GEMM, built by one warp from the caller's device
+// array offsets[0..G]. The offsets are not trusted: each is clamped into
+// [0, rows] and raised to the running maximum of the ones before it, so the
+// groups [s_off[g], s_end[g]) are disjoint, in order and inside the rows of
+// the operands whatever the array holds (a valid array passes unchanged).
+// With s_tstart, also the first tile of every group (tile_rows-row blocks
+// times tiles_per_mblk column blocks) and the total in s_tstart[G].
+__device__ __forceinline__ void build_group_table(const int32_t* __restrict__ offsets, int G,
+                                                  int rows, int tile_rows, int tiles_per_mblk,
+                                                  int* s_off, int* s_end, int* s_tstart,
+                                                  int lane) {
+  int run = 0;                                   // running maximum of the clamped offsets
+  for (int base = 0; base <= G; base += 32) {
+    const int j = base + lane;
+    int v = 0;
+    if (j <= G) v = min(max(__ldg(offsets + j), 0), rows);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v = max(v, n);
+    }
+    v = max(v, run);
+    if (j <= G) s_off[j] = v;
+    run = __shfl_sync(0xffffffffu, v, 31);
+  }
+  __syncwarp();
+  int carry = 0;
+  for (int base = 0; base < G; base += 32) {
+    const int g = base + lane;
+    int nt = 0;
+    if (g < G) {
+      const int o0 = s_off[g], o1 = s_off[g + 1];
+      s_end[g] = o1;
+      nt = (o1 - o0 + tile_rows - 1) / tile_rows * tiles_per_mblk;
+    }
+    if (s_tstart) {
+      int v = nt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+      }
+      if (g < G) s_tstart[g] = carry + v - nt;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  if (lane == 0) {
+    s_end[G] = s_off[G];
+    if (s_tstart) s_tstart[G] = carry;
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + __expf(-a)); }
 
 template <int BN, int EPI>
@@ -112,31 +165,7 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     tmem_relinquish();
   } else if (warp == 1) {
     // Group table: row offsets and the first tile of every group (warp scan).
-    int carry = 0;
-    for (int base = 0; base < G; base += 32) {
-      const int g = base + lane;
-      int nt = 0;
-      if (g < G) {
-        const int o0 = offsets[g];
-        const int o1 = offsets[g + 1];
-        s_off[g] = o0;
-        s_end[g] = o1 > o0 ? o1 : o0;
-        nt = (o1 > o0 ? (o1 - o0 + kBM - 1) / kBM : 0) * n_blocks_n;
-      }
-      int v = nt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
-      }
-      if (g < G) s_tstart[g] = carry + v - nt;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-    if (lane == 0) {
-      s_tstart[G] = carry;
-      s_off[G] = offsets[G];
-      s_end[G] = offsets[G];
-    }
+    build_group_table(offsets, G, rows, kBM, n_blocks_n, s_off, s_end, s_tstart, lane);
   }
   tc_fence_before();
   __syncthreads();

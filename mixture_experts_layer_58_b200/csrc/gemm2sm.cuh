@@ -302,31 +302,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     tmem_alloc_2sm(tmem_slot, 512);
     tmem_relinquish_2sm();
   } else if (warp == 1) {
-    int carry = 0;
-    for (int base = 0; base < G; base += 32) {
-      const int g = base + lane;
-      int nt = 0;
-      if (g < G) {
-        const int o0 = offsets[g];
-        const int o1 = offsets[g + 1];
-        s_off[g] = o0;
-        s_end[g] = o1 > o0 ? o1 : o0;
-        nt = (o1 > o0 ? (o1 - o0 + kBM2 - 1) / kBM2 : 0) * n_blocks_n;
-      }
-      int v = nt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
-      }
-      if (g < G) s_tstart[g] = carry + v - nt;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-    if (lane == 0) {
-      s_tstart[G] = carry;
-      s_off[G] = offsets[G];
-      s_end[G] = offsets[G];
-    }
+    build_group_table(offsets, G, rows, kBM2, n_blocks_n, s_off, s_end, s_tstart, lane);
   }
   tc_fence_before();
   __syncthreads();

@@ -50,38 +50,6 @@ struct BwdCfg {
 
 __device__ __forceinline__ float sigmoid_f32(float a) { return 1.0f / (1.0f + __expf(-a)); }
 
-// Group table shared by both kernels: s_off/s_end from offsets, and for the
-// dgrad kernel the first tile of every group (row tiles of 128 x n blocks).
-__device__ __forceinline__ void build_group_table(const int32_t* offsets, int G, int tiles_per_mblk,
-                                                  int* s_off, int* s_end, int* s_tstart,
-                                                  int lane) {
-  int carry = 0;
-  for (int base = 0; base < G; base += 32) {
-    const int g = base + lane;
-    int nt = 0;
-    if (g < G) {
-      const int o0 = offsets[g];
-      const int o1 = offsets[g + 1];
-      s_off[g] = o0;
-      s_end[g] = o1 > o0 ? o1 : o0;
-      nt = (o1 > o0 ? (o1 - o0 + kBM - 1) / kBM : 0) * tiles_per_mblk;
-    }
-    int v = nt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += n;
-    }
-    if (g < G) s_tstart[g] = carry + v - nt;
-    carry += __shfl_sync(0xffffffffu, v, 31);
-  }
-  if (lane == 0) {
-    s_tstart[G] = carry;
-    s_off[G] = offsets[G];
-    s_end[G] = offsets[G];
-  }
-}
-
 // ---------------------------------------------------------------------------
 // dgrad: out[rows of g, n] = sum_k A[row, k] W_g[k, n]; K = w_rows per group.
 // EPI_DG_SWIGLU_BWD: n indexes h columns (N = inter); with ac [rows, 2*inter]
@@ -143,7 +111,7 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   } else if (warp == 1) {
-    build_group_table(offsets, G, n_blocks_n, s_off, s_end, s_tstart, lane);
+    build_group_table(offsets, G, rows, kBM, n_blocks_n, s_off, s_end, s_tstart, lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -390,12 +358,7 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   } else if (warp == 1) {
-    for (int g = lane; g < G; g += 32) {
-      const int o0 = offsets[g];
-      const int o1 = offsets[g + 1];
-      s_off[g] = o0;
-      s_end[g] = min(o1 > o0 ? o1 : o0, rows);
-    }
+    build_group_table(offsets, G, rows, kBM, 0, s_off, s_end, nullptr, lane);
   }
   tc_fence_before();
   __syncthreads();

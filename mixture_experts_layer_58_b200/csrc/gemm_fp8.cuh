@@ -129,31 +129,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   } else if (warp == 1) {
-    int carry = 0;
-    for (int base = 0; base < G; base += 32) {
-      const int g = base + lane;
-      int nt = 0;
-      if (g < G) {
-        const int o0 = offsets[g];
-        const int o1 = offsets[g + 1];
-        s_off[g] = o0;
-        s_end[g] = o1 > o0 ? o1 : o0;
-        nt = (o1 > o0 ? (o1 - o0 + kBM - 1) / kBM : 0) * n_blocks_n;
-      }
-      int v = nt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
-      }
-      if (g < G) s_tstart[g] = carry + v - nt;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-    if (lane == 0) {
-      s_tstart[G] = carry;
-      s_off[G] = offsets[G];
-      s_end[G] = offsets[G];
-    }
+    build_group_table(offsets, G, rows, kBM, n_blocks_n, s_off, s_end, s_tstart, lane);
   }
   tc_fence_before();
   __syncthreads();

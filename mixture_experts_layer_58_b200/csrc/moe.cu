@@ -961,7 +961,7 @@ int moe_centroid_grad(const void* x_perm, const float* dz_perm, const int32_t* e
   if (rows > 0 && (!x_perm || !dz_perm || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
   dim3 grid(n_routed, (d + kCentroidCols - 1) / kCentroidCols);
   centroid_grad_kernel<<<grid, 32 * kCentroidWarps, 0, as_stream(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x_perm), dz_perm, expert_offsets, d,
+      static_cast<const __nv_bfloat16*>(x_perm), dz_perm, expert_offsets, rows, d,
       static_cast<__nv_bfloat16*>(de));
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
