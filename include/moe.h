@@ -32,6 +32,14 @@
  *     moe_get_device_status() reports after the stream has drained.
  *   - Tokens with index >= T, experts with no tokens and T = 0 are all valid:
  *     an empty batch produces zero counts and enqueues no expert work.
+ *   - Device state: the grouped GEMMs hand out their tiles through one of 256
+ *     device counters per GPU, taken round robin when the call enqueues and
+ *     zeroed on the call's stream just before its kernel. Two launches share
+ *     a counter only if 256 other GEMM launches were enqueued between them,
+ *     so at most 256 GEMM launches may be in flight at once on one device. A
+ *     launch captured into a CUDA graph keeps the counter it took: do not
+ *     replay one graph on two streams at the same time (their launches would
+ *     share counters and skip or repeat tiles).
  *
  * Supported shapes (others return MOE_ERR_UNSUPPORTED_SHAPE):
  *   d % 256 == 0, inter % 128 == 0, 1 <= top_k <= 8, top_k <= n_routed <= 256,

@@ -39,7 +39,8 @@ thread_local int t_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
-  bool ready = false;
+  // set (release) after the fields below; read (acquire) before using them
+  std::atomic<bool> ready{false};
   int num_sms = 0;
   unsigned int* status = nullptr;
   int* tile_counters = nullptr;
@@ -70,16 +71,16 @@ int device_info(DeviceInfo** out) {
   MOE_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_INVALID_ARG;
   DeviceInfo& di = g_dev[dev];
-  if (!di.ready) {
+  if (!di.ready.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!di.ready) {
+    if (!di.ready.load(std::memory_order_relaxed)) {
       MOE_CUDA(cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev));
       void* p = nullptr;
       MOE_CUDA(cudaGetSymbolAddress(&p, g_status));
       di.status = static_cast<unsigned int*>(p);
       MOE_CUDA(cudaGetSymbolAddress(&p, g_tile_counters));
       di.tile_counters = static_cast<int*>(p);
-      di.ready = true;
+      di.ready.store(true, std::memory_order_release);
     }
   }
   *out = &di;
@@ -997,7 +998,9 @@ namespace {
 constexpr int kNoAllocScratchInts = 65536;   // 256 KiB: ceil(T/128) * n_routed <= 65536
 __device__ __align__(256) int32_t g_permute_scratch[kNoAllocScratchInts];
 
-int32_t* g_scratch_ptr[kMaxDevices];          // device address of the array, per device
+// device address of the array, per device; published with release order
+// after the lookup, read with acquire order
+std::atomic<int32_t*> g_scratch_ptr[kMaxDevices];
 std::mutex g_scratch_mu;
 
 // Device address of g_permute_scratch on the current device. In host code the
@@ -1007,15 +1010,18 @@ int scratch_address(int32_t** out) {
   int dev = 0;
   MOE_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_INVALID_ARG;
-  if (!g_scratch_ptr[dev]) {
+  int32_t* ptr = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!ptr) {
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    ptr = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+    if (!ptr) {
       void* p = nullptr;
       MOE_CUDA(cudaGetSymbolAddress(&p, g_permute_scratch));
-      g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+      ptr = static_cast<int32_t*>(p);
+      g_scratch_ptr[dev].store(ptr, std::memory_order_release);
     }
   }
-  *out = g_scratch_ptr[dev];
+  *out = ptr;
   return MOE_OK;
 }
 

@@ -92,3 +92,30 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert ei.value.status == L.MOE_ERR_UNSUPPORTED_SHAPE
     torch.cuda.synchronize()
     assert int(off[0]) == -9          # nothing was launched
+
+
+def _random_routing(T, n, k, seed):
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.argsort(torch.rand(T, n, generator=g), dim=1)[:, :k].to(torch.int32)
+    counts = torch.bincount(idx.flatten().long(), minlength=n).to(torch.int32)
+    u = torch.randn(T, 256, generator=g).bfloat16()
+    return u.cuda(), idx.cuda(), counts.cuda()
+
+
+def test_noalloc_at_its_largest_accepted_size():
+    # ceil(32768/128) * 256 = 65536 histogram entries: exactly the scratch
+    # array, every entry of it used; one token more is refused
+    T, d, n, k = 32768, 256, 256, 8
+    u, idx, counts = _random_routing(T, n, k, seed=5)
+    want = _with_workspace(u, idx, counts, T, d, n, k)
+    got = _no_alloc(u, idx, counts, T, d, n, k)
+    torch.cuda.synchronize()
+    _same(got, want)
+    T1 = T + 1
+    u1 = torch.zeros((T1, d), dtype=torch.bfloat16, device="cuda")
+    idx1 = torch.zeros((T1, k), dtype=torch.int32, device="cuda")
+    x, off, pos, src = _outputs(T1, d, n, k)
+    with pytest.raises(L.MoEError) as ei:
+        L.moe_permute_noalloc(u1, idx1, counts, T1, d, n, k, x, off, pos, src)
+    assert ei.value.status == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_get_device_status() == 0
