@@ -16,8 +16,14 @@ tokens / max-over-ranks device time) with inputs resident in HBM; `e2e` is the
 same metric through the public API with the batch copied from pinned host
 memory and the output copied back inside the timed region; `roofline` is the
 routed expert up-projection kernel (the dominant launch) against the measured
-bf16 tensor peak; `cpu_baseline` is the fp64 oracle on a bounded sample.
-`--impl reference` times that oracle alone as the reference arm.
+burst bf16 tensor peak (the sustained peak and the nominal rate at the run's
+median SM clock beside it); `routing` counts the batch's near-ties and checks
+the first timed step's expert indices against fp64 keys; `cpu_baseline` is the
+fp64 oracle on a bounded sample. The default V3-prefill run then times, in the
+same process, V3 decode (HBM roofline over the expert weights it touches), its
+softmax-gate form and FP8 prefill (`variants`). `--gpus N` started as one
+process re-launches itself as N ranks. `--impl reference` times the oracle
+alone as the reference arm.
 """
 from __future__ import annotations
 
@@ -290,8 +296,7 @@ def run_train(args, cfg, rank, world, local, dev):
     kname = max(kms, key=kms.get)
     flops = 2.0 * T * K * 2 * I * d
     pk = peaks()
-    peak = pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]
-    achieved = flops / (kms[kname] * 1e-3) / 1e12
+    clocks = clk.summary()
     fwd_flops = T * cfg.flops_per_token()
     # backward: dgrad and wgrad of every forward GEMM except the router's
     # (2x the expert FLOPs), plus O(T K d) elementwise work
@@ -334,23 +339,232 @@ def run_train(args, cfg, rank, world, local, dev):
                        "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2"},
             "step_tflops": step_flops / (ms_step * 1e-3) / 1e12,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+            "roofline": {**tensor_roofline(flops, kms[kname], pk, clocks), "traffic": None,
                          "kernel": {"dx": "grouped_dgrad_bf16_kernel<store> (moe_expert_up_backward)",
                                     "dw13": "grouped_wgrad_bf16_kernel (moe_expert_wgrad, dW13)"}[kname],
-                         "kernel_ms": kms[kname], "other_ms": kms,
-                         "peak_source": f"{pk['_source']} bf16_tflops_sustained"},
+                         "other_ms": kms},
             "e2e": {"value": T * world / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * T * d * 2, "d2h_bytes_per_step": T * d * 2,
                     "api": "MoELayer.forward(train=True) + MoELayer.backward"},
             "gpu_launches": args.steps * (lay.launches_per_step() + lay.launches_per_backward()),
-            "clocks": clk.summary(),
+            "clocks": clocks,
         }), flush=True)
 
 
 def L_status() -> int:
     from mixture_experts_layer_58_b200 import _lib as L
     return L.moe_get_device_status()
+
+
+# per-SM dense bf16 MMA rate of sm_100a: an M=128, N=256, K=16 tcgen05.mma
+# (1 M flop) issues every 128 clocks on one SM
+BF16_FLOP_PER_CLK_PER_SM = 8192
+NUM_SMS = 148
+
+
+def tensor_roofline(flops, kernel_ms, pk, clocks, fp8=False):
+    """Achieved TFLOP/s of a kernel against the measured peaks: `frac` is
+    against the burst bf16 peak (a kernel timed inside a step of tens of ms
+    runs at burst clocks), with the sustained peak and the nominal tensor
+    rate at the run's median SM clock beside it. FP8 takes 2x (the nominal
+    fp8/bf16 ratio of sm_100a's tensor cores)."""
+    ratio = 2.0 if fp8 else 1.0
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    burst = pk["bf16_tflops"] * ratio
+    sust = (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * ratio
+    out = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+           "frac": achieved / burst, "frac_of_sustained": achieved / sust,
+           "peak_sustained": sust, "kernel_ms": kernel_ms,
+           "peak_source": f"{pk['_source']} bf16_tflops (burst)"
+                          + (" x 2 (nominal fp8/bf16)" if fp8 else "")}
+    mhz = (clocks or {}).get("sm_mhz")
+    if mhz:
+        nominal = NUM_SMS * BF16_FLOP_PER_CLK_PER_SM * ratio * mhz * 1e6 / 1e12
+        out["nominal_at_median_clock"] = nominal
+        out["frac_of_nominal_at_median_clock"] = achieved / nominal
+    return out
+
+
+def routing_check(u, e, b, kind, K, idx_gpu):
+    """Statistic of one routed batch: near-ties (a token whose K+1 largest
+    selection keys, taken in fp64 from the same bf16 inputs and fp32 bias,
+    hold an adjacent pair closer than 1e-5) and, outside them, tokens whose
+    GPU selection differs from the fp64 top-K. Computed with torch fp64 on
+    the device; a report, not the product path."""
+    import torch
+    z = u.double() @ e.double().T
+    key = torch.sigmoid(z) + (b.double()[None, :] if b is not None else 0.0) \
+        if kind == "sigmoid" else z
+    top = torch.topk(key, K + 1, dim=1)
+    gaps = top.values[:, :-1] - top.values[:, 1:]
+    near = (gaps < 1e-5).any(dim=1)
+    want = top.indices[:, :K].to(torch.int32)
+    bad = (want != idx_gpu).any(dim=1) & ~near
+    return {"tokens": int(u.shape[0]), "near_ties": int(near.sum()),
+            "index_mismatch_outside_near_ties": int(bad.sum()),
+            "keys": "fp64 (torch on the device) from the bf16 u, e and the fp32 bias "
+                    "of the first timed step"}
+
+
+def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
+    """W warm-up steps, then K timed steps between barriers and device
+    syncs (CUDA events on the launching stream, clocks sampled throughout).
+    A step is the forward plus the bias update. Returns the timings and the
+    routing of the first and last timed steps."""
+    import torch
+    import torch.distributed as dist
+    from mixture_experts_layer_58_b200 import _lib as L
+    from mixture_experts_layer_58_b200 import dp
+    T = u.shape[0]
+    timers, recv_rows, snap = {}, [], {}
+
+    def step(i=None):
+        lay.forward(u, timers=timers if i is not None else None)
+        if i == 0:
+            snap["idx0"] = lay.topk_idx.clone()
+            snap["counts0"] = lay.counts.clone()
+        if i is not None and i == args.steps - 1:
+            snap["counts1"] = lay.counts.clone()
+        if ep_mode and i is not None:
+            recv_rows.append(lay.last_plan.n_recv)
+        if cfg.gate_kind == "sigmoid":
+            if world > 1 or ep_mode:
+                lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
+            else:
+                lay.update_bias()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if L.moe_get_device_status() != 0:
+        raise SystemExit("device timeout during warm-up")
+    bias0 = lay.bias.clone()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if world > 1 or ep_mode:
+        tt = torch.tensor([ms], device=u.device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    if L.moe_get_device_status() != 0:
+        raise SystemExit("device timeout during the timed region")
+    stage_ms = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in timers.items()}
+    return {"ms_step": ms / args.steps, "stage_ms": stage_ms, "clocks": clk.summary(),
+            "recv_rows": recv_rows, "bias0": bias0, **snap}
+
+
+def decode_hbm(cfg, counts, ms_step, pk):
+    """HBM roofline of a decode-sized step: the bytes it must move at least,
+    i.e. the W1/W3/W2 of every routed expert the batch touched and of the
+    shared expert(s), the centroids, and the activations (u in, x_perm and
+    y_perm written and read, h written and read, out written)."""
+    T, K, d, I = cfg.T, cfg.top_k, cfg.d, cfg.inter
+    wb = 1 if cfg.fp8 else 2
+    touched = int((counts > 0).sum())
+    weights = (touched * 3 * I * d + 3 * cfg.shared_inter * d) * wb
+    acts = (T * d * 2 + 2 * T * K * d * 2 + 2 * T * K * I * 2 + T * d * 2
+            + cfg.n_routed * d * 2)
+    byts = weights + acts
+    gbs = byts / (ms_step * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / pk["hbm_gbs"], "bytes_per_step": byts,
+            "expert_weight_bytes": weights, "experts_touched": touched,
+            "peak_source": f"{pk['_source']} hbm_gbs", "time": "whole layer step"}
+
+
+def up_kernel_roofline(cfg, lay, t, pk, up_rows, recorded):
+    """Roofline of the dominant launch, the routed up-projection + SwiGLU:
+    tensor-bound for prefill-sized groups, HBM-bound (its W13 slabs) for
+    decode-sized ones."""
+    T, K, d, I = cfg.T, cfg.top_k, cfg.d, cfg.inter
+    up_ms = t["stage_ms"]["up"]
+    kname = ("grouped_gemm_fp8_kernel<SwiGLU> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
+             "grouped_gemm_bf16_pair_kernel<SwiGLU, gather> (moe_expert_up_swiglu_gather)"
+             if lay.fused_gather else
+             "grouped_gemm bf16 <SwiGLU>, CTA-pair or 1-CTA tiles by group size "
+             "(moe_expert_up_swiglu)")
+    if T * K < 256 * cfg.n_routed:
+        touched = int((t["counts1"] > 0).sum())
+        wbytes = (1 if cfg.fp8 else 2) * 2 * I * d
+        up_bytes = touched * wbytes + T * K * d * (1 if cfg.fp8 else 2) + T * K * I * 2
+        gbs = up_bytes / (up_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"], "traffic": recorded, "kernel": kname,
+                "kernel_ms": up_ms, "bytes_per_launch": up_bytes, "experts_touched": touched,
+                "peak_source": f"{pk['_source']} hbm_gbs"}
+    r = tensor_roofline(2.0 * up_rows * d * 2 * I, up_ms, pk, t["clocks"], cfg.fp8)
+    r.update({"traffic": recorded, "kernel": kname})
+    return r
+
+
+def variant_line(name, args, dev, local, stream, pk):
+    """One more workload timed in the same process (decode, its softmax-gate
+    form, FP8 prefill): device time per step, stages, rooflines and the
+    routing statistic of its first timed step."""
+    import torch
+    from mixture_experts_layer_58_b200 import synth
+    from mixture_experts_layer_58_b200.layer import MoELayer
+    cfg = synth.CONFIGS[name]
+    W1, W3, W2 = synth.all_expert_weights(cfg, "cuda")
+    e_host, b_host = synth.centroids(cfg), synth.bias(cfg)
+    lay = MoELayer(e_host, b_host, W1, W3, W2, synth.shared_weights(cfg, "cuda"),
+                   top_k=cfg.top_k, routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
+                   gamma=cfg.gamma, fp8=cfg.fp8, device=dev)
+    del W1, W3, W2
+    torch.cuda.empty_cache()
+    u = synth.tokens(cfg).to(dev)
+    lay.allocate(cfg.T)
+    t = time_forward(lay, u, cfg, args, 1, False, local, stream)
+    T, K = cfg.T, cfg.top_k
+    line = {"workload": cfg.name, "T": T, "gate": cfg.gate_kind,
+            "dtype": "e4m3 (fp32 promotion)" if cfg.fp8 else "bf16",
+            "ms_per_step": t["ms_step"], "value": T / (t["ms_step"] * 1e-3),
+            "unit": "tokens/s", "steps": args.steps, "warmup": args.warmup,
+            "stage_ms": t["stage_ms"], "clocks": t["clocks"],
+            "gpu_launches": args.steps * lay.launches_per_step(),
+            "max_expert_load": {"first_timed_step": int(t["counts0"].max()),
+                                "last_timed_step": int(t["counts1"].max())}}
+    line["routing"] = routing_check(u, lay.centroids, t["bias0"] if cfg.gate_kind == "sigmoid"
+                                    else None, cfg.gate_kind, K, t["idx0"])
+    line["roofline"] = up_kernel_roofline(cfg, lay, t, pk, T * K, None)
+    if T * K < 256 * cfg.n_routed:
+        line["layer_hbm"] = decode_hbm(cfg, t["counts1"].cpu(), t["ms_step"], pk)
+    else:
+        lt = T * cfg.flops_per_token() / (t["ms_step"] * 1e-3) / 1e12
+        line["layer_tflops"] = lt
+        line["layer_frac_of_tensor_peak"] = lt / (pk["bf16_tflops"] * (2 if cfg.fp8 else 1))
+    if cfg.fp8:
+        try:
+            line["roofline"]["cublas_fp8_tflops_live"] = cublas_fp8_tflops(dev)
+        except (RuntimeError, AttributeError) as exc:   # context only
+            line["roofline"]["cublas_fp8_tflops_live"] = f"not measured: {exc}"[:120]
+    del lay, u
+    torch.cuda.empty_cache()
+    return line
+
+
+def relaunch_ranks(args, argv):
+    """`bench.py --gpus N` (N > 1) started as one plain process: start N ranks
+    on this node with torch.distributed.run (one per GPU, rendezvous on
+    127.0.0.1) and return their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1",
+           "--nproc-per-node", str(args.gpus), "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -372,13 +586,22 @@ def main():
                          "experts split over the ranks, token rows exchanged by NCCL "
                          "all-to-all (bf16 forward, five-call mode)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the decode and FP8 workloads timed after V3 prefill")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    args = ap.parse_args()
+    argv = sys.argv[1:]
+    args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch_ranks(args, argv))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one rank per GPU")
 
     from mixture_experts_layer_58_b200 import synth
     cfg = synth.CONFIGS[args.config]
@@ -441,51 +664,12 @@ def main():
     lay.allocate(T)
     stream = torch.cuda.current_stream()
 
-    up_timers = {}
-    recv_rows = []        # rows this rank's experts received, per timed step (ep)
-
-    def step(timed=False):
-        lay.forward(u, timers=up_timers if timed else None)
-        if ep_mode and timed:
-            recv_rows.append(lay.last_plan.n_recv)
-        if cfg.gate_kind == "sigmoid":
-            if world > 1 or ep_mode:
-                lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
-            else:
-                lay.update_bias()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if L.moe_get_device_status() != 0:
-        raise SystemExit("device timeout during warm-up")
-
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        t_start.record(stream)
-        for _ in range(args.steps):
-            step(timed=True)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-    ms = t_start.elapsed_time(t_end)
-    up_ms = sum(a.elapsed_time(b) for a, b in up_timers["up"]) / args.steps
-    stage_ms = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in up_timers.items()}
-    if world > 1 or ep_mode:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    if L.moe_get_device_status() != 0:
-        raise SystemExit("device timeout during the timed region")
-    ms_step = ms / args.steps
+    t = time_forward(lay, u, cfg, args, world, ep_mode, local, stream)
+    ms_step = t["ms_step"]
     value = T * world / (ms_step * 1e-3)
-    counts = lay.counts.cpu()
+    counts = t["counts1"].cpu()
+    routing = (routing_check(u, lay.centroids, t["bias0"] if cfg.gate_kind == "sigmoid" else None,
+                             cfg.gate_kind, K, t["idx0"]) if not ep_mode else None)
 
     # ---- e2e: host batch in pinned memory -> device, forward, output back.
     # Copies run on their own stream into double buffers, so step i+1's
@@ -499,6 +683,10 @@ def main():
     up_done = [torch.cuda.Event() for _ in range(2)]
     fwd_done = [torch.cuda.Event() for _ in range(2)]
     down_done = [torch.cuda.Event() for _ in range(2)]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
 
     def upload(i):
         b = i % 2
@@ -551,36 +739,10 @@ def main():
     pk = peaks()
     # the routed rows this rank's up-projection processes: its own T*K rows,
     # or under expert parallelism the rows its experts received
-    up_rows = sum(recv_rows) / len(recv_rows) if recv_rows else T * K
-    up_flops = 2.0 * up_rows * d * 2 * I
-    achieved = up_flops / (up_ms * 1e-3) / 1e12
-    # an FP8 contraction takes the measured bf16 peak x the nominal fp8/bf16 ratio (2)
-    ratio = 2.0 if cfg.fp8 else 1.0
-    peak = (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]) * ratio
-    kname = ("grouped_gemm_fp8_kernel<SwiGLU> (moe_expert_up_swiglu_fp8)" if cfg.fp8 else
-             "grouped_gemm_bf16_pair_kernel<SwiGLU, gather> (moe_expert_up_swiglu_gather)"
-             if lay.fused_gather else
-             "grouped_gemm bf16 <SwiGLU>, CTA-pair or 1-CTA tiles by group size "
-             "(moe_expert_up_swiglu)")
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak,
-                # the recorded counters are those of the single-GPU launch
-                "traffic": None if ep_mode else recorded_traffic(cfg.name),
-                "kernel": kname, "kernel_ms": up_ms,
-                "peak_source": f"{pk['_source']} bf16_tflops_sustained"
-                               + (" x 2 (nominal fp8/bf16)" if cfg.fp8 else "")}
-    if T * K < 256 * cfg.n_routed:
-        # decode-sized groups: the up-projection streams the W13 slabs of every
-        # expert the batch touches from HBM; its roofline is the copy bandwidth
-        touched = int((counts > 0).sum())
-        wbytes = (1 if cfg.fp8 else 2) * 2 * I * d
-        up_bytes = touched * wbytes + T * K * d * (1 if cfg.fp8 else 2) + T * K * I * 2
-        gbs = up_bytes / (up_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": gbs / pk["hbm_gbs"], "traffic": None, "kernel": kname,
-                    "kernel_ms": up_ms, "bytes_per_launch": up_bytes,
-                    "experts_touched": touched,
-                    "peak_source": f"{pk['_source']} hbm_gbs"}
+    up_rows = sum(t["recv_rows"]) / len(t["recv_rows"]) if t["recv_rows"] else T * K
+    # the recorded counters are those of the single-GPU launch
+    roofline = up_kernel_roofline(cfg, lay, t, pk, up_rows,
+                                  None if ep_mode else recorded_traffic(cfg.name))
     if cfg.fp8:
         try:
             roofline["cublas_fp8_tflops_live"] = cublas_fp8_tflops(dev)
@@ -592,7 +754,8 @@ def main():
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (fp32 promotion)" if cfg.fp8 else "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 (fp32 promotion)" if cfg.fp8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the V3 layer shape)",
         "config": {"workload": cfg.name, "T": T, "d": d, "n_routed": cfg.n_routed, "top_k": K,
                    "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
@@ -606,18 +769,26 @@ def main():
                                    f"dp{world}" if world > 1 else "single"),
                    "l2": "inputs larger than L2 (22.6 GB of expert weights streamed per step)"
                    if cfg.weights_on_gpu else "L2 not flushed: small workload",
-                   "max_expert_load": int(counts.max()), "mean_expert_load": T * K / cfg.n_routed},
+                   "bias": "updated at the end of every step (the timed work), so the load "
+                           "drifts toward balance over the steps",
+                   "max_expert_load": {"first_timed_step": int(t["counts0"].max()),
+                                       "last_timed_step": int(counts.max())},
+                   "mean_expert_load": T * K / cfg.n_routed},
         "layer_tflops": layer_tflops,
         "layer_frac_of_bf16_peak": layer_tflops / pk["bf16_tflops"],
-        "layer_frac_of_tensor_peak": layer_tflops / (pk["bf16_tflops"] * ratio),
+        "layer_frac_of_tensor_peak": layer_tflops / (pk["bf16_tflops"] * (2 if cfg.fp8 else 1)),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2, "api": type(lay).__name__ + ".forward",
                 "copies": "pinned host, own stream, overlapped with neighbouring steps"},
-        "stage_ms": stage_ms,
+        "stage_ms": t["stage_ms"],
         "gpu_launches": args.steps * lay.launches_per_step(),
-        "clocks": clk.summary(),
+        "clocks": t["clocks"],
     }
+    if routing is not None:
+        result["routing"] = routing
+    if T * K < 256 * cfg.n_routed:
+        result["layer_hbm"] = decode_hbm(cfg, counts, ms_step, pk)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -631,6 +802,15 @@ def main():
             "value": n / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"oracle full layer (fp64) on the first {n} of {T} tokens, {sec:.1f} s; "
                       f"host has {os.cpu_count()} cores"}
+
+    # ---- the other V3-shape workloads, same process, after the headline line's
+    # measurements: decode (HBM-bound), its softmax-gate form, FP8 prefill
+    if (cfg.name == "v3p" and world == 1 and not ep_mode and args.mode == "five-call"
+            and not args.no_variants):
+        del lay, u, u_buf, o_buf
+        torch.cuda.empty_cache()
+        result["variants"] = {n: variant_line(n, args, dev, local, stream, pk)
+                              for n in ("v3d", "v3d_softmax", "v3p_fp8")}
 
     if rank == 0:
         print(json.dumps(result), flush=True)

@@ -9,12 +9,13 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(extra_env=None):
-    env = dict(os.environ)
+def _run(extra_env=None, gpus=1):
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
     env.update(extra_env or {})
     return subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny",
-                           "--steps", "2", "--warmup", "3"], cwd=ROOT, env=env,
-                          capture_output=True, text=True, timeout=300)
+                           "--steps", "2", "--warmup", "3", "--gpus", str(gpus)], cwd=ROOT,
+                          env=env, capture_output=True, text=True, timeout=300)
 
 
 def test_reference_arm_prints_one_contract_line():
@@ -38,6 +39,23 @@ def test_reference_arm_prints_one_contract_line():
 
 
 def test_reference_arm_other_ranks_exit_quietly():
-    p = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    p = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, gpus=2)
     assert p.returncode == 0, p.stderr[-2000:]
     assert not [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_gpus_n_starts_n_ranks():
+    """`bench.py --gpus 2` run as one plain process starts two ranks itself
+    (torch.distributed.run on 127.0.0.1); each sees WORLD_SIZE 2, rank 0
+    prints the one line with n_gpus 2 and the other rank exits quietly."""
+    p = _run(gpus=2)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_world_size_must_match_gpus():
+    p = _run({"RANK": "0", "WORLD_SIZE": "3", "LOCAL_RANK": "0"}, gpus=2)
+    assert p.returncode != 0
+    assert "WORLD_SIZE=3" in p.stderr
