@@ -295,6 +295,37 @@ MOE_API int moe_combine(const void* y_perm, const int32_t* pos, const float* top
                         const void* shared_out, const void* residual, int T, int d, int top_k,
                         void* out, moe_stream_t stream);
 
+/* ------------------------------------------------------------------ fused scatter
+ * The gate-weighted combine of the output equation h'_t (technical report
+ * summary, Method §2) moved into the down-projection's epilogue: each routed
+ * row leaves the GEMM already multiplied by its gate g_{i,t} and lands in the
+ * row of its (token, slot) pair, so the combine only adds K rows that sit next
+ * to each other. Deterministic: no atomics, the same fixed summation order.
+ * One forward in this mode: moe_route, moe_permute, moe_slot_index,
+ * moe_expert_up_swiglu, moe_expert_down_scatter, moe_combine_slots.
+ *
+ * moe_slot_index: dst_slot [rows] int32 out: dst_slot[pos[s]] = s for every
+ *   pair s = t*top_k + k whose pos[s] (moe_permute's) lies in [0, rows); the
+ *   other entries are set to -1. The inverse of pos.
+ * moe_expert_down_scatter: moe_expert_down whose output row r goes to row
+ *   dst_slot[r] of y_slots [T*top_k, d] bf16 (16-B aligned), multiplied in
+ *   fp32 by topk_gate[dst_slot[r]] before the one bf16 rounding. Rows whose
+ *   dst_slot lies outside [0, T*top_k) are not stored. Other arguments as
+ *   moe_expert_down.
+ * moe_combine_slots: out_t = residual_t + shared_t + sum over the slots k
+ *   with pos[t,k] >= 0 of y_slots[t*top_k + k] (fp32 sums in slot order, one
+ *   bf16 rounding). Arguments as moe_combine without topk_gate.
+ */
+MOE_API int moe_slot_index(const int32_t* pos, int T, int top_k, int rows, int32_t* dst_slot,
+                           moe_stream_t stream);
+MOE_API int moe_expert_down_scatter(const void* h, const int32_t* group_offsets, int G, int rows,
+                                    int inter, int d, const void* w2, const int32_t* dst_slot,
+                                    const float* topk_gate, int T, int top_k, void* y_slots,
+                                    moe_stream_t stream);
+MOE_API int moe_combine_slots(const void* y_slots, const int32_t* pos, const void* shared_out,
+                              const void* residual, int T, int d, int top_k, void* out,
+                              moe_stream_t stream);
+
 /* ------------------------------------------------------------------ bias update
  * Auxiliary-loss-free balancing (technical report summary, Method §2): at the
  * end of a step, b_i <- b_i - gamma if expert i is overloaded and

@@ -64,6 +64,10 @@ _SIGS = {
     "moe_expert_down_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_bias_update": (_i, [_vp, _vp, _i, _ll, _i, _f, _vp]),
+    "moe_slot_index": (_i, [_vp, _i, _i, _i, _vp, _vp]),
+    "moe_expert_down_scatter": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _i, _vp,
+                                     _vp]),
+    "moe_combine_slots": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_pack_w13": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_strerror": (ctypes.c_char_p, [_i]),
     "moe_last_cuda_error": (_i, []),
@@ -233,6 +237,23 @@ def moe_expert_down_fp8(h8, h_scales, group_offsets, G, rows, inter, d, w2, w2_s
 def moe_combine(y_perm, pos, topk_gate, shared_out, residual, T, d, top_k, out, stream=None):
     _check(_L().moe_combine(_p(y_perm), _p(pos), _p(topk_gate), _p(shared_out), _p(residual), T,
                             d, top_k, _p(out), _stream(stream)), "moe_combine")
+
+
+def moe_slot_index(pos, T, top_k, rows, dst_slot, stream=None):
+    _check(_L().moe_slot_index(_p(pos), T, top_k, rows, _p(dst_slot), _stream(stream)),
+           "moe_slot_index")
+
+
+def moe_expert_down_scatter(h, group_offsets, G, rows, inter, d, w2, dst_slot, topk_gate, T,
+                            top_k, y_slots, stream=None):
+    _check(_L().moe_expert_down_scatter(_p(h), _p(group_offsets), G, rows, inter, d, _p(w2),
+                                        _p(dst_slot), _p(topk_gate), T, top_k, _p(y_slots),
+                                        _stream(stream)), "moe_expert_down_scatter")
+
+
+def moe_combine_slots(y_slots, pos, shared_out, residual, T, d, top_k, out, stream=None):
+    _check(_L().moe_combine_slots(_p(y_slots), _p(pos), _p(shared_out), _p(residual), T, d,
+                                  top_k, _p(out), _stream(stream)), "moe_combine_slots")
 
 
 def moe_bias_update(expert_counts, bias, n_routed, T, top_k, gamma, stream=None):

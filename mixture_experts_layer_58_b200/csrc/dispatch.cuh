@@ -186,6 +186,9 @@ __device__ __forceinline__ void add_bf16x8(float (&a)[8], const uint4& v) {
 
 // out_t = residual_t + shared_t + sum_k g[t,k] * y_perm[pos[t,k]]; one warp
 // per token, fp32 sums in a fixed order, one bf16 rounding.
+// SLOTS (the fused-scatter mode): the routed rows already carry their gate
+// and sit in slot order, y[t*K + k]; slot k counts when pos[t,k] >= 0.
+template <bool SLOTS>
 __global__ void __launch_bounds__(256)
 combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ pos,
                const float* __restrict__ gate, const __nv_bfloat16* __restrict__ shared_out,
@@ -197,7 +200,7 @@ combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restri
   const int nvec = d >> 3;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     const int myp = lane < K ? pos[static_cast<size_t>(t) * K + lane] : -1;
-    const float myg = lane < K ? gate[static_cast<size_t>(t) * K + lane] : 0.0f;
+    const float myg = (!SLOTS && lane < K) ? gate[static_cast<size_t>(t) * K + lane] : 1.0f;
     int p[kMaxTopK];
     float g[kMaxTopK];
 #pragma unroll
@@ -205,6 +208,7 @@ combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restri
       p[k] = __shfl_sync(0xffffffffu, myp, k);
       g[k] = __shfl_sync(0xffffffffu, myg, k);
       if (k >= K || p[k] < 0 || p[k] >= total) p[k] = -1;
+      else if (SLOTS) p[k] = t * K + k;
     }
     const size_t row = static_cast<size_t>(t) * d;
     for (int v0 = lane; v0 < nvec; v0 += 64) {
@@ -233,8 +237,11 @@ combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restri
         if (residual) add_bf16x8(a[j], rv[j]);
         if (shared_out) add_bf16x8(a[j], sv[j]);
 #pragma unroll
-        for (int k = 0; k < kMaxTopK; ++k)
-          if (p[k] >= 0) acc_bf16x8(a[j], yv[j][k], g[k]);
+        for (int k = 0; k < kMaxTopK; ++k) {
+          if (p[k] < 0) continue;
+          if (SLOTS) add_bf16x8(a[j], yv[j][k]);
+          else acc_bf16x8(a[j], yv[j][k], g[k]);
+        }
         uint4 o;
         o.x = pack_bf16x2(a[j][0], a[j][1]);
         o.y = pack_bf16x2(a[j][2], a[j][3]);
@@ -243,6 +250,19 @@ combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restri
         *(reinterpret_cast<uint4*>(out + row) + v) = o;
       }
     }
+  }
+}
+
+// dst_slot[pos[s]] = s for every (token, slot) pair s = t*K + k that has a
+// row in [0, rows); the caller sets dst_slot to -1 first, so rows no pair
+// maps to stay -1. The inverse of the dispatch's pos.
+__global__ void __launch_bounds__(256)
+slot_index_kernel(const int32_t* __restrict__ pos, long long n_pairs, int rows,
+                  int32_t* __restrict__ dst_slot) {
+  for (long long s = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; s < n_pairs;
+       s += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int p = pos[s];
+    if (p >= 0 && p < rows) dst_slot[p] = static_cast<int32_t>(s);
   }
 }
 

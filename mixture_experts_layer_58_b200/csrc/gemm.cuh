@@ -27,7 +27,18 @@ constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
 constexpr int kGemmThreads = 192;
 constexpr int kMaxGroups = 1024;
 
-enum { EPI_STORE = 0, EPI_SWIGLU = 1 };
+enum { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SCATTER = 2 };
+
+// EPI_SCATTER (the down-projection of the fused-scatter mode): output row r
+// of a group goes to row slot[r] of the output, a (token, slot) row of a
+// [T*K, d] buffer, multiplied by scale[slot[r]] (the token's gate for that
+// expert) in fp32 before its bf16 rounding. Rows whose slot lies outside
+// [0, n_slots) are not stored.
+struct ScatterOut {
+  const int32_t* slot;
+  const float* scale;
+  int n_slots;
+};
 
 template <int BN>
 struct GemmCfg {
@@ -124,7 +135,8 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB,
                          const int32_t* __restrict__ offsets, int G, int K, int n_per_group,
                          int rows, __nv_bfloat16* __restrict__ out, int ldo,
-                         __nv_bfloat16* __restrict__ ac, unsigned int* status) {
+                         __nv_bfloat16* __restrict__ ac, unsigned int* status,
+                         ScatterOut sc) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -303,17 +315,32 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       } else {
-        __nv_bfloat16* dst_row = out + static_cast<size_t>(grow) * ldo + n_blk * BN;
+        int drow = grow;
+        bool store = valid;
+        float scale = 1.0f;
+        if constexpr (EPI == EPI_SCATTER) {
+          drow = valid ? __ldg(sc.slot + grow) : -1;
+          store = valid && drow >= 0 && drow < sc.n_slots;
+          scale = store ? __ldg(sc.scale + drow) : 0.0f;
+        }
+        __nv_bfloat16* dst_row = out + static_cast<size_t>(store ? drow : 0) * ldo + n_blk * BN;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32cols(taddr + c, r);
           tmem_ld_wait();
-          if (valid) {
+          if (store) {
             uint32_t pk[16];
+            if constexpr (EPI == EPI_SCATTER) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(scale * __uint_as_float(r[2 * i]),
+                                    scale * __uint_as_float(r[2 * i + 1]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            }
             uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
 #pragma unroll
             for (int v = 0; v < 4; ++v)

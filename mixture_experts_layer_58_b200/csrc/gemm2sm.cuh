@@ -248,7 +248,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                               int rows, __nv_bfloat16* __restrict__ out, int ldo,
                               __nv_bfloat16* __restrict__ ac,
                               const int32_t* __restrict__ src_rows, int* tile_counter,
-                              unsigned int* status) {
+                              unsigned int* status, ScatterOut sc) {
   constexpr int BN = 256;
   using C = Gemm2smCfg;
   extern __shared__ uint8_t smem_raw[];
@@ -519,9 +519,20 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         } else {
           // X = [32 tokens][128 output features of this CTA]
+          if constexpr (EPI == EPI_SCATTER) {
+            // lane i holds the gate of the chunk's token i (0 past the group)
+            const int gr = row0 + j0 + lane;
+            const int sl = gr < row_end ? __ldg(sc.slot + gr) : -1;
+            const float gl = (sl >= 0 && sl < sc.n_slots) ? __ldg(sc.scale + sl) : 0.0f;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            X[i * 128 + quarter * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+            for (int i = 0; i < 32; ++i)
+              X[i * 128 + quarter * 32 + lane] =
+                  __float2bfloat16_rn(__shfl_sync(0xffffffffu, gl, i) * __uint_as_float(v[i]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              X[i * 128 + quarter * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+          }
           if (!xfer_sync(&xready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
           __nv_bfloat16* dst0 = out + n_blk * BN + static_cast<int>(rank) * 128;
 #pragma unroll
@@ -529,9 +540,15 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const int idx = et + 128 * k;
             const int r = idx >> 4, seg = idx & 15;
             const int grow = row0 + j0 + r;
-            if (grow < row_end)
-              *reinterpret_cast<uint4*>(dst0 + static_cast<size_t>(grow) * ldo + seg * 8) =
+            if (grow < row_end) {
+              int drow = grow;
+              if constexpr (EPI == EPI_SCATTER) {
+                drow = __ldg(sc.slot + grow);
+                if (drow < 0 || drow >= sc.n_slots) continue;
+              }
+              *reinterpret_cast<uint4*>(dst0 + static_cast<size_t>(drow) * ldo + seg * 8) =
                   *reinterpret_cast<const uint4*>(X + r * 128 + seg * 8);
+            }
           }
         }
         ok = true;

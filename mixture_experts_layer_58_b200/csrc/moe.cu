@@ -156,7 +156,7 @@ inline cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStre
 template <int BN, int EPI>
 int launch_grouped_gemm(const void* A, int rows, int K, const void* B, int G, int n_per_group,
                         const int32_t* offsets, void* out, int ldo, cudaStream_t st,
-                        void* ac = nullptr) {
+                        void* ac = nullptr, ScatterOut sc = ScatterOut{nullptr, nullptr, 0}) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
@@ -172,7 +172,7 @@ int launch_grouped_gemm(const void* A, int rows, int K, const void* B, int G, in
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
   kern<<<grid, kGemmThreads, smem, st>>>(tmA, tmB, offsets, G, K, n_per_group, rows,
                                          static_cast<__nv_bfloat16*>(out), ldo,
-                                         static_cast<__nv_bfloat16*>(ac), di->status);
+                                         static_cast<__nv_bfloat16*>(ac), di->status, sc);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -233,7 +233,8 @@ template <int EPI>
 int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int G,
                              int n_per_group, const int32_t* offsets, void* out, int ldo,
                              cudaStream_t st, const int32_t* src_rows = nullptr,
-                             int a_rows = 0, void* ac = nullptr) {
+                             int a_rows = 0, void* ac = nullptr,
+                             ScatterOut sc = ScatterOut{nullptr, nullptr, 0}) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
@@ -260,14 +261,14 @@ int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int 
     kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
                                                  static_cast<__nv_bfloat16*>(out), ldo,
                                                  static_cast<__nv_bfloat16*>(ac), src_rows,
-                                                 counter, di->status);
+                                                 counter, di->status, sc);
   } else {
     auto kern = grouped_gemm_bf16_pair_kernel<EPI, false>;
     if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
     kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
                                                  static_cast<__nv_bfloat16*>(out), ldo,
                                                  static_cast<__nv_bfloat16*>(ac), nullptr,
-                                                 counter, di->status);
+                                                 counter, di->status, sc);
   }
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
@@ -740,8 +741,72 @@ int moe_combine(const void* y_perm, const int32_t* pos, const float* topk_gate,
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
   const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
-  combine_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
+  combine_kernel<false><<<blocks, 256, 0, as_stream(stream)>>>(
       static_cast<const __nv_bfloat16*>(y_perm), pos, topk_gate,
+      static_cast<const __nv_bfloat16*>(shared_out), static_cast<const __nv_bfloat16*>(residual),
+      T, d, top_k, static_cast<__nv_bfloat16*>(out));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ fused scatter
+int moe_slot_index(const int32_t* pos, int T, int top_k, int rows, int32_t* dst_slot,
+                   moe_stream_t stream) {
+  if (T < 0 || top_k <= 0 || rows < 0) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!dst_slot || (T > 0 && !pos)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  MOE_CUDA(cudaMemsetAsync(dst_slot, 0xFF, sizeof(int32_t) * rows, st));
+  if (T == 0) return MOE_OK;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const long long pairs = static_cast<long long>(T) * top_k;
+  const int blocks =
+      static_cast<int>(std::max(1LL, std::min<long long>((pairs + 255) / 256, di->num_sms * 8)));
+  slot_index_kernel<<<blocks, 256, 0, st>>>(pos, pairs, rows, dst_slot);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_expert_down_scatter(const void* h, const int32_t* group_offsets, int G, int rows,
+                            int inter, int d, const void* w2, const int32_t* dst_slot,
+                            const float* topk_gate, int T, int top_k, void* y_slots,
+                            moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!h || !group_offsets || !w2 || !dst_slot || !topk_gate || !y_slots || !aligned16(h) ||
+      !aligned16(w2) || !aligned16(y_slots))
+    return MOE_ERR_INVALID_ARG;
+  const ScatterOut sc{dst_slot, topk_gate, T * top_k};
+  if (use_pair_tiles(rows, G))
+    return launch_grouped_gemm_pair<EPI_SCATTER>(h, rows, inter, w2, G, d, group_offsets,
+                                                 y_slots, d, as_stream(stream), nullptr, 0,
+                                                 nullptr, sc);
+  return launch_grouped_gemm<256, EPI_SCATTER>(h, rows, inter, w2, G, d, group_offsets, y_slots,
+                                               d, as_stream(stream), nullptr, sc);
+}
+
+int moe_combine_slots(const void* y_slots, const int32_t* pos, const void* shared_out,
+                      const void* residual, int T, int d, int top_k, void* out,
+                      moe_stream_t stream) {
+  if (T < 0 || d <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!y_slots || !pos || !out || !aligned16(y_slots) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if ((shared_out && !aligned16(shared_out)) || (residual && !aligned16(residual)))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
+  combine_kernel<true><<<blocks, 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(y_slots), pos, nullptr,
       static_cast<const __nv_bfloat16*>(shared_out), static_cast<const __nv_bfloat16*>(residual),
       T, d, top_k, static_cast<__nv_bfloat16*>(out));
   MOE_CUDA(cudaGetLastError());

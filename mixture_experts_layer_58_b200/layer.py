@@ -62,8 +62,8 @@ class MoELayer:
 
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
-                 fp8: bool = False, fused_gather: bool = False, overlap_shared: bool = True,
-                 device="cuda"):
+                 fp8: bool = False, fused_gather: bool = False, fused_scatter: bool = False,
+                 overlap_shared: bool = True, device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -78,6 +78,10 @@ class MoELayer:
         # fused gather (bf16): the up-projection reads the token rows of u
         # itself, so the dispatch only computes row indices (no x_perm copy)
         self.fused_gather = bool(fused_gather) and not self.fp8
+        # fused scatter (bf16): the down-projection multiplies each routed row
+        # by its gate and writes it to its (token, slot) row; the combine then
+        # adds K adjacent rows per token
+        self.fused_scatter = bool(fused_scatter) and not self.fp8
         # bf16: run the shared expert on a side stream next to the routed path
         self.overlap_shared = bool(overlap_shared) and not self.fp8
         self.centroids = centroids.to(dev, bf).contiguous()
@@ -145,6 +149,8 @@ class MoELayer:
         self.offsets = torch.empty(self.n_routed + 1, dtype=i32, device=dev)
         self.pos = torch.empty((T, K), dtype=i32, device=dev)
         self.src = torch.empty(rows, dtype=i32, device=dev)
+        self.dst_slot = (torch.empty(rows, dtype=i32, device=dev) if self.fused_scatter
+                         else None)
         self.x_perm = (None if (self.fp8 or self.fused_gather) else
                        torch.empty((rows, d), dtype=torch.bfloat16, device=dev))
         self.y_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
@@ -184,6 +190,8 @@ class MoELayer:
         if self.fused_gather:
             L.moe_permute_index(self.topk_idx, self.counts, T, self.n_routed, self.top_k,
                                 self.offsets, self.pos, self.src, self.perm_ws, self.perm_ws_bytes)
+            if self.fused_scatter:
+                L.moe_slot_index(self.pos, T, self.top_k, T * self.top_k, self.dst_slot)
             return
         if self.fp8:
             # quantise each token once (1x128 tiles), then copy its codes K times
@@ -195,6 +203,8 @@ class MoELayer:
         L.moe_permute(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
                       self.x_perm, self.offsets, self.pos, self.src, self.perm_ws,
                       self.perm_ws_bytes)
+        if self.fused_scatter:
+            L.moe_slot_index(self.pos, T, self.top_k, T * self.top_k, self.dst_slot)
 
     def _routed_up(self, T, u):
         rows = T * self.top_k
@@ -216,6 +226,11 @@ class MoELayer:
             L.moe_quant_act_fp8(hb, rows, self.inter, h8, hs)
             L.moe_expert_down_fp8(h8, hs, self.offsets, self.n_routed, rows, self.inter, self.d,
                                   self.w2, self.w2_s, self.y_perm)
+        elif self.fused_scatter:
+            # y_perm holds the gate-weighted rows in (token, slot) order
+            L.moe_expert_down_scatter(self.ffn_ws, self.offsets, self.n_routed, rows, self.inter,
+                                      self.d, self.w2, self.dst_slot, self.topk_gate, T,
+                                      self.top_k, self.y_perm)
         else:
             L.moe_expert_down(self.ffn_ws, self.offsets, self.n_routed, rows, self.inter, self.d,
                               self.w2, self.y_perm)
@@ -244,6 +259,10 @@ class MoELayer:
 
     def combine(self, u, residual: bool = True, out=None):
         T = u.shape[0]
+        if self.fused_scatter:
+            L.moe_combine_slots(self.y_perm, self.pos, self.shared_out, u if residual else None,
+                                T, self.d, self.top_k, self.out if out is None else out)
+            return
         L.moe_combine(self.y_perm, self.pos, self.topk_gate, self.shared_out,
                       u if residual else None, T, self.d, self.top_k,
                       self.out if out is None else out)
@@ -265,8 +284,9 @@ class MoELayer:
         dst = self.out if out is None else out
         assert dst.shape == (T, self.d) and dst.dtype == torch.bfloat16 and dst.is_contiguous()
         if train:
-            if self.fp8 or self.fused_gather:
-                raise ValueError("training runs on the bf16 layer with the copy-based dispatch")
+            if self.fp8 or self.fused_gather or self.fused_scatter:
+                raise ValueError("training runs on the bf16 layer with the copy-based dispatch "
+                                 "and the plain combine")
             self._allocate_train(T)
         self._train_state = (u, residual) if train else None
         ev = _Timed(timers)
@@ -446,6 +466,8 @@ class MoELayer:
         # quantisation, down-projection
         ffn = 3 if self.fp8 else 2
         perm = 2 if self.fused_gather else 3
+        if self.fused_scatter:
+            perm += 1                       # the slot index
         n = 1 + perm + ffn + 1 + (1 if self.fp8 else 0)
         if self.ws13 is not None:
             n += ffn

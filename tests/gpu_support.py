@@ -22,7 +22,8 @@ class Inputs:
     """Seeded inputs of a workload, the device layer built from them, and an
     accessor for the oracle's copy of any expert's weights."""
 
-    def __init__(self, cfg: synth.MoEConfig, T: int | None = None, fused_gather: bool = False):
+    def __init__(self, cfg: synth.MoEConfig, T: int | None = None, fused_gather: bool = False,
+                 fused_scatter: bool = False):
         from mixture_experts_layer_58_b200.layer import MoELayer
         self.cfg = cfg
         self.u = synth.tokens(cfg, T)
@@ -37,7 +38,8 @@ class Inputs:
             self.W = (W1, W3, W2)
         self.layer = MoELayer(self.e, self.b, W1, W3, W2, self.shared, top_k=cfg.top_k,
                               routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
-                              gamma=cfg.gamma, fused_gather=fused_gather)
+                              gamma=cfg.gamma, fused_gather=fused_gather,
+                              fused_scatter=fused_scatter)
         del W1, W3, W2
         self.u_dev = self.u.cuda()
         self._cache = {}

@@ -256,3 +256,31 @@ def test_header_is_c99_and_the_library_links_from_c(lib, tmp_path):
     assert out.returncode == 0, out.stderr
     assert out.stdout.strip() == "ok"
 
+
+
+def test_fused_scatter_entry_points_reject_bad_arguments(lib):
+    # moe_slot_index(pos, T, top_k, rows, dst_slot)
+    assert lib.moe_slot_index(A, -1, 4, 8, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_slot_index(A, 2, 9, 8, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_slot_index(A, 2, 4, 8, None, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_slot_index(None, 2, 4, 8, A, None) == L.MOE_ERR_INVALID_ARG
+    # moe_expert_down_scatter(h, off, G, rows, inter, d, w2, slot, gate, T, K, y)
+    ok = dict(h=A, off=A, G=4, rows=64, inter=128, d=256, w2=A, slot=A, gate=A, T=16, K=4, y=A)
+
+    def ds(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.moe_expert_down_scatter(a["h"], a["off"], a["G"], a["rows"], a["inter"],
+                                           a["d"], a["w2"], a["slot"], a["gate"], a["T"],
+                                           a["K"], a["y"], None)
+    assert ds(d=100) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert ds(T=-1) == L.MOE_ERR_INVALID_ARG
+    assert ds(slot=None) == L.MOE_ERR_INVALID_ARG
+    assert ds(gate=None) == L.MOE_ERR_INVALID_ARG
+    assert ds(y=MIS) == L.MOE_ERR_INVALID_ARG
+    # moe_combine_slots(y, pos, shared, residual, T, d, K, out)
+    assert lib.moe_combine_slots(A, A, None, None, 4, 256, 9, A, None) == \
+        L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_combine_slots(MIS, A, None, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_slots(A, None, None, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_slots(A, A, MIS, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
