@@ -406,6 +406,21 @@ def routing_check(u, e, b, kind, K, idx_gpu):
                     "of the first timed step"}
 
 
+def bias_step(lay, cfg, T, world, ep_mode):
+    """The end-of-step bias update: this batch's loads on one GPU; the loads
+    summed over the ranks otherwise (the peer-memory expert-parallel layer
+    has them from its device plan already)."""
+    from mixture_experts_layer_58_b200 import dp
+    if cfg.gate_kind != "sigmoid":
+        return
+    if hasattr(lay, "global_counts"):
+        lay.update_bias()
+    elif world > 1 or ep_mode:
+        lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
+    else:
+        lay.update_bias()
+
+
 def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
     """W warm-up steps, then K timed steps between barriers and device
     syncs (CUDA events on the launching stream, clocks sampled throughout).
@@ -425,13 +440,9 @@ def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
             snap["counts0"] = lay.counts.clone()
         if i is not None and i == args.steps - 1:
             snap["counts1"] = lay.counts.clone()
-        if ep_mode and i is not None:
+        if ep_mode and i is not None and hasattr(lay, "last_plan"):
             recv_rows.append(lay.last_plan.n_recv)
-        if cfg.gate_kind == "sigmoid":
-            if world > 1 or ep_mode:
-                lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
-            else:
-                lay.update_bias()
+        bias_step(lay, cfg, T, world, ep_mode)
 
     for _ in range(args.warmup):
         step()
@@ -574,17 +585,22 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="v3p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--mode", default="five-call", choices=["five-call", "fused", "train"],
+    ap.add_argument("--mode", default="five-call",
+                    choices=["five-call", "fused", "scatter", "train"],
                     help="five-call: route, permute (copy), grouped FFN, combine, bias update; "
                          "fused: the up-projection gathers the token rows itself (bf16; measured "
-                         "slower: the TMA gathers are request-rate bound); train: forward with "
-                         "saved pre-activations + backward + bias update (bf16)")
+                         "slower: the TMA gathers are request-rate bound); scatter: the "
+                         "down-projection applies the gates and writes slot-ordered rows, the "
+                         "combine adds adjacent rows (bf16); train: forward with saved "
+                         "pre-activations + backward + bias update (bf16)")
     ap.add_argument("--no-overlap", action="store_true",
                     help="run the shared expert after the routed experts on one stream")
-    ap.add_argument("--parallel", default="dp", choices=["dp", "ep"],
+    ap.add_argument("--parallel", default="dp", choices=["dp", "ep", "ep-p2p"],
                     help="dp: every rank holds all experts, its own batch; ep: the routed "
                          "experts split over the ranks, token rows exchanged by NCCL "
-                         "all-to-all (bf16 forward, five-call mode)")
+                         "all-to-all; ep-p2p: the same split, rows stored into and read back "
+                         "from the owners' buffers by the library's kernels over peer memory, "
+                         "planned on the device (bf16 forward, five-call mode)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the decode and FP8 workloads timed after V3 prefill")
@@ -614,7 +630,7 @@ def main():
     import torch.distributed as dist
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    ep_mode = args.parallel == "ep"
+    ep_mode = args.parallel in ("ep", "ep-p2p")
     if ep_mode and (cfg.fp8 or args.mode != "five-call"):
         raise SystemExit("--parallel ep runs the bf16 five-call forward")
     if world > 1 or ep_mode:
@@ -646,15 +662,17 @@ def main():
     W1, W3, W2 = synth.all_expert_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
     shared = synth.shared_weights(cfg, "cuda" if cfg.weights_on_gpu else "cpu")
     if ep_mode:
-        from mixture_experts_layer_58_b200.ep import ExpertParallelMoELayer
-        lay = ExpertParallelMoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
-                                     routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
-                                     gamma=cfg.gamma, overlap_shared=not args.no_overlap,
-                                     device=dev)
+        from mixture_experts_layer_58_b200.ep import (ExpertParallelMoELayer,
+                                                      PeerExpertParallelMoELayer)
+        cls = PeerExpertParallelMoELayer if args.parallel == "ep-p2p" else ExpertParallelMoELayer
+        lay = cls(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
+                  routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
+                  overlap_shared=not args.no_overlap, device=dev)
     else:
         lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
                        routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
                        fp8=cfg.fp8, fused_gather=(args.mode == "fused"),
+                       fused_scatter=(args.mode == "scatter"),
                        overlap_shared=not args.no_overlap, device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
@@ -707,11 +725,7 @@ def main():
             stream.wait_event(up_done[b])
             stream.wait_event(down_done[b])       # o_buf[b] downloaded
             lay.forward(u_buf[b], out=o_buf[b])
-            if cfg.gate_kind == "sigmoid":
-                if world > 1 or ep_mode:
-                    lay.update_bias(lay.counts, dp.sync_load(lay.counts, T))
-                else:
-                    lay.update_bias()
+            bias_step(lay, cfg, T, world, ep_mode)
             fwd_done[b].record(stream)
             with torch.cuda.stream(copy):
                 copy.wait_event(fwd_done[b])
@@ -739,7 +753,12 @@ def main():
     pk = peaks()
     # the routed rows this rank's up-projection processes: its own T*K rows,
     # or under expert parallelism the rows its experts received
-    up_rows = sum(t["recv_rows"]) / len(t["recv_rows"]) if t["recv_rows"] else T * K
+    if t["recv_rows"]:
+        up_rows = sum(t["recv_rows"]) / len(t["recv_rows"])
+    elif hasattr(lay, "goff"):
+        up_rows = int(lay.goff[-1])          # the last step's received rows (read after timing)
+    else:
+        up_rows = T * K
     # the recorded counters are those of the single-GPU launch
     roofline = up_kernel_roofline(cfg, lay, t, pk, up_rows,
                                   None if ep_mode else recorded_traffic(cfg.name))
@@ -760,9 +779,13 @@ def main():
         "config": {"workload": cfg.name, "T": T, "d": d, "n_routed": cfg.n_routed, "top_k": K,
                    "n_shared": cfg.n_shared, "inter": I, "routed_scale": cfg.routed_scale,
                    "gate": cfg.gate_kind, "global_batch_tokens": T * world,
-                   "mode": ("expert-parallel: NCCL all-to-all dispatch/return, rows "
+                   "mode": ("expert-parallel over peer memory: rows stored into and read "
+                            "back from the owners' buffers by the library's kernels, plan on "
+                            "the device" if args.parallel == "ep-p2p" else
+                            "expert-parallel: NCCL all-to-all dispatch/return, rows "
                             "regrouped by expert on the receiving rank" if ep_mode else
-                            "fused gather" if lay.fused_gather else "five-call"),
+                            "fused gather" if lay.fused_gather else
+                            "fused scatter" if lay.fused_scatter else "five-call"),
                    "shared_expert": "side stream, overlapped" if lay.overlap_shared
                    else "after the routed experts",
                    "parallelism": (f"ep{world}" if ep_mode else
@@ -815,6 +838,8 @@ def main():
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1 or ep_mode:
+        if hasattr(lay, "close"):
+            lay.close()
         dist.barrier()
         dist.destroy_process_group()
 

@@ -194,8 +194,8 @@ MOE_API int moe_permute_noalloc(const void* u, const int32_t* topk_idx,
  * dtype MOE_FP8_E4M3: x, w13, w2 are E4M3 codes (1 byte) with fp32 scales
  *   x_scales [rows, d/128], w13_scales [G, 2, inter/128, d/128] (w13 packed by
  *   moe_pack_w13_fp8), w2_scales [G, d/128, inter/128] (see the FP8 section);
- *   y stays bf16; workspace holds h as bf16 [rows, inter], then as E4M3
- *   [rows, inter] + its scales [rows, inter/128].
+ *   y stays bf16; workspace holds h as E4M3 codes [rows, inter] + its
+ *   scales [rows, inter/128] (quantised in the up-projection's epilogue).
  */
 MOE_API int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_offsets,
                             int G, int rows, int d, int inter, const void* w13,
@@ -233,8 +233,8 @@ MOE_API int moe_expert_down(const void* h, const int32_t* group_offsets, int G, 
  * 448 = largest E4M3 value). Codes are decided in fp32: scale = amax / 448
  * (an all-zero tile gets 1) and x / scale are IEEE fp32 divisions, the
  * quotient is rounded to E4M3 to nearest-even, saturating at +-448. The
- * intermediate h is held in bf16 between the two GEMMs (as in the bf16 path)
- * and quantised from that value.
+ * intermediate h is quantised in the up-projection's epilogue straight from
+ * its fp32 value (it never goes to memory in a wider type).
  * E4M3 tensors are 1 byte per element, 16-B aligned; scales fp32, 4-B aligned.
  * The routing (moe_route) stays bf16: the expert indices must be exact.
  *
@@ -248,16 +248,18 @@ MOE_API int moe_expert_down(const void* h, const int32_t* group_offsets, int G, 
  *   then pack the codes into w13 [G, 2*inter, d] with 64-row chunks
  *   interleaved (W1 rows 0..63, W3 rows 0..63, W1 rows 64..127, ...).
  *   inter % 64 == 0.
- * moe_permute_fp8: moe_permute for E4M3 rows: u8 [T, d] codes + u_scales
- *   [T, d/128] (from moe_quant_act_fp8, quantised once per token) are copied
- *   to x8 [T*top_k, d] + x_scales [T*top_k, d/128]; other arguments as
- *   moe_permute.
+ * moe_permute_fp8: moe_permute with E4M3 rows out: each token's bf16 row of
+ *   u [T, d] is quantised once (1x128 tiles, the rule above) and its codes
+ *   and tile scales are written to each of its rows of x8 [T*top_k, d] and
+ *   x_scales [T*top_k, d/128]; with u8 [T, d] and u_scales [T, d/128] given
+ *   (both or neither), also to the token's own row there (the shared
+ *   expert's input). Other arguments as moe_permute.
  * moe_expert_up_swiglu_fp8 / moe_expert_down_fp8: the two halves of
  *   moe_grouped_ffn in FP8. The first reads x8/x_scales and the packed w13 with
- *   w13_scales [G, 2, inter/128, d/128] and writes h = silu(a) * b as bf16
- *   [rows, inter]; the caller quantises h per 1x128 tile with
- *   moe_quant_act_fp8 (h8, h_scales); the second reads h8/h_scales and w2 with
- *   w2_scales [G, d/128, inter/128] and writes bf16 y.
+ *   w13_scales [G, 2, inter/128, d/128] and writes h = silu(a) * b quantised:
+ *   codes h8 [rows, inter] (16-B aligned) and scales h_scales [rows,
+ *   inter/128]; the second reads h8/h_scales and w2 with w2_scales [G, d/128,
+ *   inter/128] and writes bf16 y.
  */
 MOE_API int moe_quant_act_fp8(const void* x, int rows, int cols, void* q, float* scales,
                               moe_stream_t stream);
@@ -265,15 +267,15 @@ MOE_API int moe_quant_weights_fp8(const void* w, int G, int R, int C, void* q, f
                                   moe_stream_t stream);
 MOE_API int moe_pack_w13_fp8(const void* w13_stacked, int G, int inter, int d, void* w13,
                              moe_stream_t stream);
-MOE_API int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_idx,
-                            const int32_t* expert_counts, int T, int d, int n_routed, int top_k,
-                            void* x8, float* x_scales, int32_t* expert_offsets, int32_t* pos,
+MOE_API int moe_permute_fp8(const void* u, const int32_t* topk_idx, const int32_t* expert_counts,
+                            int T, int d, int n_routed, int top_k, void* x8, float* x_scales,
+                            void* u8, float* u_scales, int32_t* expert_offsets, int32_t* pos,
                             int32_t* src_token, void* workspace, size_t ws_bytes,
                             moe_stream_t stream);
 MOE_API int moe_expert_up_swiglu_fp8(const void* x8, const float* x_scales,
                                      const int32_t* group_offsets, int G, int rows, int d,
-                                     int inter, const void* w13, const float* w13_scales, void* h,
-                                     moe_stream_t stream);
+                                     int inter, const void* w13, const float* w13_scales,
+                                     void* h8, float* h_scales, moe_stream_t stream);
 MOE_API int moe_expert_down_fp8(const void* h8, const float* h_scales,
                                 const int32_t* group_offsets, int G, int rows, int inter, int d,
                                 const void* w2, const float* w2_scales, void* y,
@@ -475,6 +477,70 @@ MOE_API int moe_ep_plan(const int32_t* local_counts, const int32_t* recv_counts,
 MOE_API int moe_gather_rows(const void* src, int n_src, const int32_t* index, int n, int d,
                             void* dst, moe_stream_t stream);
 
+/* ------------------------------------------------------------------ expert parallelism over peer memory
+ * The same split of the experts over W ranks, with the token rows moved by
+ * this library's own kernels through peer memory instead of all-to-all
+ * collectives, and every step planned on the device (no host read):
+ *   moe_route, moe_permute_index        this rank's tokens (no row copy)
+ *   all-gather of the loads             all_counts [W, n_routed] int32 (the
+ *                                       caller's collective, e.g. NCCL)
+ *   moe_ep_plan_device                  where this rank's rows go
+ *   moe_ep_dispatch_p2p                 rows stored into the owners' buffers
+ *   barrier (caller)                    every rank's stores have landed
+ *   moe_expert_up_swiglu, moe_expert_down   on x_recv, G = n_local, rows =
+ *                                       its capacity, the plan's offsets
+ *   barrier (caller)                    every owner's outputs are written
+ *   moe_ep_combine_p2p                  each token's K outputs read back
+ *   moe_bias_update(global_counts, ..., T summed over the ranks)
+ * Rank q's receive buffer x_recv [capacity, d] is expert-major: expert e's
+ * rows from rank 0, then from rank 1, ..., each in that rank's token order
+ * (the order one GPU's stable dispatch gives the ranks' batches laid end to
+ * end), so the result equals the single-GPU layer on that batch. The
+ * buffers of the other ranks are reached through peer pointers (CUDA IPC,
+ * moe_ipc_*); with one rank they are local. Plain peer loads and stores, no
+ * TMA multicast.
+ *
+ * moe_ep_plan_device: one small kernel. all_counts [world, world*n_local]
+ *   (row q = rank q's moe_route counts); writes dest_row [n_routed] (first row
+ *   of this rank's rows for expert E in its owner's receive buffer),
+ *   group_offsets [n_local + 1] (this rank's own receive buffer, expert-major)
+ *   and global_counts [n_routed] (the loads summed over the ranks). A receive
+ *   buffer that would need more than recv_capacity rows sets bit 16 of the
+ *   device status word (moe_get_device_status then returns
+ *   MOE_ERR_DEVICE_TIMEOUT); the rows past the capacity are not moved.
+ *   world * n_local <= 256.
+ * moe_ep_dispatch_p2p: token t's row of u goes to row dest_row[E] + pos[t,k]
+ *   - expert_offsets[E] of peer_x[E / n_local], for each slot k with E =
+ *   topk_idx[t,k]. peer_x: DEVICE array of `world` pointers to the ranks'
+ *   receive buffers [recv_capacity, d] bf16 (16-B aligned), as mapped on this
+ *   GPU. pos, expert_offsets: moe_permute_index's.
+ * moe_ep_combine_p2p: moe_combine whose routed rows are read from
+ *   peer_y[E / n_local] at the rows the dispatch wrote (peer_y: DEVICE array
+ *   of `world` pointers to the ranks' expert output buffers [recv_capacity,
+ *   d] bf16). out may alias residual.
+ * moe_ipc_get_handle: the 64-byte CUDA IPC handle of the allocation that
+ *   holds dev_ptr, and dev_ptr's byte offset in it. moe_ipc_open_handle maps
+ *   a handle from another process on this GPU (*base = the allocation's
+ *   start; add the offset); moe_ipc_close_handle unmaps it.
+ */
+MOE_API int moe_ep_plan_device(const int32_t* all_counts, int world, int n_local, int rank,
+                               long long recv_capacity, int32_t* dest_row,
+                               int32_t* group_offsets, int32_t* global_counts,
+                               moe_stream_t stream);
+MOE_API int moe_ep_dispatch_p2p(const void* u, const int32_t* topk_idx, const int32_t* pos,
+                                const int32_t* expert_offsets, const int32_t* dest_row, int T,
+                                int d, int n_routed, int top_k, int world, void* const* peer_x,
+                                long long recv_capacity, moe_stream_t stream);
+MOE_API int moe_ep_combine_p2p(const void* const* peer_y, const int32_t* topk_idx,
+                               const int32_t* pos, const int32_t* expert_offsets,
+                               const int32_t* dest_row, const float* topk_gate,
+                               const void* shared_out, const void* residual, int T, int d,
+                               int n_routed, int top_k, int world, long long recv_capacity,
+                               void* out, moe_stream_t stream);
+MOE_API int moe_ipc_get_handle(const void* dev_ptr, void* handle, long long* offset);
+MOE_API int moe_ipc_open_handle(const void* handle, void** base);
+MOE_API int moe_ipc_close_handle(void* base);
+
 /* ------------------------------------------------------------------ helpers
  * moe_pack_w13: build the interleaved w13 [G, 2*inter, d] from w1 and w3
  * [G, inter, d] (all bf16, 16-B aligned; layout described at moe_grouped_ffn).
@@ -489,7 +555,9 @@ MOE_API const char* moe_strerror(int status);
 MOE_API int moe_last_cuda_error(void);
 
 /* Synchronises the current device, then writes the device status word of the
- * current device (0 = no kernel timed out) to *status; clears it if `clear`.
+ * current device to *status; clears it if `clear`. Bits: 1, 2, 4 a pipeline
+ * wait of a GEMM ran out (producer, MMA, epilogue), 8 the self-test below,
+ * 16 an expert-parallel receive buffer was too small. 0 = none of these.
  * Returns MOE_ERR_DEVICE_TIMEOUT if the word was non-zero. */
 MOE_API int moe_get_device_status(unsigned int* status, int clear);
 
@@ -501,9 +569,12 @@ MOE_API int moe_get_device_status(unsigned int* status, int clear);
  * counterpart in the pages. */
 MOE_API int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream);
 
-/* Library version, major*10000 + minor*100 + patch. 0.2.0 (200) adds, over
+/* Library version, major*10000 + minor*100 + patch. 0.2.0 (200) added, over
  * the forward's five calls of 0.1.0: the FP8 variant, the fused-gather
- * up-projection, the backward and the expert-parallel entry points. */
+ * up-projection, the backward and the expert-parallel entry points. 0.3.0
+ * (300): the fused scatter, expert parallelism over peer memory, the FP8
+ * dispatch and up-projection quantising in place (their signatures
+ * changed), device-side clamping of group offsets. */
 MOE_API int moe_version(void);
 
 #ifdef __cplusplus

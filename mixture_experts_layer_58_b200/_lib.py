@@ -57,9 +57,9 @@ _SIGS = {
     "moe_expert_down": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "moe_quant_act_fp8": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "moe_quant_weights_fp8": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
-    "moe_permute_fp8": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
-                             _sz, _vp]),
-    "moe_expert_up_swiglu_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_permute_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                             _vp, _sz, _vp]),
+    "moe_expert_up_swiglu_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
     "moe_pack_w13_fp8": (_i, [_vp, _i, _i, _i, _vp, _vp]),
     "moe_expert_down_fp8": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
@@ -86,6 +86,13 @@ _SIGS = {
     "moe_ep_plan": (_i, [_vp, _vp, _i, _i, _ll, _vp, _vp, _vp, _vp, _vp,
                          ctypes.POINTER(ctypes.c_longlong)]),
     "moe_gather_rows": (_i, [_vp, _i, _vp, _i, _i, _vp, _vp]),
+    "moe_ep_plan_device": (_i, [_vp, _i, _i, _i, _ll, _vp, _vp, _vp, _vp]),
+    "moe_ep_dispatch_p2p": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _ll, _vp]),
+    "moe_ep_combine_p2p": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                _ll, _vp, _vp]),
+    "moe_ipc_get_handle": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_longlong)]),
+    "moe_ipc_open_handle": (_i, [_vp, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_ipc_close_handle": (_i, [_vp]),
 }
 
 _LIB = None
@@ -207,19 +214,19 @@ def moe_quant_weights_fp8(w, G, R, C, q, scales, stream=None):
            "moe_quant_weights_fp8")
 
 
-def moe_permute_fp8(u8, u_scales, topk_idx, expert_counts, T, d, n_routed, top_k, x8, x_scales,
-                    expert_offsets, pos, src_token, workspace, ws_bytes, stream=None):
-    _check(_L().moe_permute_fp8(_p(u8), _p(u_scales), _p(topk_idx), _p(expert_counts), T, d,
-                                n_routed, top_k, _p(x8), _p(x_scales), _p(expert_offsets), _p(pos),
-                                _p(src_token), _p(workspace), ws_bytes, _stream(stream)),
+def moe_permute_fp8(u, topk_idx, expert_counts, T, d, n_routed, top_k, x8, x_scales, u8,
+                    u_scales, expert_offsets, pos, src_token, workspace, ws_bytes, stream=None):
+    _check(_L().moe_permute_fp8(_p(u), _p(topk_idx), _p(expert_counts), T, d, n_routed, top_k,
+                                _p(x8), _p(x_scales), _p(u8), _p(u_scales), _p(expert_offsets),
+                                _p(pos), _p(src_token), _p(workspace), ws_bytes, _stream(stream)),
            "moe_permute_fp8")
 
 
-def moe_expert_up_swiglu_fp8(x8, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales, h,
-                             stream=None):
+def moe_expert_up_swiglu_fp8(x8, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales, h8,
+                             h_scales, stream=None):
     _check(_L().moe_expert_up_swiglu_fp8(_p(x8), _p(x_scales), _p(group_offsets), G, rows, d,
-                                         inter, _p(w13), _p(w13_scales), _p(h), _stream(stream)),
-           "moe_expert_up_swiglu_fp8")
+                                         inter, _p(w13), _p(w13_scales), _p(h8), _p(h_scales),
+                                         _stream(stream)), "moe_expert_up_swiglu_fp8")
 
 
 def moe_pack_w13_fp8(w13_stacked, G, inter, d, w13, stream=None):
@@ -297,6 +304,48 @@ def moe_ep_plan(local_counts, recv_counts, world, n_local, recv_capacity, send_s
 def moe_gather_rows(src, n_src, index, n, d, dst, stream=None):
     _check(_L().moe_gather_rows(_p(src), n_src, _p(index), n, d, _p(dst), _stream(stream)),
            "moe_gather_rows")
+
+
+def moe_ep_plan_device(all_counts, world, n_local, rank, recv_capacity, dest_row,
+                       group_offsets, global_counts, stream=None):
+    _check(_L().moe_ep_plan_device(_p(all_counts), world, n_local, rank, int(recv_capacity),
+                                   _p(dest_row), _p(group_offsets), _p(global_counts),
+                                   _stream(stream)), "moe_ep_plan_device")
+
+
+def moe_ep_dispatch_p2p(u, topk_idx, pos, expert_offsets, dest_row, T, d, n_routed, top_k,
+                        world, peer_x, recv_capacity, stream=None):
+    _check(_L().moe_ep_dispatch_p2p(_p(u), _p(topk_idx), _p(pos), _p(expert_offsets),
+                                    _p(dest_row), T, d, n_routed, top_k, world, _p(peer_x),
+                                    int(recv_capacity), _stream(stream)), "moe_ep_dispatch_p2p")
+
+
+def moe_ep_combine_p2p(peer_y, topk_idx, pos, expert_offsets, dest_row, topk_gate, shared_out,
+                       residual, T, d, n_routed, top_k, world, recv_capacity, out, stream=None):
+    _check(_L().moe_ep_combine_p2p(_p(peer_y), _p(topk_idx), _p(pos), _p(expert_offsets),
+                                   _p(dest_row), _p(topk_gate), _p(shared_out), _p(residual), T,
+                                   d, n_routed, top_k, world, int(recv_capacity), _p(out),
+                                   _stream(stream)), "moe_ep_combine_p2p")
+
+
+def moe_ipc_get_handle(tensor) -> tuple:
+    """(64-byte IPC handle of the allocation holding tensor's data, byte offset)."""
+    h = ctypes.create_string_buffer(64)
+    off = ctypes.c_longlong(0)
+    _check(_L().moe_ipc_get_handle(_p(tensor), h, ctypes.byref(off)), "moe_ipc_get_handle")
+    return h.raw, off.value
+
+
+def moe_ipc_open_handle(handle: bytes) -> int:
+    """Map another process's allocation on this GPU; returns its base address."""
+    base = ctypes.c_void_p(0)
+    _check(_L().moe_ipc_open_handle(ctypes.create_string_buffer(handle, 64), ctypes.byref(base)),
+           "moe_ipc_open_handle")
+    return base.value
+
+
+def moe_ipc_close_handle(base: int) -> None:
+    _check(_L().moe_ipc_close_handle(base), "moe_ipc_close_handle")
 
 
 def moe_get_device_status(clear: bool = True) -> int:

@@ -127,17 +127,20 @@ quant_weight_fp8_kernel(const __nv_bfloat16* __restrict__ w, int R, int C,
 }
 
 // ---------------------------------------------------------------- dispatch
-// FP8 form of the permute copy: each token's E4M3 row (d bytes) and its d/128
-// tile scales, written to each of its K rows.
+// FP8 dispatch with the activation quantisation fused in: one warp per token
+// reads its bf16 row once, quantises every 1x128 tile by the rule of
+// quant_act_fp8_kernel (lanes 0-15 tile 2i, lanes 16-31 tile 2i+1) and writes
+// the codes and the tile's scale to each of the token's K rows of x8 / xs;
+// with u8 given, also to the token's own row of u8 / us (the shared expert's
+// input). Each token is quantised once, however many experts it goes to.
 __global__ void __launch_bounds__(256)
-permute_copy_fp8_kernel(const uint8_t* __restrict__ u8, const float* __restrict__ us,
-                        const int32_t* __restrict__ pos, int T, int d, int K,
-                        uint8_t* __restrict__ x8, float* __restrict__ xs) {
+permute_quant_fp8_kernel(const __nv_bfloat16* __restrict__ u, const int32_t* __restrict__ pos,
+                         int T, int d, int K, uint8_t* __restrict__ x8, float* __restrict__ xs,
+                         uint8_t* __restrict__ u8, float* __restrict__ us) {
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const long long total = static_cast<long long>(T) * K;
-  const int nvec = d >> 4;
-  const int ns = d / kQBlock;
+  const int tiles = d / kQBlock;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     const int my = lane < K ? pos[static_cast<size_t>(t) * K + lane] : -1;
     int p[kMaxTopK];
@@ -146,26 +149,44 @@ permute_copy_fp8_kernel(const uint8_t* __restrict__ u8, const float* __restrict_
       p[k] = __shfl_sync(0xffffffffu, my, k);
       if (k >= K || p[k] < 0 || p[k] >= total) p[k] = -1;
     }
-    const uint4* srow = reinterpret_cast<const uint4*>(u8 + static_cast<size_t>(t) * d);
-    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
-      uint4 x[4];
+    const __nv_bfloat16* ur = u + static_cast<size_t>(t) * d;
+    for (int t0 = 0; t0 < tiles; t0 += 2) {
+      const int tile = t0 + (lane >> 4);
+      const bool active = tile < tiles;
+      float v[8];
+      float m = 0.0f;
+      if (active) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(ur + tile * kQBlock) + (lane & 15));
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (v0 + 32 * j < nvec) x[j] = __ldg(srow + v0 + 32 * j);
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h[i]);
+          v[2 * i] = f.x;
+          v[2 * i + 1] = f.y;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+      }
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (!active) continue;
+      const float s = fp8_scale_of(m);
+      uint2 q;
+      q.x = to_e4m3x4(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s), __fdiv_rn(v[2], s),
+                      __fdiv_rn(v[3], s));
+      q.y = to_e4m3x4(__fdiv_rn(v[4], s), __fdiv_rn(v[5], s), __fdiv_rn(v[6], s),
+                      __fdiv_rn(v[7], s));
+      const size_t col = static_cast<size_t>(tile) * kQBlock;
 #pragma unroll
       for (int k = 0; k < kMaxTopK; ++k) {
         if (p[k] < 0) continue;
-        uint4* drow = reinterpret_cast<uint4*>(x8 + static_cast<size_t>(p[k]) * d);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (v0 + 32 * j < nvec) drow[v0 + 32 * j] = x[j];
+        reinterpret_cast<uint2*>(x8 + static_cast<size_t>(p[k]) * d + col)[lane & 15] = q;
+        if ((lane & 15) == 0) xs[static_cast<size_t>(p[k]) * tiles + tile] = s;
       }
-    }
-    for (int i = lane; i < ns; i += 32) {
-      const float s = us[static_cast<size_t>(t) * ns + i];
-#pragma unroll
-      for (int k = 0; k < kMaxTopK; ++k)
-        if (p[k] >= 0) xs[static_cast<size_t>(p[k]) * ns + i] = s;
+      if (u8) {
+        reinterpret_cast<uint2*>(u8 + static_cast<size_t>(t) * d + col)[lane & 15] = q;
+        if ((lane & 15) == 0) us[static_cast<size_t>(t) * tiles + tile] = s;
+      }
     }
   }
 }

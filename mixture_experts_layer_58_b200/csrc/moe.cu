@@ -201,7 +201,8 @@ int make_tmap_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 template <int EPI>
 int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int K, const void* B,
                             const float* b_scales, int G, int n_per_group,
-                            const int32_t* offsets, void* out, int ldo, cudaStream_t st) {
+                            const int32_t* offsets, void* out, int ldo, cudaStream_t st,
+                            void* qout = nullptr, float* qscales = nullptr) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
@@ -212,13 +213,14 @@ int launch_grouped_gemm_fp8(const void* A, const float* a_scales, int rows, int 
   const size_t smem = GemmF8Cfg::smem_bytes(G);
   auto kern = grouped_gemm_fp8_kernel<EPI>;
   if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
-  const long long max_tiles =
-      (static_cast<long long>(rows) / kBM + G) * static_cast<long long>(n_per_group / kF8BN);
+  const long long max_tiles = (static_cast<long long>(rows) / kBM + G) *
+                              static_cast<long long>(n_per_group / (kF8BN * f8_subtiles<EPI>()));
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, max_tiles)));
   int* counter = di->tile_counters + (di->next_counter.fetch_add(1) % kTileCounters);
   MOE_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   kern<<<grid, kF8Threads, smem, st>>>(tmA, tmB, a_scales, b_scales, offsets, G, K, n_per_group,
-                                       rows, static_cast<__nv_bfloat16*>(out), ldo, counter,
+                                       rows, static_cast<__nv_bfloat16*>(out), ldo,
+                                       static_cast<uint8_t*>(qout), qscales, counter,
                                        di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
@@ -384,7 +386,7 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, unsign
 
 extern "C" {
 
-int moe_version(void) { return 200; }
+int moe_version(void) { return 300; }
 
 int moe_selftest_wait_timeout(int limit_ms, moe_stream_t stream) {
   if (limit_ms <= 0 || limit_ms > 10000) return MOE_ERR_INVALID_ARG;
@@ -403,7 +405,7 @@ const char* moe_strerror(int s) {
     case MOE_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer, bad size or enum)";
     case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
     case MOE_ERR_CUDA: return "CUDA error (see moe_last_cuda_error)";
-    case MOE_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out, or a device-side limit was hit";
     case MOE_ERR_WORKSPACE: return "workspace missing or too small";
     default: return "unknown status";
   }
@@ -540,10 +542,9 @@ int moe_permute_index(const int32_t* topk_idx, const int32_t* expert_counts, int
 size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dtype) {
   if (rows <= 0 || inter <= 0) return 256;
   if (dtype == MOE_FP8_E4M3) {
-    const size_t hbf = (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
     const size_t codes = (static_cast<size_t>(rows) * inter + 255) / 256 * 256;
     const size_t scales = (static_cast<size_t>(rows) * (inter / 128) * 4 + 255) / 256 * 256;
-    return hbf + codes + scales;
+    return codes + scales;
   }
   return (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
 }
@@ -602,13 +603,10 @@ int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t* group_o
       !aligned16(workspace))
     return MOE_ERR_WORKSPACE;
   if (dtype == MOE_FP8_E4M3) {
-    uint8_t* hbf = static_cast<uint8_t*>(workspace);
-    uint8_t* h8 = hbf + (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
+    uint8_t* h8 = static_cast<uint8_t*>(workspace);
     float* hs = reinterpret_cast<float*>(h8 + (static_cast<size_t>(rows) * inter + 255) / 256 * 256);
     rc = moe_expert_up_swiglu_fp8(x, x_scales, group_offsets, G, rows, d, inter, w13, w13_scales,
-                                  hbf, stream);
-    if (rc != MOE_OK) return rc;
-    rc = moe_quant_act_fp8(hbf, rows, inter, h8, hs, stream);
+                                  h8, hs, stream);
     if (rc != MOE_OK) return rc;
     return moe_expert_down_fp8(h8, hs, group_offsets, G, rows, inter, d, w2, w2_scales, y, stream);
   }
@@ -648,9 +646,9 @@ int moe_quant_weights_fp8(const void* w, int G, int R, int C, void* q, float* sc
   return MOE_OK;
 }
 
-int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_idx,
-                    const int32_t* expert_counts, int T, int d, int n_routed, int top_k, void* x8,
-                    float* x_scales, int32_t* expert_offsets, int32_t* pos, int32_t* src_token,
+int moe_permute_fp8(const void* u, const int32_t* topk_idx, const int32_t* expert_counts, int T,
+                    int d, int n_routed, int top_k, void* x8, float* x_scales, void* u8,
+                    float* u_scales, int32_t* expert_offsets, int32_t* pos, int32_t* src_token,
                     void* workspace, size_t ws_bytes, moe_stream_t stream) {
   if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
   if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
@@ -662,8 +660,10 @@ int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_i
     MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (n_routed + 1), st));
     return MOE_OK;
   }
-  if (!u8 || !u_scales || !topk_idx || !x8 || !x_scales || !pos || !src_token ||
-      !aligned16(u8) || !aligned16(x8) || !aligned4(u_scales) || !aligned4(x_scales))
+  if (!u || !topk_idx || !x8 || !x_scales || !pos || !src_token || !aligned16(u) ||
+      !aligned16(x8) || !aligned4(x_scales))
+    return MOE_ERR_INVALID_ARG;
+  if ((u8 == nullptr) != (u_scales == nullptr) || (u8 && (!aligned16(u8) || !aligned4(u_scales))))
     return MOE_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < moe_permute_workspace_size(T, n_routed) || !aligned16(workspace))
     return MOE_ERR_WORKSPACE;
@@ -678,24 +678,27 @@ int moe_permute_fp8(const void* u8, const float* u_scales, const int32_t* topk_i
                                                expert_offsets, pos, src_token);
   MOE_CUDA(cudaGetLastError());
   const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
-  permute_copy_fp8_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint8_t*>(u8), u_scales, pos,
-                                                  T, d, top_k, static_cast<uint8_t*>(x8), x_scales);
+  permute_quant_fp8_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(u), pos, T,
+                                                   d, top_k, static_cast<uint8_t*>(x8), x_scales,
+                                                   static_cast<uint8_t*>(u8), u_scales);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
 
 int moe_expert_up_swiglu_fp8(const void* x8, const float* x_scales, const int32_t* group_offsets,
                              int G, int rows, int d, int inter, const void* w13,
-                             const float* w13_scales, void* h, moe_stream_t stream) {
+                             const float* w13_scales, void* h8, float* h_scales,
+                             moe_stream_t stream) {
   int rc = check_ffn_shape(G, rows, d, inter);
   if (rc != MOE_OK) return rc;
   if (rows == 0) return MOE_OK;
-  if (!x8 || !x_scales || !group_offsets || !w13 || !w13_scales || !h || !aligned16(x8) ||
-      !aligned16(w13) || !aligned16(h) || !aligned4(x_scales) || !aligned4(w13_scales))
+  if (!x8 || !x_scales || !group_offsets || !w13 || !w13_scales || !h8 || !h_scales ||
+      !aligned16(x8) || !aligned16(w13) || !aligned16(h8) || !aligned4(x_scales) ||
+      !aligned4(w13_scales) || !aligned4(h_scales))
     return MOE_ERR_INVALID_ARG;
-  return launch_grouped_gemm_fp8<EPI8_SWIGLU>(x8, x_scales, rows, d, w13, w13_scales, G,
-                                              2 * inter, group_offsets, h, inter,
-                                              as_stream(stream));
+  return launch_grouped_gemm_fp8<EPI8_SWIGLU_Q>(x8, x_scales, rows, d, w13, w13_scales, G,
+                                                2 * inter, group_offsets, nullptr, inter,
+                                                as_stream(stream), h8, h_scales);
 }
 
 int moe_pack_w13_fp8(const void* w13_stacked, int G, int inter, int d, void* w13,
@@ -834,6 +837,121 @@ int moe_ep_plan(const int32_t* local_counts, const int32_t* recv_counts, int wor
                                    send_splits, recv_splits, group_offsets, regroup, ungroup);
   if (r < 0) return MOE_ERR_INVALID_ARG;
   *n_recv = r;
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ expert parallelism over peer memory
+int moe_ep_plan_device(const int32_t* all_counts, int world, int n_local, int rank,
+                       long long recv_capacity, int32_t* dest_row, int32_t* group_offsets,
+                       int32_t* global_counts, moe_stream_t stream) {
+  if (world < 1 || n_local < 1 || rank < 0 || rank >= world || recv_capacity < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (static_cast<long long>(world) * n_local > kRouteMaxExperts)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!all_counts || !dest_row || !group_offsets || !global_counts) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  ep_plan_device_kernel<<<1, 256, 0, as_stream(stream)>>>(all_counts, world, n_local, rank,
+                                                          recv_capacity, dest_row, group_offsets,
+                                                          global_counts, di->status);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_ep_dispatch_p2p(const void* u, const int32_t* topk_idx, const int32_t* pos,
+                        const int32_t* expert_offsets, const int32_t* dest_row, int T, int d,
+                        int n_routed, int top_k, int world, void* const* peer_x,
+                        long long recv_capacity, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0 || world < 1 || recv_capacity < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 8 != 0 ||
+      n_routed % world != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!u || !topk_idx || !pos || !expert_offsets || !dest_row || !peer_x || !aligned16(u))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
+  ep_dispatch_p2p_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(u), topk_idx, pos, expert_offsets, dest_row, T, d, top_k,
+      n_routed, n_routed / world, reinterpret_cast<__nv_bfloat16* const*>(peer_x),
+      recv_capacity);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_ep_combine_p2p(const void* const* peer_y, const int32_t* topk_idx, const int32_t* pos,
+                       const int32_t* expert_offsets, const int32_t* dest_row,
+                       const float* topk_gate, const void* shared_out, const void* residual,
+                       int T, int d, int n_routed, int top_k, int world, long long recv_capacity,
+                       void* out, moe_stream_t stream) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0 || world < 1 || recv_capacity < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 8 != 0 ||
+      n_routed % world != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!peer_y || !topk_idx || !pos || !expert_offsets || !dest_row || !topk_gate || !out ||
+      !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if ((shared_out && !aligned16(shared_out)) || (residual && !aligned16(residual)))
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc != MOE_OK) return rc;
+  const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
+  ep_combine_p2p_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16* const*>(peer_y), topk_idx, pos, expert_offsets,
+      dest_row, topk_gate, static_cast<const __nv_bfloat16*>(shared_out),
+      static_cast<const __nv_bfloat16*>(residual), T, d, top_k, n_routed, n_routed / world,
+      recv_capacity, static_cast<__nv_bfloat16*>(out));
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+int moe_ipc_get_handle(const void* dev_ptr, void* handle, long long* offset) {
+  if (!dev_ptr || !handle || !offset) return MOE_ERR_INVALID_ARG;
+  static PFN_cuMemGetAddressRange_v3020 range = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
+  });
+  if (!range) return cuda_fail(cudaErrorNotSupported);
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  const CUresult r = range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr));
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return MOE_ERR_CUDA;
+  }
+  cudaIpcMemHandle_t h;
+  MOE_CUDA(cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)));
+  std::memcpy(handle, &h, sizeof(h));
+  *offset = static_cast<long long>(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+  return MOE_OK;
+}
+
+int moe_ipc_open_handle(const void* handle, void** base) {
+  if (!handle || !base) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  MOE_CUDA(cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess));
+  return MOE_OK;
+}
+
+int moe_ipc_close_handle(void* base) {
+  if (!base) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(cudaIpcCloseMemHandle(base));
   return MOE_OK;
 }
 

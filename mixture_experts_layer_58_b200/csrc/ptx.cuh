@@ -14,6 +14,7 @@ enum : unsigned int {
   kStatusTimeoutMma = 2u,
   kStatusTimeoutEpilogue = 4u,
   kStatusTimeoutSelfTest = 8u,
+  kStatusEpOverflow = 16u,        // a peer-memory receive buffer was too small (not a wait)
 };
 
 // Upper bound for any single wait on an mbarrier, in nanoseconds of the

@@ -281,3 +281,232 @@ class ExpertParallelMoELayer(MoELayer):
         if self.gate_kind == "sigmoid":
             n += 1
         return n
+
+
+class PeerExpertParallelMoELayer(MoELayer):
+    """Expert parallelism with the token rows moved through peer memory by the
+    library's own kernels, planned on the device (bf16 forward).
+
+    Rank p holds the routed experts [p*n_local, (p+1)*n_local), as in
+    ExpertParallelMoELayer; the centroids, the bias and the shared expert are
+    replicated. One forward on every rank (all ranks call it with the same T):
+
+        moe_route, moe_permute_index   this rank's tokens, no row copy
+        all-gather of the loads        all_counts [W, N_r] (NCCL, on the device)
+        moe_ep_plan_device             rows' destinations, own group offsets,
+                                       loads summed over the ranks
+        moe_ep_dispatch_p2p            each token row stored into its experts'
+                                       owners' receive buffers
+        barrier                        (a one-element all-reduce)
+        up- and down-projection        on the receive buffer, expert-major
+        barrier
+        moe_ep_combine_p2p             each token's K outputs read back from
+                                       the owners, gate-weighted, + shared + u
+
+    Nothing is read back to the host. The receive buffers hold recv_capacity
+    rows (default W*T*K, every rank's every row: no step can overflow); the
+    other ranks' buffers are mapped with CUDA IPC. With world/rank given and no
+    group the layer is one of several ranks emulated in one process: the
+    caller links them with link_emulated_ranks and drives the stages (begin,
+    plan, dispatch, experts, finish) in rank order, which needs no kernel to
+    wait on another."""
+
+    def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
+                 routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
+                 group=None, world: int | None = None, rank: int | None = None,
+                 recv_capacity: int | None = None, overlap_shared: bool = True, device="cuda"):
+        self.group = group
+        self.emulated = world is not None and group is None
+        self.world = dist.get_world_size(group) if world is None else int(world)
+        self.rank = dist.get_rank(group) if rank is None else int(rank)
+        n_routed = centroids.shape[0]
+        if n_routed % self.world:
+            raise ValueError(f"{n_routed} routed experts do not split over {self.world} ranks")
+        self.n_local = n_routed // self.world
+        self.expert_lo = self.rank * self.n_local
+        if w1.shape[0] == n_routed and self.n_local != n_routed:
+            sl = slice(self.expert_lo, self.expert_lo + self.n_local)
+            w1, w3, w2 = w1[sl], w3[sl], w2[sl]
+        if w1.shape[0] != self.n_local:
+            raise ValueError(f"expected {self.n_local} or {n_routed} experts, got {w1.shape[0]}")
+        super().__init__(centroids, bias, w1, w3, w2, shared, top_k=top_k,
+                         routed_scale=routed_scale, gate_kind=gate_kind, gamma=gamma,
+                         fused_gather=True, overlap_shared=overlap_shared, device=device)
+        self.recv_capacity_arg = recv_capacity
+        self._mapped = []          # IPC bases opened on this GPU
+        self._recv_T = -1
+
+    # ------------------------------------------------------------------ buffers
+    def allocate(self, T: int) -> None:
+        super().allocate(T)
+        if T == self._recv_T:
+            return
+        dev, bf = self.device, torch.bfloat16
+        cap = (int(self.recv_capacity_arg) if self.recv_capacity_arg is not None
+               else max(1, self.world * T * self.top_k))
+        self._unmap_peers()
+        self.recv_capacity = cap
+        self.x_recv = torch.empty((cap, self.d), dtype=bf, device=dev)
+        self.h_recv = torch.empty((cap, self.inter), dtype=bf, device=dev)
+        self.y_recv = torch.empty((cap, self.d), dtype=bf, device=dev)
+        i32 = torch.int32
+        self.all_counts = torch.zeros((self.world, self.n_routed), dtype=i32, device=dev)
+        self.dest_row = torch.empty(self.n_routed, dtype=i32, device=dev)
+        self.goff = torch.empty(self.n_local + 1, dtype=i32, device=dev)
+        self.global_counts = torch.empty(self.n_routed, dtype=i32, device=dev)
+        self._barrier_t = torch.zeros(1, dtype=i32, device=dev)
+        self._recv_T = T
+        if not self.emulated:
+            self._map_peers()
+
+    def _unmap_peers(self):
+        if not self._mapped:
+            return
+        # every rank closes its mappings before any rank frees the buffers
+        for base in self._mapped:
+            L.moe_ipc_close_handle(base)
+        self._mapped = []
+        dist.barrier(group=self.group)
+
+    def _map_peers(self):
+        """Pointer tables of the ranks' receive and output buffers as seen
+        from this GPU (one all-gather of the IPC handles)."""
+        xs, ys = [0] * self.world, [0] * self.world
+        xs[self.rank], ys[self.rank] = self.x_recv.data_ptr(), self.y_recv.data_ptr()
+        if self.world > 1:
+            mine = (L.moe_ipc_get_handle(self.x_recv), L.moe_ipc_get_handle(self.y_recv))
+            allh = [None] * self.world
+            dist.all_gather_object(allh, mine, group=self.group)
+            for q in range(self.world):
+                if q == self.rank:
+                    continue
+                (hx, ox), (hy, oy) = allh[q]
+                bx, by = L.moe_ipc_open_handle(hx), L.moe_ipc_open_handle(hy)
+                self._mapped += [bx, by]
+                xs[q], ys[q] = bx + ox, by + oy
+        self.set_peer_tables(xs, ys)
+
+    def set_peer_tables(self, x_ptrs, y_ptrs):
+        """Device tables of the W receive (x) and output (y) buffer addresses."""
+        self.peer_x = torch.tensor(x_ptrs, dtype=torch.int64, device=self.device)
+        self.peer_y = torch.tensor(y_ptrs, dtype=torch.int64, device=self.device)
+
+    # ------------------------------------------------------------------ stages
+    def begin(self, u, timers=None):
+        """Route this rank's tokens and compute their dispatch rows (and start
+        the shared expert on the side stream). Leaves the loads in self.counts."""
+        assert u.dtype == torch.bfloat16 and u.is_contiguous() and u.device.type == "cuda"
+        T = u.shape[0]
+        self.allocate(T)
+        ev = _Timed(timers)
+        self._side_used = False
+        if T > 0 and self.ws13 is not None and self.overlap_shared:
+            side = self._fork()
+            u.record_stream(side)
+            with torch.cuda.stream(side):
+                with ev("shared"):
+                    self.shared_ffn(u)
+            self._join_event.record(side)
+            self._side_used = True
+        with ev("route"):
+            self.route(u)
+        with ev("permute"):
+            self.permute(u)
+
+    def plan(self):
+        """Device plan from self.all_counts (every rank's loads)."""
+        L.moe_ep_plan_device(self.all_counts, self.world, self.n_local, self.rank,
+                             self.recv_capacity, self.dest_row, self.goff, self.global_counts)
+
+    def dispatch(self, u, timers=None):
+        with _Timed(timers)("dispatch"):
+            L.moe_ep_dispatch_p2p(u, self.topk_idx, self.pos, self.offsets, self.dest_row,
+                                  u.shape[0], self.d, self.n_routed, self.top_k, self.world,
+                                  self.peer_x, self.recv_capacity)
+
+    def experts(self, timers=None):
+        """This rank's experts on its receive buffer (the group offsets come
+        from the device plan; rows past them are never touched)."""
+        ev = _Timed(timers)
+        cap = self.recv_capacity
+        with ev("up"):
+            L.moe_expert_up_swiglu(self.x_recv, self.goff, self.n_local, cap, self.d, self.inter,
+                                   self.w13, self.h_recv)
+        with ev("down"):
+            L.moe_expert_down(self.h_recv, self.goff, self.n_local, cap, self.inter, self.d,
+                              self.w2, self.y_recv)
+
+    def finish(self, u, residual: bool = True, out=None, timers=None):
+        T = u.shape[0]
+        dst = self.out if out is None else out
+        assert dst.shape == (T, self.d) and dst.dtype == torch.bfloat16 and dst.is_contiguous()
+        ev = _Timed(timers)
+        if T > 0:
+            if self._side_used:
+                torch.cuda.current_stream().wait_event(self._join_event)
+            elif self.ws13 is not None:
+                with ev("shared"):
+                    self.shared_ffn(u)
+            with ev("combine"):
+                L.moe_ep_combine_p2p(self.peer_y, self.topk_idx, self.pos, self.offsets,
+                                     self.dest_row, self.topk_gate, self.shared_out,
+                                     u if residual else None, T, self.d, self.n_routed,
+                                     self.top_k, self.world, self.recv_capacity, dst)
+        return dst
+
+    def _barrier(self):
+        dist.all_reduce(self._barrier_t, group=self.group)
+
+    # ------------------------------------------------------------------ forward
+    def forward(self, u, residual: bool = True, out=None, train: bool = False, timers=None):
+        """h' for this rank's tokens u [T, d] (bf16, device). Every rank of the
+        group calls it with the same T (the exchanges are collectives)."""
+        if train:
+            raise ValueError("the expert-parallel layer runs the forward only")
+        if self.emulated:
+            raise RuntimeError("an emulated rank is driven through its stages")
+        self.begin(u, timers)
+        with _Timed(timers)("exchange_counts"):
+            dist.all_gather_into_tensor(self.all_counts.view(-1), self.counts, group=self.group)
+        self.plan()
+        self.dispatch(u, timers)
+        self._barrier()
+        self.experts(timers)
+        self._barrier()
+        return self.finish(u, residual, out, timers)
+
+    def update_bias(self, counts=None, T=None):
+        """End-of-step bias update from the loads summed over the ranks (the
+        device plan's global_counts) and the tokens of all ranks."""
+        T_all = self.world * self._T if T is None else T
+        L.moe_bias_update(self.global_counts if counts is None else counts, self.bias,
+                          self.n_routed, T_all, self.top_k, self.gamma)
+
+    def step(self, u):
+        out = self.forward(u)
+        if self.gate_kind == "sigmoid":
+            self.update_bias()
+        return out
+
+    # route (1 + a memset), permute index (2), plan, dispatch, up, down, shared
+    # FFN (2), combine; the all-gather and the barriers are NCCL's
+    def launches_per_step(self) -> int:
+        n = 1 + 2 + 1 + 1 + 2 + 1
+        if self.ws13 is not None:
+            n += 2
+        if self.gate_kind == "sigmoid":
+            n += 1
+        return n
+
+    def close(self):
+        """Unmap the other ranks' buffers (collective: every rank calls it)."""
+        self._unmap_peers()
+
+
+def link_emulated_ranks(layers) -> None:
+    """Point every emulated rank's peer tables at the buffers of all of them
+    (ranks emulated in one process on one GPU, in rank order)."""
+    xs = [lay.x_recv.data_ptr() for lay in layers]
+    ys = [lay.y_recv.data_ptr() for lay in layers]
+    for lay in layers:
+        lay.set_peer_tables(xs, ys)

@@ -194,10 +194,11 @@ class MoELayer:
                 L.moe_slot_index(self.pos, T, self.top_k, T * self.top_k, self.dst_slot)
             return
         if self.fp8:
-            # quantise each token once (1x128 tiles), then copy its codes K times
-            L.moe_quant_act_fp8(u, T, self.d, self.u8, self.u_s)
-            L.moe_permute_fp8(self.u8, self.u_s, self.topk_idx, self.counts, T, self.d,
-                              self.n_routed, self.top_k, self.x8, self.x_s, self.offsets,
+            # each token quantised once (1x128 tiles) inside the dispatch, its
+            # codes written to its K rows and to u8 for the shared expert
+            L.moe_permute_fp8(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
+                              self.x8, self.x_s, self.u8 if self.ws13 is not None else None,
+                              self.u_s if self.ws13 is not None else None, self.offsets,
                               self.pos, self.src, self.perm_ws, self.perm_ws_bytes)
             return
         L.moe_permute(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
@@ -212,9 +213,9 @@ class MoELayer:
             L.moe_expert_up_swiglu_gather(u, T, self.src, self.offsets, self.n_routed, rows, self.d,
                                           self.inter, self.w13, self.ffn_ws)
         elif self.fp8:
-            hb, h8, hs = self._fp8_h()
+            h8, hs = self._fp8_h()
             L.moe_expert_up_swiglu_fp8(self.x8, self.x_s, self.offsets, self.n_routed, rows,
-                                       self.d, self.inter, self.w13, self.w13_s, hb)
+                                       self.d, self.inter, self.w13, self.w13_s, h8, hs)
         else:
             L.moe_expert_up_swiglu(self.x_perm, self.offsets, self.n_routed, rows, self.d,
                                    self.inter, self.w13, self.ffn_ws)
@@ -222,8 +223,7 @@ class MoELayer:
     def _routed_down(self, T):
         rows = T * self.top_k
         if self.fp8:
-            hb, h8, hs = self._fp8_h()
-            L.moe_quant_act_fp8(hb, rows, self.inter, h8, hs)
+            h8, hs = self._fp8_h()
             L.moe_expert_down_fp8(h8, hs, self.offsets, self.n_routed, rows, self.inter, self.d,
                                   self.w2, self.w2_s, self.y_perm)
         elif self.fused_scatter:
@@ -236,13 +236,12 @@ class MoELayer:
                               self.w2, self.y_perm)
 
     def _fp8_h(self):
-        """Views of the FP8 FFN workspace: bf16 h, its E4M3 codes, their scales
-        (the layout moe_grouped_ffn uses)."""
+        """Views of the FP8 FFN workspace: h's E4M3 codes and their 1x128
+        scales (the layout moe_grouped_ffn uses)."""
         rows = self._T * self.top_k
-        hb = self.ffn_ws
-        h8 = self.ffn_ws[(rows * self.inter * 2 + 255) // 256 * 256:]
+        h8 = self.ffn_ws
         hs = h8[(rows * self.inter + 255) // 256 * 256:]
-        return hb, h8, hs
+        return h8, hs
 
     def shared_ffn(self, u):
         if self.ws13 is None:
@@ -462,13 +461,13 @@ class MoELayer:
     # + the activation quantisation), routed and shared FFN, combine (1),
     # bias update (1)
     def launches_per_step(self) -> int:
-        # bf16: up and down one launch each; FP8: up-projection, h
-        # quantisation, down-projection
-        ffn = 3 if self.fp8 else 2
+        # up and down one launch each (FP8: h is quantised in the
+        # up-projection's epilogue, u in the dispatch)
+        ffn = 2
         perm = 2 if self.fused_gather else 3
         if self.fused_scatter:
             perm += 1                       # the slot index
-        n = 1 + perm + ffn + 1 + (1 if self.fp8 else 0)
+        n = 1 + perm + ffn + 1
         if self.ws13 is not None:
             n += ffn
         if self.gate_kind == "sigmoid":

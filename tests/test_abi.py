@@ -155,20 +155,28 @@ def test_fp8_entry_points_reject_bad_arguments(lib):
     assert lib.moe_quant_weights_fp8(A, 2, 100, 256, A, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
     assert lib.moe_quant_weights_fp8(A, 0, 128, 256, A, A, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_quant_weights_fp8(A, 2, 128, 256, MIS, A, None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_permute_fp8(A, None, A, A, 64, 256, 16, 4, A, A, A, A, A, A, 4096,
+    # moe_permute_fp8(u, idx, counts, T, d, n, K, x8, xs, u8, us, off, pos, src, ws, wsb)
+    assert lib.moe_permute_fp8(A, A, A, 64, 256, 16, 4, A, None, None, None, A, A, A, A, 4096,
                                None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_permute_fp8(A, A, A, A, 64, 256, 16, 4, A, A, A, A, A, None, 4096,
+    assert lib.moe_permute_fp8(A, A, A, 64, 256, 16, 4, A, A, A, None, A, A, A, A, 4096,
+                               None) == L.MOE_ERR_INVALID_ARG          # u8 without u_scales
+    assert lib.moe_permute_fp8(MIS, A, A, 64, 256, 16, 4, A, A, None, None, A, A, A, A, 4096,
+                               None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute_fp8(A, A, A, 64, 256, 16, 4, A, A, None, None, A, A, A, None, 4096,
                                None) == L.MOE_ERR_WORKSPACE
-    assert lib.moe_expert_up_swiglu_fp8(A, None, A, 4, 256, 256, 128, A, A, A,
+    # moe_expert_up_swiglu_fp8(x8, xs, off, G, rows, d, inter, w13, w13s, h8, hs)
+    assert lib.moe_expert_up_swiglu_fp8(A, None, A, 4, 256, 256, 128, A, A, A, A,
                                         None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_expert_up_swiglu_fp8(A, A, A, 4, 256, 256, 128, A, A, MIS,
+    assert lib.moe_expert_up_swiglu_fp8(A, A, A, 4, 256, 256, 128, A, A, MIS, A,
+                                        None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_up_swiglu_fp8(A, A, A, 4, 256, 256, 128, A, A, A, None,
                                         None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_pack_w13_fp8(A, 2, 100, 256, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
     assert lib.moe_pack_w13_fp8(None, 2, 128, 256, A, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_down_fp8(A, A, A, 4, 256, 128, 256, A, A, MIS,
                                    None) == L.MOE_ERR_INVALID_ARG
     assert L.moe_grouped_ffn_workspace_size(1024, 2048, L.MOE_FP8_E4M3) == \
-        1024 * 2048 * 2 + 1024 * 2048 + 1024 * 16 * 4
+        1024 * 2048 + 1024 * 16 * 4
 
 
 def test_fused_gather_entry_points_reject_bad_arguments(lib):
@@ -284,3 +292,30 @@ def test_fused_scatter_entry_points_reject_bad_arguments(lib):
     assert lib.moe_combine_slots(MIS, A, None, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_combine_slots(A, None, None, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_combine_slots(A, A, MIS, None, 4, 256, 4, A, None) == L.MOE_ERR_INVALID_ARG
+
+
+def test_peer_memory_ep_entry_points_reject_bad_arguments(lib):
+    # moe_ep_plan_device(all_counts, world, n_local, rank, cap, dest, goff, gcounts)
+    assert lib.moe_ep_plan_device(A, 0, 8, 0, 10, A, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan_device(A, 2, 8, 2, 10, A, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan_device(A, 2, 8, 0, -1, A, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan_device(A, 4, 65, 0, 10, A, A, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_ep_plan_device(A, 2, 8, 0, 10, None, A, A, None) == L.MOE_ERR_INVALID_ARG
+    # moe_ep_dispatch_p2p(u, idx, pos, off, dest, T, d, n_routed, K, world, peer_x, cap)
+    assert lib.moe_ep_dispatch_p2p(A, A, A, A, A, 4, 256, 16, 4, 3, A, 10, None) == \
+        L.MOE_ERR_UNSUPPORTED_SHAPE                                  # 16 experts over 3 ranks
+    assert lib.moe_ep_dispatch_p2p(MIS, A, A, A, A, 4, 256, 16, 4, 2, A, 10, None) == \
+        L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_dispatch_p2p(A, A, A, A, A, 4, 256, 16, 4, 2, None, 10, None) == \
+        L.MOE_ERR_INVALID_ARG
+    # moe_ep_combine_p2p(peer_y, idx, pos, off, dest, gate, shared, res, T, d, n, K, W, cap, out)
+    assert lib.moe_ep_combine_p2p(A, A, A, A, A, A, None, None, 4, 256, 16, 9, 2, 10, A,
+                                  None) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_ep_combine_p2p(A, A, A, A, A, None, None, None, 4, 256, 16, 4, 2, 10, A,
+                                  None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_combine_p2p(A, A, A, A, A, A, None, None, 4, 256, 16, 4, 2, 10, MIS,
+                                  None) == L.MOE_ERR_INVALID_ARG
+    # IPC helpers: null arguments
+    assert lib.moe_ipc_get_handle(None, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ipc_open_handle(None, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ipc_close_handle(None) == L.MOE_ERR_INVALID_ARG

@@ -60,6 +60,93 @@ def test_weight_quant_bit_exact():
         assert np.array_equal(q[g].cpu().numpy(), want_q)
 
 
+def test_fp8_dispatch_quantises_each_token_once_bit_exact():
+    """moe_permute_fp8 on bf16 rows: every copied row's codes and scales equal
+    the oracle's 1x128 quantisation of its token, and u8 / u_scales hold the
+    token's own codes."""
+    cfg = synth.CONFIGS["tiny"].replace(T=383, d=512)
+    u = _rand_bf16((cfg.T, cfg.d), 11)
+    u[5, :128] = 0                                # an all-zero tile: scale 1
+    u[9] *= 1e-4
+    g = torch.Generator().manual_seed(3)
+    idx = torch.argsort(torch.rand(cfg.T, cfg.n_routed, generator=g), 1)[:, :cfg.top_k]
+    idx = idx.to(torch.int32).cuda()
+    counts = torch.bincount(idx.flatten().long(), minlength=cfg.n_routed).to(torch.int32)
+    T, d, K, n = cfg.T, cfg.d, cfg.top_k, cfg.n_routed
+    x8 = torch.empty((T * K, d), dtype=torch.uint8, device="cuda")
+    xs = torch.empty((T * K, d // 128), dtype=torch.float32, device="cuda")
+    u8 = torch.empty((T, d), dtype=torch.uint8, device="cuda")
+    us = torch.empty((T, d // 128), dtype=torch.float32, device="cuda")
+    off = torch.empty(n + 1, dtype=torch.int32, device="cuda")
+    pos = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    src = torch.empty(T * K, dtype=torch.int32, device="cuda")
+    wsb = L.moe_permute_workspace_size(T, n)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    L.moe_permute_fp8(u, idx, counts.cuda(), T, d, n, K, x8, xs, u8, us, off, pos, src, ws, wsb)
+    torch.cuda.synchronize()
+    want_q, want_s = of.quant_act_1x128(u.float().cpu().numpy())
+    assert np.array_equal(u8.cpu().numpy(), want_q)
+    assert np.array_equal(us.cpu().numpy(), want_s)
+    srct = src.cpu().numpy().astype(np.int64)
+    assert np.array_equal(x8.cpu().numpy(), want_q[srct])
+    assert np.array_equal(xs.cpu().numpy(), want_s[srct])
+    disp = om.dispatch(idx.cpu().numpy(), n)
+    assert np.array_equal(pos.cpu().numpy(), disp.pos)
+
+
+def test_fp8_up_projection_quantises_h_in_place():
+    """moe_expert_up_swiglu_fp8 writes h as E4M3 codes + 1x128 scales decided
+    from its fp32 value. Against the oracle's quantisation of the exact h of
+    the same FP8 operands: scales within fp32 accumulation error, and a code
+    may differ only where h sits at a rounding boundary (by one step)."""
+    sizes = [1, 0, 17, 128, 129, 300]
+    G, d, inter = len(sizes), 512, 256
+    rows = sum(sizes)
+    x = _rand_bf16((rows, d), 13)
+    w1 = _rand_bf16((G, inter, d), 14, 0.05)
+    w3 = _rand_bf16((G, inter, d), 15, 0.05)
+    x8 = torch.empty((rows, d), dtype=torch.uint8, device="cuda")
+    xs = torch.empty((rows, d // 128), dtype=torch.float32, device="cuda")
+    L.moe_quant_act_fp8(x, rows, d, x8, xs)
+    stacked = torch.stack([w1, w3], dim=1).contiguous()
+    sq = torch.empty((G, 2, inter, d), dtype=torch.uint8, device="cuda")
+    w13s = torch.empty((G, 2, inter // 128, d // 128), dtype=torch.float32, device="cuda")
+    L.moe_quant_weights_fp8(stacked, 2 * G, inter, d, sq, w13s)
+    w13q = torch.empty((G, 2 * inter, d), dtype=torch.uint8, device="cuda")
+    L.moe_pack_w13_fp8(sq, G, inter, d, w13q)
+    off = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32, device="cuda")
+    h8 = torch.full((rows + 8, inter), 0x55, dtype=torch.uint8, device="cuda")
+    hs = torch.full((rows + 8, inter // 128), -1.0, dtype=torch.float32, device="cuda")
+    L.moe_expert_up_swiglu_fp8(x8, xs, off, G, rows, d, inter, w13q, w13s, h8, hs)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    assert bool((h8[rows:] == 0x55).all()) and bool((hs[rows:] == -1.0).all())
+    xq, xsc = x8.cpu().numpy(), xs.cpu().numpy()
+    o = off.cpu().tolist()
+    got_q, got_s = h8[:rows].cpu().numpy(), hs[:rows].cpu().numpy()
+    n_codes = n_diff = 0
+    for i in range(G):
+        a, b = o[i], o[i + 1]
+        if a == b:
+            continue
+        w1q, w1sc = of.quant_weight_128x128(w1[i].float().cpu().numpy())
+        w3q, w3sc = of.quant_weight_128x128(w3[i].float().cpu().numpy())
+        ga = of.fp8_gemm(xq[a:b], xsc[a:b], w1q, w1sc)
+        gb = of.fp8_gemm(xq[a:b], xsc[a:b], w3q, w3sc)
+        h = ga / (1.0 + np.exp(-ga)) * gb
+        want_q, want_s = of.quant_act_1x128(h)
+        np.testing.assert_allclose(got_s[a:b], want_s, rtol=1e-5)
+        dq = got_q[a:b] != want_q
+        n_codes += dq.size
+        n_diff += int(dq.sum())
+        if dq.any():
+            # a differing code is the neighbouring E4M3 value
+            gv = of.e4m3_decode(got_q[a:b][dq])
+            wv = of.e4m3_decode(want_q[dq])
+            assert np.all(np.abs(gv - wv) <= 0.126 * np.maximum(np.abs(wv), 2.0 ** -6))
+    assert n_diff <= 1e-3 * n_codes, (n_diff, n_codes)
+
+
 def test_fp8_grouped_ffn_vs_oracle_emulation():
     """Group sizes over every tile path, E4M3 operands from the library's own
     quantisers (bit-exact to the oracle's, checked above); the oracle runs the
