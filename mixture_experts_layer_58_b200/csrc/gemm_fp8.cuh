@@ -27,11 +27,10 @@
 //               [64 + 32*half, +32) of the same 32 h columns (B is W1/W3
 //               interleaved in 64-row chunks), for the down-projection the
 //               columns [64*half, +64). 64 fp32 accumulators per thread.
-// Epilogues: EPI8_SWIGLU — h = silu(a) * b written as bf16; EPI8_SWIGLU_Q —
-// h quantised in the epilogue, straight from its fp32 value, to E4M3 codes
-// with one fp32 scale per 1x128 tile of h (the activation rule: scale =
-// max|h| / 448, codes decided in fp32), so h never goes to memory in a wider
-// type; EPI8_STORE — bf16 output.
+// Epilogues: EPI8_SWIGLU_Q — h = silu(a) * b quantised in the epilogue,
+// straight from its fp32 value, to E4M3 codes with one fp32 scale per 1x128
+// tile of h (the activation rule: scale = max|h| / 448, codes decided in
+// fp32), so h never goes to memory in a wider type; EPI8_STORE — bf16 output.
 // A 1x128 tile of h spans two 128-column tiles of the up-projection (64 h
 // columns each), so EPI8_SWIGLU_Q gives each CTA tile two column sub-tiles
 // of the same token rows, one after the other: a thread keeps its 32 h values
@@ -51,7 +50,7 @@ constexpr int kF8Stages = 6;
 constexpr int kF8Threads = 320;
 constexpr int kF8EpiThreads = 256;
 
-enum { EPI8_STORE = 0, EPI8_SWIGLU = 1, EPI8_SWIGLU_Q = 2 };
+enum { EPI8_STORE = 0, EPI8_SWIGLU_Q = 2 };
 
 // column sub-tiles per CTA tile
 template <int EPI>
@@ -245,7 +244,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     // the thread's two runs of 32 columns
-    constexpr bool kSwiglu = EPI == EPI8_SWIGLU || EPI == EPI8_SWIGLU_Q;
+    constexpr bool kSwiglu = EPI == EPI8_SWIGLU_Q;
     const int col0 = kSwiglu ? 32 * half : 64 * half;
     const int col1 = kSwiglu ? 64 + 32 * half : 64 * half + 32;
     const int ksb = num_kb;                   // scale blocks along K
@@ -379,17 +378,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         } else if (valid) {
           __nv_bfloat16* yrow = out + static_cast<size_t>(grow) * ldo;
-          if constexpr (EPI == EPI8_SWIGLU) {
-            uint4* dst = reinterpret_cast<uint4*>(yrow + nb_col * 64 + 32 * half);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              float h[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) h[i] = silu_f32(acc0[8 * v + i]) * acc1[8 * v + i];
-              dst[v] = make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]),
-                                  pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
-            }
-          } else {
+          {
             uint4* d0 = reinterpret_cast<uint4*>(yrow + nb_col * kF8BN + col0);
             uint4* d1 = reinterpret_cast<uint4*>(yrow + nb_col * kF8BN + col1);
 #pragma unroll
