@@ -601,6 +601,9 @@ def main():
                          "all-to-all; ep-p2p: the same split, rows stored into and read back "
                          "from the owners' buffers by the library's kernels over peer memory, "
                          "planned on the device (bf16 forward, five-call mode)")
+    ap.add_argument("--micro-batches", type=int, default=1, choices=[1, 2],
+                    help="ep-p2p: split each step's tokens in two, the exchange of one "
+                         "beside the expert GEMMs of the other")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the decode and FP8 workloads timed after V3 prefill")
@@ -664,10 +667,17 @@ def main():
     if ep_mode:
         from mixture_experts_layer_58_b200.ep import (ExpertParallelMoELayer,
                                                       PeerExpertParallelMoELayer)
-        cls = PeerExpertParallelMoELayer if args.parallel == "ep-p2p" else ExpertParallelMoELayer
-        lay = cls(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
-                  routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
-                  overlap_shared=not args.no_overlap, device=dev)
+        if args.parallel == "ep-p2p":
+            lay = PeerExpertParallelMoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
+                                             routed_scale=cfg.routed_scale,
+                                             gate_kind=cfg.gate_kind, gamma=cfg.gamma,
+                                             micro_batches=args.micro_batches,
+                                             overlap_shared=not args.no_overlap, device=dev)
+        else:
+            lay = ExpertParallelMoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
+                                         routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
+                                         gamma=cfg.gamma, overlap_shared=not args.no_overlap,
+                                         device=dev)
     else:
         lay = MoELayer(e_host, b_host, W1, W3, W2, shared, top_k=cfg.top_k,
                        routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
@@ -781,7 +791,10 @@ def main():
                    "gate": cfg.gate_kind, "global_batch_tokens": T * world,
                    "mode": ("expert-parallel over peer memory: rows stored into and read "
                             "back from the owners' buffers by the library's kernels, plan on "
-                            "the device" if args.parallel == "ep-p2p" else
+                            "the device" + (", two micro-batches, the exchange of one beside "
+                                            "the expert GEMMs of the other"
+                                            if args.micro_batches == 2 else "")
+                            if args.parallel == "ep-p2p" else
                             "expert-parallel: NCCL all-to-all dispatch/return, rows "
                             "regrouped by expert on the receiving rank" if ep_mode else
                             "fused gather" if lay.fused_gather else

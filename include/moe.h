@@ -504,7 +504,9 @@ MOE_API int moe_gather_rows(const void* src, int n_src, const int32_t* index, in
  *   (row q = rank q's moe_route counts); writes dest_row [n_routed] (first row
  *   of this rank's rows for expert E in its owner's receive buffer),
  *   group_offsets [n_local + 1] (this rank's own receive buffer, expert-major)
- *   and global_counts [n_routed] (the loads summed over the ranks). A receive
+ *   and global_counts [n_routed] (the loads summed over the ranks, plus
+ *   add_counts [n_routed] when it is not NULL: an earlier micro-batch's
+ *   global_counts, so that the last one holds the step's). A receive
  *   buffer that would need more than recv_capacity rows sets bit 16 of the
  *   device status word (moe_get_device_status then returns
  *   MOE_ERR_DEVICE_TIMEOUT); the rows past the capacity are not moved.
@@ -524,9 +526,9 @@ MOE_API int moe_gather_rows(const void* src, int n_src, const int32_t* index, in
  *   start; add the offset); moe_ipc_close_handle unmaps it.
  */
 MOE_API int moe_ep_plan_device(const int32_t* all_counts, int world, int n_local, int rank,
-                               long long recv_capacity, int32_t* dest_row,
-                               int32_t* group_offsets, int32_t* global_counts,
-                               moe_stream_t stream);
+                               long long recv_capacity, const int32_t* add_counts,
+                               int32_t* dest_row, int32_t* group_offsets,
+                               int32_t* global_counts, moe_stream_t stream);
 MOE_API int moe_ep_dispatch_p2p(const void* u, const int32_t* topk_idx, const int32_t* pos,
                                 const int32_t* expert_offsets, const int32_t* dest_row, int T,
                                 int d, int n_routed, int top_k, int world, void* const* peer_x,

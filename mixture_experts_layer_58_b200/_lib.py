@@ -86,7 +86,7 @@ _SIGS = {
     "moe_ep_plan": (_i, [_vp, _vp, _i, _i, _ll, _vp, _vp, _vp, _vp, _vp,
                          ctypes.POINTER(ctypes.c_longlong)]),
     "moe_gather_rows": (_i, [_vp, _i, _vp, _i, _i, _vp, _vp]),
-    "moe_ep_plan_device": (_i, [_vp, _i, _i, _i, _ll, _vp, _vp, _vp, _vp]),
+    "moe_ep_plan_device": (_i, [_vp, _i, _i, _i, _ll, _vp, _vp, _vp, _vp, _vp]),
     "moe_ep_dispatch_p2p": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _ll, _vp]),
     "moe_ep_combine_p2p": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                 _ll, _vp, _vp]),
@@ -307,10 +307,10 @@ def moe_gather_rows(src, n_src, index, n, d, dst, stream=None):
 
 
 def moe_ep_plan_device(all_counts, world, n_local, rank, recv_capacity, dest_row,
-                       group_offsets, global_counts, stream=None):
+                       group_offsets, global_counts, add_counts=None, stream=None):
     _check(_L().moe_ep_plan_device(_p(all_counts), world, n_local, rank, int(recv_capacity),
-                                   _p(dest_row), _p(group_offsets), _p(global_counts),
-                                   _stream(stream)), "moe_ep_plan_device")
+                                   _p(add_counts), _p(dest_row), _p(group_offsets),
+                                   _p(global_counts), _stream(stream)), "moe_ep_plan_device")
 
 
 def moe_ep_dispatch_p2p(u, topk_idx, pos, expert_offsets, dest_row, T, d, n_routed, top_k,

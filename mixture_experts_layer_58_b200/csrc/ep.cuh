@@ -131,11 +131,13 @@ namespace moe {
 // buffer needing more than `capacity` rows sets kStatusEpOverflow (the
 // dispatch then drops the rows past the capacity: never a silent result,
 // the status word reports it).
+// add_counts (may be NULL) is added to global_counts: the loads of an
+// earlier micro-batch of the same step, so the bias update sees the step's.
 __global__ void __launch_bounds__(256)
 ep_plan_device_kernel(const int32_t* __restrict__ all_counts, int world, int n_local, int rank,
-                      long long capacity, int32_t* __restrict__ dest_row,
-                      int32_t* __restrict__ group_offsets, int32_t* __restrict__ global_counts,
-                      unsigned int* status) {
+                      long long capacity, const int32_t* __restrict__ add_counts,
+                      int32_t* __restrict__ dest_row, int32_t* __restrict__ group_offsets,
+                      int32_t* __restrict__ global_counts, unsigned int* status) {
   __shared__ long long s_scan[256];
   const int n_routed = world * n_local;
   const int E = threadIdx.x;
@@ -160,7 +162,7 @@ ep_plan_device_kernel(const int32_t* __restrict__ all_counts, int world, int n_l
     const long long base = owner0 > 0 ? s_scan[owner0 - 1] : 0;
     const long long recv_off = s_scan[E] - tot - base;     // exclusive, within the owner
     dest_row[E] = static_cast<int32_t>(recv_off + before);
-    global_counts[E] = static_cast<int32_t>(tot);
+    global_counts[E] = static_cast<int32_t>(tot + (add_counts ? add_counts[E] : 0));
     if (E / n_local == rank) {
       const int e = E - owner0;
       group_offsets[e] = static_cast<int32_t>(recv_off);

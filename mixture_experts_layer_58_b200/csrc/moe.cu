@@ -842,8 +842,8 @@ int moe_ep_plan(const int32_t* local_counts, const int32_t* recv_counts, int wor
 
 // ------------------------------------------------------------------ expert parallelism over peer memory
 int moe_ep_plan_device(const int32_t* all_counts, int world, int n_local, int rank,
-                       long long recv_capacity, int32_t* dest_row, int32_t* group_offsets,
-                       int32_t* global_counts, moe_stream_t stream) {
+                       long long recv_capacity, const int32_t* add_counts, int32_t* dest_row,
+                       int32_t* group_offsets, int32_t* global_counts, moe_stream_t stream) {
   if (world < 1 || n_local < 1 || rank < 0 || rank >= world || recv_capacity < 0)
     return MOE_ERR_INVALID_ARG;
   if (static_cast<long long>(world) * n_local > kRouteMaxExperts)
@@ -853,8 +853,9 @@ int moe_ep_plan_device(const int32_t* all_counts, int world, int n_local, int ra
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
   ep_plan_device_kernel<<<1, 256, 0, as_stream(stream)>>>(all_counts, world, n_local, rank,
-                                                          recv_capacity, dest_row, group_offsets,
-                                                          global_counts, di->status);
+                                                          recv_capacity, add_counts, dest_row,
+                                                          group_offsets, global_counts,
+                                                          di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

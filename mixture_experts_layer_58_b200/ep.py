@@ -314,7 +314,11 @@ class PeerExpertParallelMoELayer(MoELayer):
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
                  group=None, world: int | None = None, rank: int | None = None,
-                 recv_capacity: int | None = None, overlap_shared: bool = True, device="cuda"):
+                 recv_capacity: int | None = None, micro_batches: int = 1,
+                 overlap_shared: bool = True, device="cuda"):
+        if micro_batches not in (1, 2):
+            raise ValueError("micro_batches must be 1 or 2")
+        self.micro_batches = int(micro_batches)
         self.group = group
         self.emulated = world is not None and group is None
         self.world = dist.get_world_size(group) if world is None else int(world)
@@ -335,6 +339,8 @@ class PeerExpertParallelMoELayer(MoELayer):
         self.recv_capacity_arg = recv_capacity
         self._mapped = []          # IPC bases opened on this GPU
         self._recv_T = -1
+        self._mb = None            # the two micro-batch halves (micro_batches == 2)
+        self._comm = None
 
     # ------------------------------------------------------------------ buffers
     def allocate(self, T: int) -> None:
@@ -413,10 +419,12 @@ class PeerExpertParallelMoELayer(MoELayer):
         with ev("permute"):
             self.permute(u)
 
-    def plan(self):
-        """Device plan from self.all_counts (every rank's loads)."""
+    def plan(self, add_counts=None):
+        """Device plan from self.all_counts (every rank's loads); add_counts:
+        an earlier micro-batch's summed loads, folded into global_counts."""
         L.moe_ep_plan_device(self.all_counts, self.world, self.n_local, self.rank,
-                             self.recv_capacity, self.dest_row, self.goff, self.global_counts)
+                             self.recv_capacity, self.dest_row, self.goff, self.global_counts,
+                             add_counts)
 
     def dispatch(self, u, timers=None):
         with _Timed(timers)("dispatch"):
@@ -465,6 +473,8 @@ class PeerExpertParallelMoELayer(MoELayer):
             raise ValueError("the expert-parallel layer runs the forward only")
         if self.emulated:
             raise RuntimeError("an emulated rank is driven through its stages")
+        if self.micro_batches == 2 and u.shape[0] >= 2:
+            return self._forward_two(u, residual, out, timers)
         self.begin(u, timers)
         with _Timed(timers)("exchange_counts"):
             dist.all_gather_into_tensor(self.all_counts.view(-1), self.counts, group=self.group)
@@ -473,14 +483,90 @@ class PeerExpertParallelMoELayer(MoELayer):
         self._barrier()
         self.experts(timers)
         self._barrier()
+        self._step_counts = self.global_counts
+        self._step_T = u.shape[0]
         return self.finish(u, residual, out, timers)
+
+    def micro_batch_halves(self):
+        """The two halves of a two-micro-batch step: this layer and a second
+        one sharing its weights, bias and process group, with buffers of its
+        own (each half holds the first or second half of the tokens)."""
+        if self._mb is None:
+            import copy
+            other = copy.copy(self)
+            other._mb = None
+            other._side = None           # its own side stream and events
+            other._T = other._recv_T = -1
+            other._mapped = []
+            other.micro_batches = 1
+            self._mb = (self, other)
+        return self._mb
+
+    def _forward_two(self, u, residual, out, timers):
+        """Two micro-batches, the exchange of one beside the expert GEMMs of
+        the other (the overlap the technical report arranges with DualPipe):
+
+            main:  begin A, begin B | all-gather, plan, dispatch A, barrier
+            comm:                     all-gather, plan, dispatch B, barrier
+            main:  experts A   (beside B's dispatch)
+            comm:  barrier, combine A   (beside B's experts)
+            main:  experts B, barrier, combine B; then waits for comm
+
+        The collectives are issued in the same order on every rank."""
+        T = u.shape[0]
+        T1 = T // 2
+        A, B = self.micro_batch_halves()
+        if out is None:
+            if getattr(self, "_out_full", None) is None or self._out_full.shape[0] != T:
+                self._out_full = torch.empty((T, self.d), dtype=torch.bfloat16,
+                                             device=self.device)
+            out = self._out_full
+        assert out.shape == (T, self.d) and out.dtype == torch.bfloat16 and out.is_contiguous()
+        dst = out
+        uA, uB = u[:T1], u[T1:]
+        oA, oB = dst[:T1], dst[T1:]
+        cur = torch.cuda.current_stream()
+        if self._comm is None:
+            self._comm = torch.cuda.Stream(device=self.device)
+        comm = self._comm
+        A.begin(uA, timers)
+        B.begin(uB)
+        dist.all_gather_into_tensor(A.all_counts.view(-1), A.counts, group=self.group)
+        A.plan()
+        A.dispatch(uA, timers)
+        A._barrier()
+        comm.wait_stream(cur)
+        with torch.cuda.stream(comm):
+            dist.all_gather_into_tensor(B.all_counts.view(-1), B.counts, group=self.group)
+            B.plan(add_counts=A.global_counts)
+            B.dispatch(uB)
+            B._barrier()
+            b_ready = torch.cuda.Event()
+            b_ready.record(comm)
+        A.experts(timers)
+        a_done = torch.cuda.Event()
+        a_done.record(cur)
+        with torch.cuda.stream(comm):
+            comm.wait_event(a_done)
+            A._barrier()
+            A.finish(uA, residual, oA)
+        cur.wait_event(b_ready)
+        B.experts()
+        B._barrier()
+        B.finish(uB, residual, oB)
+        cur.wait_stream(comm)
+        uA.record_stream(comm)
+        self._step_counts = B.global_counts
+        self._step_T = T
+        return dst
 
     def update_bias(self, counts=None, T=None):
         """End-of-step bias update from the loads summed over the ranks (the
-        device plan's global_counts) and the tokens of all ranks."""
-        T_all = self.world * self._T if T is None else T
-        L.moe_bias_update(self.global_counts if counts is None else counts, self.bias,
-                          self.n_routed, T_all, self.top_k, self.gamma)
+        device plan's global_counts; with two micro-batches the second one's,
+        which includes the first's) and the tokens of all ranks."""
+        T_all = self.world * getattr(self, "_step_T", self._T) if T is None else T
+        c = getattr(self, "_step_counts", self.global_counts) if counts is None else counts
+        L.moe_bias_update(c, self.bias, self.n_routed, T_all, self.top_k, self.gamma)
 
     def step(self, u):
         out = self.forward(u)
@@ -494,6 +580,7 @@ class PeerExpertParallelMoELayer(MoELayer):
         n = 1 + 2 + 1 + 1 + 2 + 1
         if self.ws13 is not None:
             n += 2
+        n *= self.micro_batches
         if self.gate_kind == "sigmoid":
             n += 1
         return n
@@ -501,6 +588,8 @@ class PeerExpertParallelMoELayer(MoELayer):
     def close(self):
         """Unmap the other ranks' buffers (collective: every rank calls it)."""
         self._unmap_peers()
+        if self._mb is not None:
+            self._mb[1]._unmap_peers()
 
 
 def link_emulated_ranks(layers) -> None:

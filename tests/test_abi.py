@@ -296,11 +296,12 @@ def test_fused_scatter_entry_points_reject_bad_arguments(lib):
 
 def test_peer_memory_ep_entry_points_reject_bad_arguments(lib):
     # moe_ep_plan_device(all_counts, world, n_local, rank, cap, dest, goff, gcounts)
-    assert lib.moe_ep_plan_device(A, 0, 8, 0, 10, A, A, A, None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_ep_plan_device(A, 2, 8, 2, 10, A, A, A, None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_ep_plan_device(A, 2, 8, 0, -1, A, A, A, None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_ep_plan_device(A, 4, 65, 0, 10, A, A, A, None) == L.MOE_ERR_UNSUPPORTED_SHAPE
-    assert lib.moe_ep_plan_device(A, 2, 8, 0, 10, None, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan_device(A, 0, 8, 0, 10, None, A, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan_device(A, 2, 8, 2, 10, None, A, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan_device(A, 2, 8, 0, -1, None, A, A, A, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan_device(A, 4, 65, 0, 10, None, A, A, A, None) == \
+        L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_ep_plan_device(A, 2, 8, 0, 10, None, None, A, A, None) == L.MOE_ERR_INVALID_ARG
     # moe_ep_dispatch_p2p(u, idx, pos, off, dest, T, d, n_routed, K, world, peer_x, cap)
     assert lib.moe_ep_dispatch_p2p(A, A, A, A, A, 4, 256, 16, 4, 3, A, 10, None) == \
         L.MOE_ERR_UNSUPPORTED_SHAPE                                  # 16 experts over 3 ranks

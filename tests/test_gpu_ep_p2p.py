@@ -152,8 +152,12 @@ def _free_port() -> int:
     return p
 
 
-@pytest.mark.parametrize("name", ["tiny", "mid"])
-def test_p2p_forward_through_nccl_one_rank(name):
+@pytest.mark.parametrize("name,mb", [("tiny", 1), ("mid", 1), ("tiny", 2), ("mid", 2)])
+def test_p2p_forward_through_nccl_one_rank(name, mb):
+    """forward() with its NCCL all-gather and barriers in a one-rank group
+    (mb = 2: two micro-batches, the second's exchange on its own stream beside
+    the first's GEMMs) equals the single-GPU layer; step()'s bias update
+    matches the oracle's on the loads of the whole step."""
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(_free_port())
     dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=120))
@@ -162,7 +166,8 @@ def test_p2p_forward_through_nccl_one_rank(name):
         e, b = synth.centroids(cfg), synth.bias(cfg)
         W1, W3, W2, shared = _weights(cfg)
         lay = PeerExpertParallelMoELayer(e, b, W1, W3, W2, shared, top_k=cfg.top_k,
-                                         routed_scale=cfg.routed_scale, gamma=cfg.gamma)
+                                         routed_scale=cfg.routed_scale, gamma=cfg.gamma,
+                                         micro_batches=mb)
         assert lay.world == 1 and lay.n_local == cfg.n_routed
         u = synth.tokens(cfg)
         out = lay.step(u.cuda()).float().cpu()
@@ -171,7 +176,8 @@ def test_p2p_forward_through_nccl_one_rank(name):
                           routed_scale=cfg.routed_scale, gamma=cfg.gamma)
         ref = single.forward(u.cuda()).float().cpu()
         check_close(out.numpy(), ref.numpy(), max_tol=4e-3, mean_tol=1e-3, what="vs single GPU")
-        want_b = om.bias_update(lay.counts.cpu().numpy(), b.numpy(), cfg.T, cfg.top_k, cfg.gamma)
+        counts = single.counts.cpu().numpy()
+        want_b = om.bias_update(counts, b.numpy(), cfg.T, cfg.top_k, cfg.gamma)
         assert np.array_equal(lay.bias.cpu().numpy(), want_b)
         assert L.moe_get_device_status() == 0
         lay.close()
