@@ -421,10 +421,15 @@ MOE_API int moe_combine_dx(const void* dout, const void* dx_perm, const int32_t*
                            moe_stream_t stream);
 
 /* moe_centroid_grad: de_i = sum over the rows r of expert i of dz_perm[r] *
- * x_perm[r] (x_perm row r = u of the token routed there), bf16 [n_routed, d]. */
+ * x_perm[r] (x_perm row r = u of the token routed there), bf16 [n_routed, d].
+ * The rows are summed in chunks of 128 (so that a hot expert spreads over
+ * many blocks), then the chunks in order: the result is reproducible.
+ * workspace >= moe_centroid_grad_workspace_size(rows, n_routed, d) bytes,
+ * 16-B aligned. n_routed < 1024. */
 MOE_API int moe_centroid_grad(const void* x_perm, const float* dz_perm,
                               const int32_t* expert_offsets, int n_routed, int rows, int d,
-                              void* de, moe_stream_t stream);
+                              void* de, void* workspace, size_t ws_bytes, moe_stream_t stream);
+MOE_API size_t moe_centroid_grad_workspace_size(int rows, int n_routed, int d);
 
 /* ------------------------------------------------------------------ expert parallelism
  * The routed experts split evenly over W ranks: rank p holds experts

@@ -82,7 +82,8 @@ _SIGS = {
     "moe_gate_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp,
                                _vp]),
     "moe_combine_dx": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
-    "moe_centroid_grad": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_centroid_grad": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "moe_centroid_grad_workspace_size": (_sz, [_i, _i, _i]),
     "moe_ep_plan": (_i, [_vp, _vp, _i, _i, _ll, _vp, _vp, _vp, _vp, _vp,
                          ctypes.POINTER(ctypes.c_longlong)]),
     "moe_gather_rows": (_i, [_vp, _i, _vp, _i, _i, _vp, _vp]),
@@ -403,9 +404,15 @@ def moe_combine_dx(dout, dx_perm, pos, dx_shared, dz, topk_idx, centroids, T, d,
            "moe_combine_dx")
 
 
-def moe_centroid_grad(x_perm, dz_perm, expert_offsets, n_routed, rows, d, de, stream=None):
+def moe_centroid_grad(x_perm, dz_perm, expert_offsets, n_routed, rows, d, de, workspace,
+                      ws_bytes, stream=None):
     _check(_L().moe_centroid_grad(_p(x_perm), _p(dz_perm), _p(expert_offsets), n_routed, rows, d,
-                                  _p(de), _stream(stream)), "moe_centroid_grad")
+                                  _p(de), _p(workspace), ws_bytes, _stream(stream)),
+           "moe_centroid_grad")
+
+
+def moe_centroid_grad_workspace_size(rows, n_routed, d) -> int:
+    return int(_L().moe_centroid_grad_workspace_size(rows, n_routed, d))
 
 
 def moe_strerror(status: int) -> str:

@@ -197,36 +197,89 @@ combine_dx_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
   }
 }
 
-// de_i = sum over the rows r of group i of dz_perm[r] x_perm[r]. Block
-// (group i, 256 columns): warp w sums rows w, w+8, ... of the group (each lane
-// 8 columns, four rows in flight), then the 8 partial sums are added in a
-// fixed order through shared memory (no atomics: the result is reproducible).
+// de_i = sum over the rows r of group i of dz_perm[r] x_perm[r], in two
+// passes so that a hot expert's rows are spread over many blocks and the sum
+// keeps a fixed order (no atomics: reproducible):
+//   table:  one block cuts every expert's rows into chunks of kCentroidChunk
+//           rows (expert-major) and writes each chunk's row range;
+//   pass 1: block (chunk, 256 columns) sums its <= 128 rows (warp w rows
+//           w, w+8, ...; each lane 8 columns, four rows in flight), the 8 warp
+//           partials added in order through shared memory, fp32 to workspace;
+//   pass 2: block (expert, 256 columns) adds its chunks' partials in chunk
+//           order and rounds once to bf16.
+// Offsets are clamped into [0, rows] and made non-decreasing first, so x_perm
+// is never read outside its rows.
 constexpr int kCentroidCols = 256;
 constexpr int kCentroidWarps = 8;
+constexpr int kCentroidChunk = 128;
+constexpr int kCentroidMaxExperts = 1024;
+
+// Workspace: chunk_start [n + 1] int32 (first chunk of each expert, then the
+// total), chunk_rows [max_chunks] int2 (row range), partials [max_chunks, d] fp32.
+__host__ __device__ inline long long centroid_max_chunks(long long rows, int n) {
+  return (rows + kCentroidChunk - 1) / kCentroidChunk + n;
+}
+
+__global__ void __launch_bounds__(1024)
+centroid_chunk_table_kernel(const int32_t* __restrict__ offsets, int n, int rows,
+                            int32_t* __restrict__ chunk_start, int2* __restrict__ chunk_rows) {
+  __shared__ int s_lo[kCentroidMaxExperts + 1];
+  __shared__ int s_scan[kCentroidMaxExperts];
+  const int e = threadIdx.x;
+  // clamped, non-decreasing offsets: running maximum of the clamped entries
+  if (e <= n) s_lo[e] = min(max(__ldg(offsets + e), 0), rows);
+  __syncthreads();
+  for (int o = 1; o <= n; o <<= 1) {
+    const int v = (e <= n && e >= o) ? s_lo[e - o] : 0;
+    __syncthreads();
+    if (e <= n && e >= o) s_lo[e] = max(s_lo[e], v);
+    __syncthreads();
+  }
+  const int r0 = e < n ? s_lo[e] : 0;
+  const int r1 = e < n ? s_lo[e + 1] : 0;
+  const int nch = (r1 - r0 + kCentroidChunk - 1) / kCentroidChunk;
+  if (e < kCentroidMaxExperts) s_scan[e] = nch;
+  __syncthreads();
+  for (int o = 1; o < kCentroidMaxExperts; o <<= 1) {
+    const int v = (e < kCentroidMaxExperts && e >= o) ? s_scan[e - o] : 0;
+    __syncthreads();
+    if (e < kCentroidMaxExperts) s_scan[e] += v;
+    __syncthreads();
+  }
+  if (e < n) {
+    const int first = s_scan[e] - nch;
+    chunk_start[e] = first;
+    for (int j = 0; j < nch; ++j) {
+      const int a = r0 + j * kCentroidChunk;
+      chunk_rows[first + j] = make_int2(a, min(a + kCentroidChunk, r1));
+    }
+    if (e == n - 1) chunk_start[n] = s_scan[e];
+  }
+}
+
 __global__ void __launch_bounds__(32 * kCentroidWarps)
-centroid_grad_kernel(const __nv_bfloat16* __restrict__ x_perm, const float* __restrict__ dz_perm,
-                     const int32_t* __restrict__ offsets, int rows, int d,
-                     __nv_bfloat16* __restrict__ de) {
+centroid_partial_kernel(const __nv_bfloat16* __restrict__ x_perm,
+                        const float* __restrict__ dz_perm, const int32_t* __restrict__ chunk_start,
+                        const int2* __restrict__ chunk_rows, int n, int d,
+                        float* __restrict__ partials) {
   __shared__ float part[kCentroidWarps][kCentroidCols + 4];
-  const int i = blockIdx.x;
+  const int c = blockIdx.x;
+  if (c >= __ldg(chunk_start + n)) return;          // past the last chunk
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int col = blockIdx.y * kCentroidCols + lane * 8;
-  // the caller's offsets are clamped into [0, rows] (an empty range if they
-  // decrease), so x_perm is never read outside its rows
-  const int r0 = min(max(__ldg(offsets + i), 0), rows);
-  const int r1 = min(max(__ldg(offsets + i + 1), r0), rows);
+  const int2 rr = chunk_rows[c];
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (col < d) {
-    int r = r0 + warp;
-    for (; r + 3 * kCentroidWarps < r1; r += 4 * kCentroidWarps) {
+    int r = rr.x + warp;
+    for (; r + 3 * kCentroidWarps < rr.y; r += 4 * kCentroidWarps) {
       uint4 q[4];
       float w[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int rr = r + j * kCentroidWarps;
-        q[j] = __ldg(reinterpret_cast<const uint4*>(x_perm + static_cast<size_t>(rr) * d + col));
-        w[j] = __ldg(dz_perm + rr);
+        const int rj = r + j * kCentroidWarps;
+        q[j] = __ldg(reinterpret_cast<const uint4*>(x_perm + static_cast<size_t>(rj) * d + col));
+        w[j] = __ldg(dz_perm + rj);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -236,7 +289,7 @@ centroid_grad_kernel(const __nv_bfloat16* __restrict__ x_perm, const float* __re
         for (int k = 0; k < 8; ++k) acc[k] = fmaf(w[j], x[k], acc[k]);
       }
     }
-    for (; r < r1; r += kCentroidWarps) {
+    for (; r < rr.y; r += kCentroidWarps) {
       float x[8];
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x_perm + static_cast<size_t>(r) * d + col)), x);
       const float w = __ldg(dz_perm + r);
@@ -247,14 +300,25 @@ centroid_grad_kernel(const __nv_bfloat16* __restrict__ x_perm, const float* __re
 #pragma unroll
   for (int k = 0; k < 8; ++k) part[warp][lane * 8 + k] = acc[k];
   __syncthreads();
-  // thread t finishes column t of the block: sum of the 8 warps in order
-  const int c = blockIdx.y * kCentroidCols + threadIdx.x;
-  if (threadIdx.x < kCentroidCols && c < d) {
+  const int cc = blockIdx.y * kCentroidCols + threadIdx.x;
+  if (threadIdx.x < kCentroidCols && cc < d) {
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < kCentroidWarps; ++w) s += part[w][threadIdx.x];
-    de[static_cast<size_t>(i) * d + c] = __float2bfloat16_rn(s);
+    partials[static_cast<size_t>(c) * d + cc] = s;
   }
+}
+
+__global__ void __launch_bounds__(kCentroidCols)
+centroid_reduce_kernel(const int32_t* __restrict__ chunk_start, const float* __restrict__ partials,
+                       int d, __nv_bfloat16* __restrict__ de) {
+  const int e = blockIdx.x;
+  const int col = blockIdx.y * kCentroidCols + threadIdx.x;
+  if (col >= d) return;
+  const int c0 = __ldg(chunk_start + e), c1 = __ldg(chunk_start + e + 1);
+  float s = 0.f;
+  for (int c = c0; c < c1; ++c) s += __ldg(partials + static_cast<size_t>(c) * d + col);
+  de[static_cast<size_t>(e) * d + col] = __float2bfloat16_rn(s);
 }
 
 }  // namespace moe

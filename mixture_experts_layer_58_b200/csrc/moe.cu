@@ -1138,16 +1138,44 @@ int moe_combine_dx(const void* dout, const void* dx_perm, const int32_t* pos,
   return MOE_OK;
 }
 
+size_t moe_centroid_grad_workspace_size(int rows, int n_routed, int d) {
+  if (rows < 0 || n_routed <= 0 || d <= 0) return 256;
+  const long long chunks = centroid_max_chunks(rows, n_routed);
+  const size_t a = (static_cast<size_t>(n_routed + 1) * 4 + 15) / 16 * 16;
+  const size_t b = (static_cast<size_t>(chunks) * 8 + 15) / 16 * 16;
+  return a + b + static_cast<size_t>(chunks) * d * 4;
+}
+
 int moe_centroid_grad(const void* x_perm, const float* dz_perm, const int32_t* expert_offsets,
-                      int n_routed, int rows, int d, void* de, moe_stream_t stream) {
+                      int n_routed, int rows, int d, void* de, void* workspace, size_t ws_bytes,
+                      moe_stream_t stream) {
   if (n_routed <= 0 || rows < 0 || d <= 0) return MOE_ERR_INVALID_ARG;
-  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d % 8 != 0 || n_routed >= kCentroidMaxExperts || (d + kCentroidCols - 1) / kCentroidCols > 65535)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!expert_offsets || !de || !aligned16(de)) return MOE_ERR_INVALID_ARG;
   if (rows > 0 && (!x_perm || !dz_perm || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
-  dim3 grid(n_routed, (d + kCentroidCols - 1) / kCentroidCols);
-  centroid_grad_kernel<<<grid, 32 * kCentroidWarps, 0, as_stream(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x_perm), dz_perm, expert_offsets, rows, d,
-      static_cast<__nv_bfloat16*>(de));
+  if (!workspace || ws_bytes < moe_centroid_grad_workspace_size(rows, n_routed, d) ||
+      !aligned16(workspace))
+    return MOE_ERR_WORKSPACE;
+  const long long chunks = centroid_max_chunks(rows, n_routed);
+  if (chunks > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* chunk_start = reinterpret_cast<int32_t*>(ws);
+  int2* chunk_rows =
+      reinterpret_cast<int2*>(ws + (static_cast<size_t>(n_routed + 1) * 4 + 15) / 16 * 16);
+  float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(chunk_rows) +
+                                             (static_cast<size_t>(chunks) * 8 + 15) / 16 * 16);
+  cudaStream_t st = as_stream(stream);
+  const int ncb = (d + kCentroidCols - 1) / kCentroidCols;
+  centroid_chunk_table_kernel<<<1, kCentroidMaxExperts, 0, st>>>(expert_offsets, n_routed, rows,
+                                                                  chunk_start, chunk_rows);
+  MOE_CUDA(cudaGetLastError());
+  centroid_partial_kernel<<<dim3(static_cast<unsigned>(chunks), ncb), 32 * kCentroidWarps, 0,
+                            st>>>(static_cast<const __nv_bfloat16*>(x_perm), dz_perm, chunk_start,
+                                  chunk_rows, n_routed, d, partials);
+  MOE_CUDA(cudaGetLastError());
+  centroid_reduce_kernel<<<dim3(n_routed, ncb), kCentroidCols, 0, st>>>(
+      chunk_start, partials, d, static_cast<__nv_bfloat16*>(de));
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

@@ -360,6 +360,8 @@ class MoELayer:
         self.dz = torch.empty((T, K), dtype=f32, device=dev)
         self.dz_perm = torch.empty(rows, dtype=f32, device=dev)
         self.du = torch.empty((T, d), dtype=bf, device=dev)
+        self.cg_ws = torch.empty(L.moe_centroid_grad_workspace_size(rows, self.n_routed, d),
+                                 dtype=torch.uint8, device=dev)
         if self.ws13 is not None:
             Is = self.shared_inter
             self.h_s = torch.empty((T, Is), dtype=bf, device=dev)
@@ -436,13 +438,13 @@ class MoELayer:
         L.moe_combine_dx(dout if residual else None, self.dx_perm, self.pos, dx_s, self.dz,
                          self.topk_idx, self.centroids, T, d, K, self.du)
         L.moe_centroid_grad(self.x_perm, self.dz_perm, self.offsets, G, rows, d,
-                            self.grad_centroids)
+                            self.grad_centroids, self.cg_ws, self.cg_ws.numel())
         return self.du
 
     def launches_per_backward(self) -> int:
         # combine bwd, down dgrad, up dgrad, 2 wgrad; shared: 4 more; gate bwd,
-        # du, centroid grad
-        return 5 + (4 if self.ws13 is not None else 0) + 3
+        # du, centroid grad (chunk table, partial sums, reduction)
+        return 5 + (4 if self.ws13 is not None else 0) + 5
 
     def update_bias(self, counts=None, T=None):
         """End-of-step bias update from this batch's loads (or from counts

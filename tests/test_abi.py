@@ -243,8 +243,14 @@ def test_backward_entry_points_reject_bad_arguments(lib):
     assert lib.moe_combine_dx(A, A, A, A, A, A, A, 64, 256, 9, A, None) == U
     assert lib.moe_combine_dx(MIS, A, A, A, A, A, A, 64, 256, 4, A, None) == E
     assert lib.moe_combine_dx(A, A, A, A, None, A, A, 64, 256, 4, A, None) == E
-    assert lib.moe_centroid_grad(A, A, A, 16, 256, 250, A, None) == U
-    assert lib.moe_centroid_grad(A, None, A, 16, 256, 256, A, None) == E
+    assert lib.moe_centroid_grad(A, A, A, 16, 256, 250, A, A, 1 << 20, None) == U
+    assert lib.moe_centroid_grad(A, None, A, 16, 256, 256, A, A, 1 << 20, None) == E
+    assert lib.moe_centroid_grad(A, A, A, 1024, 256, 256, A, A, 1 << 30, None) == U
+    assert lib.moe_centroid_grad(A, A, A, 16, 256, 256, A, None, 1 << 20, None) == \
+        L.MOE_ERR_WORKSPACE
+    assert lib.moe_centroid_grad(A, A, A, 16, 256, 256, A, A, 16, None) == L.MOE_ERR_WORKSPACE
+    # chunk starts (17 ints -> 80 B), row ranges (2 + 16 chunks -> 144 B), fp32 partials
+    assert L.moe_centroid_grad_workspace_size(256, 16, 256) == 80 + 144 + 18 * 256 * 4
 
 
 def test_header_is_c99_and_the_library_links_from_c(lib, tmp_path):

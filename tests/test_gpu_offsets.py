@@ -136,7 +136,9 @@ def test_backward_gemms_with_malformed_offsets(rows, off):
     xp = rand((rows, d), g)
     dz = torch.randn(rows, generator=g, device="cuda")
     de = torch.full((G + 1, d), SENTINEL, dtype=torch.bfloat16, device="cuda")
-    L.moe_centroid_grad(xp, dz, off_dev, G, rows, d, de[:G])
+    cws = L.moe_centroid_grad_workspace_size(rows, G, d)
+    cg_ws = torch.empty(cws, dtype=torch.uint8, device="cuda")
+    L.moe_centroid_grad(xp, dz, off_dev, G, rows, d, de[:G], cg_ws, cws)
     torch.cuda.synchronize()
     assert L.moe_get_device_status() == 0
     assert_guards(dacbig, rows, "dac")
