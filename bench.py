@@ -595,6 +595,9 @@ def main():
                          "pre-activations + backward + bias update (bf16)")
     ap.add_argument("--no-overlap", action="store_true",
                     help="run the shared expert after the routed experts on one stream")
+    ap.add_argument("--shared-join", default="auto", choices=["auto", "early", "late"],
+                    help="where the overlapped shared expert rejoins: before the routed GEMMs "
+                         "(early), before the combine (late), or by group size (auto)")
     ap.add_argument("--parallel", default="dp", choices=["dp", "ep", "ep-p2p"],
                     help="dp: every rank holds all experts, its own batch; ep: the routed "
                          "experts split over the ranks, token rows exchanged by NCCL "
@@ -683,7 +686,8 @@ def main():
                        routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
                        fp8=cfg.fp8, fused_gather=(args.mode == "fused"),
                        fused_scatter=(args.mode == "scatter"),
-                       overlap_shared=not args.no_overlap, device=dev)
+                       overlap_shared=not args.no_overlap, shared_join=args.shared_join,
+                       device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
     torch.cuda.empty_cache()
@@ -799,8 +803,8 @@ def main():
                             "regrouped by expert on the receiving rank" if ep_mode else
                             "fused gather" if lay.fused_gather else
                             "fused scatter" if lay.fused_scatter else "five-call"),
-                   "shared_expert": "side stream, overlapped" if lay.overlap_shared
-                   else "after the routed experts",
+                   "shared_expert": (f"side stream, overlapped, joins {lay.shared_join}"
+                                     if lay.overlap_shared else "after the routed experts"),
                    "parallelism": (f"ep{world}" if ep_mode else
                                    f"dp{world}" if world > 1 else "single"),
                    "l2": "inputs larger than L2 (22.6 GB of expert weights streamed per step)"

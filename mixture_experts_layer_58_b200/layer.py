@@ -63,7 +63,7 @@ class MoELayer:
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
                  fp8: bool = False, fused_gather: bool = False, fused_scatter: bool = False,
-                 overlap_shared: bool = True, device="cuda"):
+                 overlap_shared: bool = True, shared_join: str = "auto", device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -82,8 +82,14 @@ class MoELayer:
         # by its gate and writes it to its (token, slot) row; the combine then
         # adds K adjacent rows per token
         self.fused_scatter = bool(fused_scatter) and not self.fp8
-        # bf16: run the shared expert on a side stream next to the routed path
+        # bf16: run the shared expert on a side stream next to the routed path;
+        # shared_join: where the current stream waits for it -- "early" (before
+        # the routed GEMMs), "late" (before the combine) or "auto" (early when
+        # the routed groups average >= 256 rows, else late)
         self.overlap_shared = bool(overlap_shared) and not self.fp8
+        if shared_join not in ("auto", "early", "late"):
+            raise ValueError("shared_join must be 'auto', 'early' or 'late'")
+        self.shared_join = shared_join
         self.centroids = centroids.to(dev, bf).contiguous()
         self.bias = (bias.to(dev, torch.float32).contiguous() if bias is not None
                      else torch.zeros(self.n_routed, dtype=torch.float32, device=dev))
@@ -307,7 +313,9 @@ class MoELayer:
         # the shared expert overlaps only the HBM-bound route and dispatch and
         # the routed GEMMs run alone; decode-sized groups stream their weights
         # from HBM, and the shared expert runs next to them too.
-        join_early = side is not None and T * self.top_k >= 256 * self.n_routed
+        join_early = side is not None and (
+            self.shared_join == "early" or
+            (self.shared_join == "auto" and T * self.top_k >= 256 * self.n_routed))
         if T > 0:
             with ev("permute"):
                 self.permute(u)
