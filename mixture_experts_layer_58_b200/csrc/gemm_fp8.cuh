@@ -313,10 +313,21 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
           tmem_ld_wait();
           tc_fence_before();
           mbar_arrive(&pempty[pb]);
+          // packed fp32 FMAs (two lanes of fp32 per instruction, each
+          // rounded as a scalar fmaf): the promotion warps are bound by the
+          // instructions they issue per 128-K block, and this halves its FMAs
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            acc0[i] = fmaf(__uint_as_float(r0[i]), s0, acc0[i]);
-            acc1[i] = fmaf(__uint_as_float(r1[i]), s1, acc1[i]);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 q0 =
+                __ffma2_rn(make_float2(__uint_as_float(r0[i]), __uint_as_float(r0[i + 1])),
+                           make_float2(s0, s0), make_float2(acc0[i], acc0[i + 1]));
+            const float2 q1 =
+                __ffma2_rn(make_float2(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1])),
+                           make_float2(s1, s1), make_float2(acc1[i], acc1[i + 1]));
+            acc0[i] = q0.x;
+            acc0[i + 1] = q0.y;
+            acc1[i] = q1.x;
+            acc1[i + 1] = q1.y;
           }
         }
         if constexpr (EPI == EPI8_SWIGLU_Q) {
