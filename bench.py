@@ -817,6 +817,12 @@ def main():
         "layer_tflops": layer_tflops,
         "layer_frac_of_bf16_peak": layer_tflops / pk["bf16_tflops"],
         "layer_frac_of_tensor_peak": layer_tflops / (pk["bf16_tflops"] * (2 if cfg.fp8 else 1)),
+        "layer_frac_of_nominal_at_median_clock": (
+            layer_tflops / (NUM_SMS * BF16_FLOP_PER_CLK_PER_SM * (2 if cfg.fp8 else 1)
+                            * t["clocks"]["sm_mhz"] * 1e6 / 1e12)
+            if t["clocks"].get("sm_mhz") else None),
+        "target": "layer >= 60 % of the burst tensor peak (bf16 V3 prefill: <= "
+                  f"{T * cfg.flops_per_token() / (0.6 * pk['bf16_tflops'] * 1e12) * 1e3:.2f} ms)",
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2, "api": type(lay).__name__ + ".forward",
