@@ -529,6 +529,9 @@ class PeerExpertParallelMoELayer(MoELayer):
         if self._comm is None:
             self._comm = torch.cuda.Stream(device=self.device)
         comm = self._comm
+        # u and the output are used on the comm stream too
+        u.record_stream(comm)
+        dst.record_stream(comm)
         A.begin(uA, timers)
         B.begin(uB)
         dist.all_gather_into_tensor(A.all_counts.view(-1), A.counts, group=self.group)
@@ -555,7 +558,6 @@ class PeerExpertParallelMoELayer(MoELayer):
         B._barrier()
         B.finish(uB, residual, oB)
         cur.wait_stream(comm)
-        uA.record_stream(comm)
         self._step_counts = B.global_counts
         self._step_T = T
         return dst
