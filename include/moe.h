@@ -205,6 +205,15 @@ MOE_API int moe_grouped_ffn(const void* x, const float* x_scales, const int32_t*
 
 MOE_API size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dtype);
 
+/* moe_workspace_size: bytes of scratch one forward of the five calls needs if
+ * its calls share one workspace (they run in stream order): the larger of
+ * moe_permute_workspace_size(T, n_routed) and the grouped FFN's for the routed
+ * rows (T*top_k, inter) and for the shared expert(s) (T, shared_inter). The
+ * shared expert needs its own workspace if it runs beside the routed path on
+ * another stream. d is accepted for symmetry with the other calls. */
+MOE_API size_t moe_workspace_size(int T, int d, int n_routed, int top_k, int inter,
+                                  int shared_inter, moe_dtype dtype);
+
 /* The two halves of moe_grouped_ffn, for callers that keep h themselves.
  * moe_expert_up_swiglu:  h[rows, inter] = silu(x W1^T) * (x W3^T) per group.
  * moe_expert_down:       y[rows, d]     = h W2^T per group.

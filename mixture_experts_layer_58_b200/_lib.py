@@ -53,6 +53,7 @@ _SIGS = {
     "moe_grouped_ffn": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp,
                              _sz, _vp]),
     "moe_grouped_ffn_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "moe_expert_up_swiglu": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "moe_expert_down": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
     "moe_quant_act_fp8": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
@@ -189,6 +190,10 @@ def moe_grouped_ffn(x, x_scales, group_offsets, G, rows, d, inter, w13, w13_scal
     _check(_L().moe_grouped_ffn(_p(x), _p(x_scales), _p(group_offsets), G, rows, d, inter,
                                 _p(w13), _p(w13_scales), _p(w2), _p(w2_scales), dtype, _p(y),
                                 _p(workspace), ws_bytes, _stream(stream)), "moe_grouped_ffn")
+
+
+def moe_workspace_size(T, d, n_routed, top_k, inter, shared_inter=0, dtype=MOE_BF16) -> int:
+    return int(_L().moe_workspace_size(T, d, n_routed, top_k, inter, shared_inter, dtype))
 
 
 def moe_grouped_ffn_workspace_size(rows, inter, dtype=MOE_BF16) -> int:

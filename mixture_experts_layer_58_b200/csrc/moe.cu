@@ -549,6 +549,18 @@ size_t moe_grouped_ffn_workspace_size(int rows, int inter, moe_dtype dtype) {
   return (static_cast<size_t>(rows) * inter * 2 + 255) / 256 * 256;
 }
 
+size_t moe_workspace_size(int T, int d, int n_routed, int top_k, int inter, int shared_inter,
+                          moe_dtype dtype) {
+  (void)d;
+  if (T <= 0 || n_routed <= 0 || top_k <= 0 || inter <= 0) return 256;
+  const long long rows = static_cast<long long>(T) * top_k;
+  size_t ws = moe_permute_workspace_size(T, n_routed);
+  if (rows <= INT32_MAX)
+    ws = std::max(ws, moe_grouped_ffn_workspace_size(static_cast<int>(rows), inter, dtype));
+  if (shared_inter > 0) ws = std::max(ws, moe_grouped_ffn_workspace_size(T, shared_inter, dtype));
+  return ws;
+}
+
 int moe_expert_up_swiglu(const void* x, const int32_t* group_offsets, int G, int rows, int d,
                          int inter, const void* w13, void* h, moe_stream_t stream) {
   int rc = check_ffn_shape(G, rows, d, inter);

@@ -59,6 +59,10 @@ def test_workspace_sizes(lib):
     assert L.moe_permute_workspace_size(200, 16) == 256          # 2 chunks * 16 * 4 = 128 -> 256
     assert L.moe_grouped_ffn_workspace_size(131072, 2048) == 131072 * 2048 * 2
     assert L.moe_grouped_ffn_workspace_size(0, 2048) == 256
+    # one workspace for the five calls of a V3 prefill forward: the h of the
+    # routed rows dominates
+    assert L.moe_workspace_size(16384, 7168, 256, 8, 2048, 2048) == 131072 * 2048 * 2
+    assert L.moe_workspace_size(64, 256, 16, 4, 128, 4096) == 64 * 4096 * 2
 
 
 def rc_route(lib, **kw):
