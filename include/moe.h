@@ -535,9 +535,12 @@ MOE_API int moe_gather_rows(const void* src, int n_src, const int32_t* index, in
  *   of `world` pointers to the ranks' expert output buffers [recv_capacity,
  *   d] bf16). out may alias residual.
  * moe_ipc_get_handle: the 64-byte CUDA IPC handle of the allocation that
- *   holds dev_ptr, and dev_ptr's byte offset in it. moe_ipc_open_handle maps
- *   a handle from another process on this GPU (*base = the allocation's
- *   start; add the offset); moe_ipc_close_handle unmaps it.
+ *   holds dev_ptr, and dev_ptr's byte offset in it (the allocation must come
+ *   from cudaMalloc, e.g. PyTorch's default caching allocator; memory from
+ *   the virtual-memory API, such as expandable segments, has no such handle
+ *   and the call returns MOE_ERR_CUDA). moe_ipc_open_handle maps a handle
+ *   from another process on this GPU (*base = the allocation's start; add
+ *   the offset); moe_ipc_close_handle unmaps it.
  */
 MOE_API int moe_ep_plan_device(const int32_t* all_counts, int world, int n_local, int rank,
                                long long recv_capacity, const int32_t* add_counts,

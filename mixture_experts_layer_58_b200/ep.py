@@ -305,7 +305,8 @@ class PeerExpertParallelMoELayer(MoELayer):
 
     Nothing is read back to the host. The receive buffers hold recv_capacity
     rows (default W*T*K, every rank's every row: no step can overflow); the
-    other ranks' buffers are mapped with CUDA IPC. With world/rank given and no
+    other ranks' buffers are mapped with CUDA IPC, which needs PyTorch's
+    default CUDA allocator (expandable segments have no IPC handles). With world/rank given and no
     group the layer is one of several ranks emulated in one process: the
     caller links them with link_emulated_ranks and drives the stages (begin,
     plan, dispatch, experts, finish) in rank order, which needs no kernel to
