@@ -24,7 +24,9 @@ def _child(handle, offset, n, d, q):
         dst = torch.empty(n, d, dtype=torch.bfloat16, device="cuda")
         L.moe_gather_rows(base + offset, n, idx, n, d, dst)
         torch.cuda.synchronize()
-        q.put(("ok", dst.cpu()))
+        # a numpy array pickles by value (a torch CPU tensor would be shared
+        # through a file descriptor that dies with this process)
+        q.put(("ok", dst.float().cpu().numpy()))
         L.moe_ipc_close_handle(base)
     except Exception as exc:  # noqa: BLE001 - reported to the parent
         q.put(("error", repr(exc)))
@@ -50,4 +52,4 @@ def test_ipc_handle_maps_a_tensor_in_another_process(cuda_ok):
         if p.is_alive():
             p.kill()
     assert status == "ok", got
-    assert torch.equal(got, x.cpu())
+    assert torch.equal(torch.from_numpy(got), x.float().cpu())
