@@ -189,7 +189,7 @@ __device__ __forceinline__ void add_bf16x8(float (&a)[8], const uint4& v) {
 // SLOTS (the fused-scatter mode): the routed rows already carry their gate
 // and sit in slot order, y[t*K + k]; slot k counts when pos[t,k] >= 0.
 template <bool SLOTS>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)   // two blocks per SM: 16 warps of loads in flight
 combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ pos,
                const float* __restrict__ gate, const __nv_bfloat16* __restrict__ shared_out,
                const __nv_bfloat16* residual, int T, int d, int K,
