@@ -105,6 +105,30 @@ MOE_API int moe_route(const void* u, const void* centroids, const float* bias, i
                       int32_t* topk_idx, float* topk_gate, int32_t* expert_counts,
                       moe_stream_t stream);
 
+/* Split-K form of moe_route for small batches (decode). moe_route gives each
+ * CTA 128 tokens and the whole K = d, so a batch of a few hundred tokens runs
+ * on one or two SMs, each reading all of the centroids. Here CTA (b, y) takes
+ * token block b and the y-th slice of K and writes its fp32 partial logits
+ * to the workspace; a second kernel adds the slices (fixed order) and does
+ * the same selection, gates and counts as moe_route. Arguments as moe_route,
+ * plus:
+ *   workspace  device scratch, 16-B aligned, at least
+ *              moe_route_splitk_workspace_size(T, d, n_routed) bytes; owned by
+ *              the caller, overwritten, may be reused once the call's kernels
+ *              have finished on the stream. NULL or too small ->
+ *              MOE_ERR_WORKSPACE.
+ * The logits are the same fp32 sums of bf16 products as moe_route's, added in
+ * another order, so keys closer than the fp32 rounding of a sum may select
+ * differently; every other result follows from the logits as in moe_route.
+ * The slice count depends on T and d only.
+ */
+MOE_API size_t moe_route_splitk_workspace_size(int T, int d, int n_routed);
+MOE_API int moe_route_splitk(const void* u, const void* centroids, const float* bias, int T,
+                             int d, int n_routed, int top_k, moe_gate_kind kind,
+                             float routed_scale, int32_t* topk_idx, float* topk_gate,
+                             int32_t* expert_counts, void* workspace, size_t ws_bytes,
+                             moe_stream_t stream);
+
 /* ------------------------------------------------------------------ permute
  * Dispatch: copy each token's row into an expert-contiguous buffer, once per
  * selected expert (the per-expert grouping of tokens that the deepseekmodel.com

@@ -45,6 +45,9 @@ _vp, _i, _ll, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes
 
 _SIGS = {
     "moe_route": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp]),
+    "moe_route_splitk": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _sz,
+                              _vp]),
+    "moe_route_splitk_workspace_size": (_sz, [_i, _i, _i]),
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
@@ -148,6 +151,19 @@ def moe_route(u, centroids, bias, T, d, n_routed, top_k, kind, routed_scale, top
     _check(_L().moe_route(_p(u), _p(centroids), _p(bias), T, d, n_routed, top_k, k,
                           float(routed_scale), _p(topk_idx), _p(topk_gate), _p(expert_counts),
                           _stream(stream)), "moe_route")
+
+
+def moe_route_splitk_workspace_size(T, d, n_routed):
+    return _L().moe_route_splitk_workspace_size(T, d, n_routed)
+
+
+def moe_route_splitk(u, centroids, bias, T, d, n_routed, top_k, kind, routed_scale, topk_idx,
+                     topk_gate, expert_counts, workspace, ws_bytes, stream=None):
+    k = GATE_KINDS.get(kind, kind)
+    _check(_L().moe_route_splitk(_p(u), _p(centroids), _p(bias), T, d, n_routed, top_k, k,
+                                 float(routed_scale), _p(topk_idx), _p(topk_gate),
+                                 _p(expert_counts), _p(workspace), ws_bytes, _stream(stream)),
+           "moe_route_splitk")
 
 
 def moe_permute(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm, expert_offsets, pos,

@@ -341,24 +341,60 @@ int check_ffn_shape(int G, int rows, int d, int inter) {
   return MOE_OK;
 }
 
+// Split-K form of the gate GEMM for small batches: splits chosen from the
+// shapes alone (so the workspace size needs no device query) -- K blocks of
+// at least 4 stages per CTA and at most ~128 CTAs over all token blocks.
+inline int route_splits(int T, int d) {
+  const int blocks = (T + kBM - 1) / kBM;
+  const int num_kb = d / kBK;
+  int splits = std::max(1, std::min((num_kb + 3) / 4, 128 / std::max(1, blocks)));
+  const int per = (num_kb + splits - 1) / splits;
+  return (num_kb + per - 1) / per;
+}
+
 template <int TOPK>
 int launch_route_k(int kind, const CUtensorMap& tmU, const CUtensorMap& tmE, const float* bias,
                    int T, int d, int n_routed, int n_pad, uint32_t tcols, float scale,
-                   int32_t* idx, float* gate, int32_t* counts, unsigned int* status,
-                   cudaStream_t st) {
+                   int32_t* idx, float* gate, int32_t* counts, float* partial, int splits,
+                   unsigned int* status, cudaStream_t st) {
   const size_t smem = RouteSmem::bytes(n_pad);
-  const int grid = (T + kBM - 1) / kBM;
+  const int blocks = (T + kBM - 1) / kBM;
+  const int num_kb = d / kBK;
   int rc;
+  if (partial == nullptr) {
+    if (kind == MOE_GATE_SIGMOID_BIAS) {
+      auto k = route_kernel<TOPK, 0, false>;
+      if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
+      k<<<blocks, kGemmThreads, smem, st>>>(tmU, tmE, bias, T, d, n_routed, n_pad, tcols, scale,
+                                            idx, gate, counts, nullptr, num_kb, status);
+    } else {
+      auto k = route_kernel<TOPK, 1, false>;
+      if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
+      k<<<blocks, kGemmThreads, smem, st>>>(tmU, tmE, bias, T, d, n_routed, n_pad, tcols, scale,
+                                            idx, gate, counts, nullptr, num_kb, status);
+    }
+    MOE_CUDA(cudaGetLastError());
+    return MOE_OK;
+  }
+  const int per = (num_kb + splits - 1) / splits;
+  const dim3 grid(blocks, splits);
+  const int sel_blocks = (T + kSelectWarps - 1) / kSelectWarps;
   if (kind == MOE_GATE_SIGMOID_BIAS) {
-    auto k = route_kernel<TOPK, 0>;
+    auto k = route_kernel<TOPK, 0, true>;
     if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
     k<<<grid, kGemmThreads, smem, st>>>(tmU, tmE, bias, T, d, n_routed, n_pad, tcols, scale, idx,
-                                        gate, counts, status);
+                                        gate, counts, partial, per, status);
+    MOE_CUDA(cudaGetLastError());
+    route_select_kernel<TOPK, 0><<<sel_blocks, 32 * kSelectWarps, 0, st>>>(
+        partial, splits, bias, T, n_routed, n_pad, scale, idx, gate, counts);
   } else {
-    auto k = route_kernel<TOPK, 1>;
+    auto k = route_kernel<TOPK, 1, true>;
     if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
     k<<<grid, kGemmThreads, smem, st>>>(tmU, tmE, bias, T, d, n_routed, n_pad, tcols, scale, idx,
-                                        gate, counts, status);
+                                        gate, counts, partial, per, status);
+    MOE_CUDA(cudaGetLastError());
+    route_select_kernel<TOPK, 1><<<sel_blocks, 32 * kSelectWarps, 0, st>>>(
+        partial, splits, nullptr, T, n_routed, n_pad, scale, idx, gate, counts);
   }
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
@@ -430,17 +466,11 @@ int moe_get_device_status(unsigned int* status, int clear) {
 }
 
 // ------------------------------------------------------------------ route
-int moe_route(const void* u, const void* centroids, const float* bias, int T, int d, int n_routed,
-              int top_k, moe_gate_kind kind, float routed_scale, int32_t* topk_idx,
-              float* topk_gate, int32_t* expert_counts, moe_stream_t stream) {
-  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
-  if (kind != MOE_GATE_SIGMOID_BIAS && kind != MOE_GATE_SOFTMAX_TOPK) return MOE_ERR_INVALID_ARG;
-  if (!expert_counts || !centroids || !aligned16(centroids)) return MOE_ERR_INVALID_ARG;
-  if (T > 0 && (!u || !topk_idx || !topk_gate || !aligned16(u))) return MOE_ERR_INVALID_ARG;
-  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 256 != 0)
-    return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (!(routed_scale == routed_scale)) return MOE_ERR_INVALID_ARG;
-  cudaStream_t st = as_stream(stream);
+namespace {
+int route_impl(const void* u, const void* centroids, const float* bias, int T, int d,
+               int n_routed, int top_k, moe_gate_kind kind, float routed_scale,
+               int32_t* topk_idx, float* topk_gate, int32_t* expert_counts, float* partial,
+               cudaStream_t st) {
   MOE_CUDA(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * n_routed, st));
   if (T == 0) return MOE_OK;
   DeviceInfo* di;
@@ -453,10 +483,12 @@ int moe_route(const void* u, const void* centroids, const float* bias, int T, in
   if ((rc = make_tmap_bf16(&tmU, u, d, T, kBM)) != MOE_OK) return rc;
   if ((rc = make_tmap_bf16(&tmE, centroids, d, n_routed, n_pad)) != MOE_OK) return rc;
   const float* b = (kind == MOE_GATE_SIGMOID_BIAS) ? bias : nullptr;
+  const int splits = partial ? route_splits(T, d) : 1;
 #define MOE_ROUTE_CASE(KK)                                                                   \
   case KK:                                                                                   \
     return launch_route_k<KK>(kind, tmU, tmE, b, T, d, n_routed, n_pad, tcols, routed_scale, \
-                              topk_idx, topk_gate, expert_counts, di->status, st);
+                              topk_idx, topk_gate, expert_counts, partial, splits, di->status, \
+                              st);
   switch (top_k) {
     MOE_ROUTE_CASE(1)
     MOE_ROUTE_CASE(2)
@@ -469,6 +501,52 @@ int moe_route(const void* u, const void* centroids, const float* bias, int T, in
     default: return MOE_ERR_UNSUPPORTED_SHAPE;
   }
 #undef MOE_ROUTE_CASE
+}
+
+int route_check(const void* u, const void* centroids, int T, int d, int n_routed, int top_k,
+                moe_gate_kind kind, float routed_scale, int32_t* topk_idx, float* topk_gate,
+                int32_t* expert_counts) {
+  if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (kind != MOE_GATE_SIGMOID_BIAS && kind != MOE_GATE_SOFTMAX_TOPK) return MOE_ERR_INVALID_ARG;
+  if (!expert_counts || !centroids || !aligned16(centroids)) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!u || !topk_idx || !topk_gate || !aligned16(u))) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 256 != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!(routed_scale == routed_scale)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+}  // namespace
+
+int moe_route(const void* u, const void* centroids, const float* bias, int T, int d, int n_routed,
+              int top_k, moe_gate_kind kind, float routed_scale, int32_t* topk_idx,
+              float* topk_gate, int32_t* expert_counts, moe_stream_t stream) {
+  const int rc = route_check(u, centroids, T, d, n_routed, top_k, kind, routed_scale, topk_idx,
+                             topk_gate, expert_counts);
+  if (rc != MOE_OK) return rc;
+  return route_impl(u, centroids, bias, T, d, n_routed, top_k, kind, routed_scale, topk_idx,
+                    topk_gate, expert_counts, nullptr, as_stream(stream));
+}
+
+size_t moe_route_splitk_workspace_size(int T, int d, int n_routed) {
+  if (T <= 0 || d <= 0 || d % 256 != 0 || n_routed <= 0 || n_routed > kRouteMaxExperts)
+    return 16;
+  const size_t n_pad = std::max(16, (n_routed + 15) / 16 * 16);
+  const size_t bytes = static_cast<size_t>(route_splits(T, d)) * T * n_pad * sizeof(float);
+  return (bytes + 255) / 256 * 256;
+}
+
+int moe_route_splitk(const void* u, const void* centroids, const float* bias, int T, int d,
+                     int n_routed, int top_k, moe_gate_kind kind, float routed_scale,
+                     int32_t* topk_idx, float* topk_gate, int32_t* expert_counts,
+                     void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  const int rc = route_check(u, centroids, T, d, n_routed, top_k, kind, routed_scale, topk_idx,
+                             topk_gate, expert_counts);
+  if (rc != MOE_OK) return rc;
+  if (T > 0 && (!workspace || !aligned16(workspace) ||
+                ws_bytes < moe_route_splitk_workspace_size(T, d, n_routed)))
+    return MOE_ERR_WORKSPACE;
+  return route_impl(u, centroids, bias, T, d, n_routed, top_k, kind, routed_scale, topk_idx,
+                    topk_gate, expert_counts, static_cast<float*>(workspace), as_stream(stream));
 }
 
 // ------------------------------------------------------------------ permute

@@ -29,13 +29,81 @@ struct RouteSmem {
   }
 };
 
+// One token's selection, shared by the fused kernel and the split-K form:
+// fold logit z of expert j into the running top-K (keys in descending order;
+// strictly-greater insertion over ascending j = the lower index wins a tie).
 template <int TOPK, int KIND>
+__device__ __forceinline__ void route_insert(float z, int j, float bias_j, float (&kv)[TOPK],
+                                             float (&sv)[TOPK], int (&ki)[TOPK]) {
+  float s, key;
+  if constexpr (KIND == 0) {
+    s = 1.0f / (1.0f + expf(-z));
+    key = s + bias_j;
+  } else {
+    s = z;
+    key = z;
+  }
+  if (key > kv[TOPK - 1]) {
+#pragma unroll
+    for (int p = TOPK - 1; p >= 0; --p) {
+      const bool above_prev = (p > 0) && (key > kv[p > 0 ? p - 1 : 0]);
+      if (key > kv[p]) {
+        if (above_prev) {
+          kv[p] = kv[p - 1];
+          sv[p] = sv[p - 1];
+          ki[p] = ki[p - 1];
+        } else {
+          kv[p] = key;
+          sv[p] = s;
+          ki[p] = j;
+        }
+      }
+    }
+  }
+}
+
+// Gates of one token's selection (sigmoid: S s_k / sum; softmax: S softmax
+// of the selected logits), its row of topk_idx / topk_gate, and its loads
+// added to the block's shared-memory histogram.
+template <int TOPK, int KIND>
+__device__ __forceinline__ void route_emit(const float (&sv)[TOPK], const int (&ki)[TOPK],
+                                           float routed_scale, int t, int32_t* topk_idx,
+                                           float* topk_gate, int* s_hist) {
+  float g[TOPK];
+  float sum = 0.0f;
+  if constexpr (KIND == 0) {
+#pragma unroll
+    for (int p = 0; p < TOPK; ++p) {
+      g[p] = sv[p];
+      sum += sv[p];
+    }
+  } else {
+    const float m = sv[0];
+#pragma unroll
+    for (int p = 0; p < TOPK; ++p) {
+      g[p] = expf(sv[p] - m);
+      sum += g[p];
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < TOPK; ++p) {
+    topk_idx[static_cast<size_t>(t) * TOPK + p] = ki[p];
+    topk_gate[static_cast<size_t>(t) * TOPK + p] = (routed_scale * g[p]) / sum;
+    if (ki[p] >= 0) atomicAdd(&s_hist[ki[p]], 1);   // -1 only for non-finite logits
+  }
+}
+
+// PARTIAL (the split-K form for small batches): CTA (b, y) accumulates the
+// logits of token block b over K blocks [y*kb_per_split, +kb_per_split) only
+// and writes them, fp32, to partial[y][t][n_pad]; route_select_kernel adds
+// the splits and selects.
+template <int TOPK, int KIND, bool PARTIAL>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
              const float* __restrict__ bias, int T, int d, int n_routed, int n_pad,
              uint32_t tmem_cols, float routed_scale, int32_t* __restrict__ topk_idx,
              float* __restrict__ topk_gate, int32_t* __restrict__ counts,
-             unsigned int* status) {
+             float* __restrict__ partial, int kb_per_split, unsigned int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int a_bytes = kBM * kBK * 2;
@@ -51,7 +119,8 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_kb = d / kBK;
+  const int kb0 = PARTIAL ? static_cast<int>(blockIdx.y) * kb_per_split : 0;
+  const int kb1 = PARTIAL ? min(kb0 + kb_per_split, d / kBK) : d / kBK;
   const int row0 = blockIdx.x * kBM;
 
   if (warp == 0) {
@@ -83,7 +152,7 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued = 0, issued_par = 0;
-    for (int kb = 0; kb < num_kb; ++kb) {
+    for (int kb = kb0; kb < kb1; ++kb) {
       if (!mbar_wait(&empty[stage], phase ^ 1u, status, kStatusTimeoutProducer)) break;
       mbar_arrive_expect_tx(&full[stage], a_bytes + b_bytes);
       tma_load_2d(sA + stage * a_bytes, &tmU, &full[stage], kb * kBK, row0);
@@ -103,7 +172,7 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int kb = 0; kb < num_kb; ++kb) {
+    for (int kb = kb0; kb < kb1; ++kb) {
       if (!mbar_wait(&full[stage], phase, status, kStatusTimeoutMma)) {
         ok = false;
         break;
@@ -113,7 +182,7 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
       const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * b_bytes));
 #pragma unroll
       for (int k = 0; k < kBK / kUmmaK; ++k)
-        umma_bf16(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+        umma_bf16(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc, ((kb - kb0) | k) != 0);
       umma_commit(&empty[stage]);
       if (++stage == kStages) {
         stage = 0;
@@ -139,7 +208,23 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
       ki[p] = -1;
     }
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    if (have) {
+    if constexpr (PARTIAL) {
+      // this split's logits of the thread's token, fp32, to the workspace
+      if (have && t < T) {
+        float* prow = partial + (static_cast<size_t>(blockIdx.y) * T + t) * n_pad;
+        for (int c = 0; c < n_pad; c += 32) {
+          uint32_t zr[32];
+          tmem_ld_32cols(taddr + c, zr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            if (c + i < n_pad)
+              *reinterpret_cast<float4*>(prow + c + i) =
+                  make_float4(__uint_as_float(zr[i]), __uint_as_float(zr[i + 1]),
+                              __uint_as_float(zr[i + 2]), __uint_as_float(zr[i + 3]));
+        }
+      }
+    } else if (have) {
       for (int c = 0; c < n_pad; c += 32) {
         uint32_t zr[32];
         tmem_ld_32cols(taddr + c, zr);
@@ -147,66 +232,20 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int j = c + i;
-          if (j < n_routed) {
-            const float z = __uint_as_float(zr[i]);
-            float s, key;
-            if constexpr (KIND == 0) {
-              s = 1.0f / (1.0f + expf(-z));
-              key = s + s_bias[j];
-            } else {
-              s = z;
-              key = z;
-            }
-            if (key > kv[TOPK - 1]) {
-#pragma unroll
-              for (int p = TOPK - 1; p >= 0; --p) {
-                const bool above_prev = (p > 0) && (key > kv[p > 0 ? p - 1 : 0]);
-                if (key > kv[p]) {
-                  if (above_prev) {
-                    kv[p] = kv[p - 1];
-                    sv[p] = sv[p - 1];
-                    ki[p] = ki[p - 1];
-                  } else {
-                    kv[p] = key;
-                    sv[p] = s;
-                    ki[p] = j;
-                  }
-                }
-              }
-            }
-          }
+          if (j < n_routed)
+            route_insert<TOPK, KIND>(__uint_as_float(zr[i]), j, s_bias[j], kv, sv, ki);
         }
       }
     }
     tc_fence_before();
-    if (have && t < T) {
-      float g[TOPK];
-      float sum = 0.0f;
-      if constexpr (KIND == 0) {
-#pragma unroll
-        for (int p = 0; p < TOPK; ++p) {
-          g[p] = sv[p];
-          sum += sv[p];
-        }
-      } else {
-        const float m = sv[0];
-#pragma unroll
-        for (int p = 0; p < TOPK; ++p) {
-          g[p] = expf(sv[p] - m);
-          sum += g[p];
-        }
+    if constexpr (!PARTIAL) {
+      if (have && t < T)
+        route_emit<TOPK, KIND>(sv, ki, routed_scale, t, topk_idx, topk_gate, s_hist);
+      named_bar_sync(1, 128);
+      for (int e = threadIdx.x - 64; e < n_routed; e += 128) {
+        const int c = s_hist[e];
+        if (c) atomicAdd(&counts[e], c);
       }
-#pragma unroll
-      for (int p = 0; p < TOPK; ++p) {
-        topk_idx[static_cast<size_t>(t) * TOPK + p] = ki[p];
-        topk_gate[static_cast<size_t>(t) * TOPK + p] = (routed_scale * g[p]) / sum;
-        if (ki[p] >= 0) atomicAdd(&s_hist[ki[p]], 1);   // -1 only for non-finite logits
-      }
-    }
-    named_bar_sync(1, 128);
-    for (int e = threadIdx.x - 64; e < n_routed; e += 128) {
-      const int c = s_hist[e];
-      if (c) atomicAdd(&counts[e], c);
     }
   }
 
@@ -215,6 +254,101 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// Split-K second pass: one warp per token adds its logits over the splits
+// (fixed order, fp32; lane l holds experts l, l+32, ...), then selects the
+// top-K with warp shuffles: K rounds of a warp-wide maximum of (key, lower
+// expert index on equal keys), the winner leaving the candidates -- the same
+// selection and order as route_insert. Gates, idx and the histogram as the
+// fused kernel. Keys that are not finite numbers are never selected.
+constexpr int kSelectWarps = 8;
+template <int TOPK, int KIND>
+__global__ void __launch_bounds__(32 * kSelectWarps)
+route_select_kernel(const float* __restrict__ partial, int splits, const float* __restrict__ bias,
+                    int T, int n_routed, int n_pad, float routed_scale,
+                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                    int32_t* __restrict__ counts) {
+  __shared__ int s_hist[kRouteMaxExperts];
+  for (int e = threadIdx.x; e < kRouteMaxExperts; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
+  constexpr int kPer = kRouteMaxExperts / 32;
+  if (t < T) {
+    float key[kPer], sval[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int j = lane + 32 * i;
+      key[i] = -INFINITY;
+      sval[i] = 0.0f;
+      if (j < n_routed) {
+        float z = 0.0f;
+        for (int y = 0; y < splits; ++y)
+          z += __ldg(partial + (static_cast<size_t>(y) * T + t) * n_pad + j);
+        float sv, kv;
+        if constexpr (KIND == 0) {
+          sv = 1.0f / (1.0f + expf(-z));
+          kv = sv + (bias != nullptr ? __ldg(bias + j) : 0.0f);
+        } else {
+          sv = z;
+          kv = z;
+        }
+        if (kv == kv) {                                  // NaN keys are never selected
+          key[i] = kv;
+          sval[i] = sv;
+        }
+      }
+    }
+    float sel_s[TOPK];
+    int sel_j[TOPK];
+#pragma unroll
+    for (int p = 0; p < TOPK; ++p) {
+      // this lane's best remaining candidate (ascending j on equal keys)
+      float bk = -INFINITY;
+      int bj = 0x7fffffff, bi = -1;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if (key[i] > bk) {
+          bk = key[i];
+          bj = lane + 32 * i;
+          bi = i;
+        }
+      // warp maximum of (key, then the lower index)
+      float wk = bk;
+      int wj = bi >= 0 ? bj : 0x7fffffff;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        const float ok = __shfl_xor_sync(0xffffffffu, wk, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, wj, o);
+        if (ok > wk || (ok == wk && oj < wj)) {
+          wk = ok;
+          wj = oj;
+        }
+      }
+      const bool found = wk > -INFINITY;
+      float ws = 0.0f;
+      if (found && bi >= 0 && bj == wj) {
+#pragma unroll
+        for (int i = 0; i < kPer; ++i)                    // (static indexes: registers)
+          if (i == bi) {
+            ws = sval[i];
+            key[i] = -INFINITY;                           // leaves the candidates
+          }
+      }
+      // the winner's s value from its lane
+      ws = __shfl_sync(0xffffffffu, ws, found ? (wj & 31) : 0);
+      sel_s[p] = found ? ws : 0.0f;
+      sel_j[p] = found ? wj : -1;
+    }
+    if (lane == 0)
+      route_emit<TOPK, KIND>(sel_s, sel_j, routed_scale, t, topk_idx, topk_gate, s_hist);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
+    const int c = s_hist[e];
+    if (c) atomicAdd(&counts[e], c);
   }
 }
 

@@ -275,7 +275,7 @@ class ExpertParallelMoELayer(MoELayer):
     # route (1 + a memset), permute (3), regroup, up, down, ungroup, shared
     # FFN (2), combine; the exchanges are NCCL's
     def launches_per_step(self) -> int:
-        n = 1 + 3 + 4 + 1
+        n = (2 if self.route_split else 1) + 3 + 4 + 1
         if self.ws13 is not None:
             n += 2
         if self.gate_kind == "sigmoid":
@@ -580,7 +580,7 @@ class PeerExpertParallelMoELayer(MoELayer):
     # route (1 + a memset), permute index (2), plan, dispatch, up, down, shared
     # FFN (2), combine; the all-gather and the barriers are NCCL's
     def launches_per_step(self) -> int:
-        n = 1 + 2 + 1 + 1 + 2 + 1
+        n = (2 if self.route_split else 1) + 2 + 1 + 1 + 2 + 1
         if self.ws13 is not None:
             n += 2
         n *= self.micro_batches

@@ -63,7 +63,8 @@ class MoELayer:
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
                  fp8: bool = False, fused_gather: bool = False, fused_scatter: bool = False,
-                 overlap_shared: bool = True, shared_join: str = "auto", device="cuda"):
+                 overlap_shared: bool = True, shared_join: str = "auto",
+                 split_route: str = "auto", device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -90,6 +91,12 @@ class MoELayer:
         if shared_join not in ("auto", "early", "late"):
             raise ValueError("shared_join must be 'auto', 'early' or 'late'")
         self.shared_join = shared_join
+        # split_route: the gate GEMM split over K (moe_route_splitk) -- "on",
+        # "off" or "auto" (on for batches of at most 2048 tokens, where
+        # moe_route's 128-token CTAs would leave most SMs idle)
+        if split_route not in ("auto", "on", "off"):
+            raise ValueError("split_route must be 'auto', 'on' or 'off'")
+        self.split_route = split_route
         self.centroids = centroids.to(dev, bf).contiguous()
         self.bias = (bias.to(dev, torch.float32).contiguous() if bias is not None
                      else torch.zeros(self.n_routed, dtype=torch.float32, device=dev))
@@ -113,6 +120,7 @@ class MoELayer:
                 self.ws13, self.ws13_s = self.ws13
                 self.ws2, self.ws2_s = self.quant_weights(self.ws2[None])
         self._T = -1
+        self.route_split = False
 
     # ------------------------------------------------------------------ setup
     def pack_w13(self, w1, w3):
@@ -160,6 +168,12 @@ class MoELayer:
         self.x_perm = (None if (self.fp8 or self.fused_gather) else
                        torch.empty((rows, d), dtype=torch.bfloat16, device=dev))
         self.y_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
+        self.route_split = (self.split_route == "on" or
+                            (self.split_route == "auto" and T <= 2048))
+        self.route_ws_bytes = (L.moe_route_splitk_workspace_size(T, d, self.n_routed)
+                               if self.route_split else 0)
+        self.route_ws = (torch.empty(self.route_ws_bytes, dtype=torch.uint8, device=dev)
+                         if self.route_split else None)
         self.perm_ws_bytes = L.moe_permute_workspace_size(T, self.n_routed)
         self.perm_ws = torch.empty(self.perm_ws_bytes, dtype=torch.uint8, device=dev)
         dt = L.MOE_FP8_E4M3 if self.fp8 else L.MOE_BF16
@@ -187,9 +201,15 @@ class MoELayer:
     # ------------------------------------------------------------------ steps
     def route(self, u):
         T = u.shape[0]
-        L.moe_route(u, self.centroids, self.bias if self.gate_kind == "sigmoid" else None, T,
-                    self.d, self.n_routed, self.top_k, self.gate_kind, self.routed_scale,
-                    self.topk_idx, self.topk_gate, self.counts)
+        bias = self.bias if self.gate_kind == "sigmoid" else None
+        if self.route_split:
+            L.moe_route_splitk(u, self.centroids, bias, T, self.d, self.n_routed, self.top_k,
+                               self.gate_kind, self.routed_scale, self.topk_idx, self.topk_gate,
+                               self.counts, self.route_ws, self.route_ws_bytes)
+        else:
+            L.moe_route(u, self.centroids, bias, T, self.d, self.n_routed, self.top_k,
+                        self.gate_kind, self.routed_scale, self.topk_idx, self.topk_gate,
+                        self.counts)
 
     def permute(self, u):
         T = u.shape[0]
@@ -467,7 +487,7 @@ class MoELayer:
             self.update_bias()
         return out
 
-    # kernels launched by one step(): route (1 + a memset), permute (3; FP8:
+    # kernels launched by one step(): route (1, split over K 2; + a memset), permute (3; FP8:
     # + the activation quantisation), routed and shared FFN, combine (1),
     # bias update (1)
     def launches_per_step(self) -> int:
@@ -477,7 +497,7 @@ class MoELayer:
         perm = 2 if self.fused_gather else 3
         if self.fused_scatter:
             perm += 1                       # the slot index
-        n = 1 + perm + ffn + 1
+        n = (2 if self.route_split else 1) + perm + ffn + 1
         if self.ws13 is not None:
             n += ffn
         if self.gate_kind == "sigmoid":
