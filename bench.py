@@ -530,7 +530,7 @@ def variant_line(name, args, dev, local, stream, pk):
     e_host, b_host = synth.centroids(cfg), synth.bias(cfg)
     lay = MoELayer(e_host, b_host, W1, W3, W2, synth.shared_weights(cfg, "cuda"),
                    top_k=cfg.top_k, routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
-                   gamma=cfg.gamma, fp8=cfg.fp8, device=dev)
+                   gamma=cfg.gamma, fp8=cfg.fp8, split_route=args.split_route, device=dev)
     del W1, W3, W2
     torch.cuda.empty_cache()
     u = synth.tokens(cfg).to(dev)
@@ -598,6 +598,9 @@ def main():
     ap.add_argument("--shared-join", default="auto", choices=["auto", "early", "late"],
                     help="where the overlapped shared expert rejoins: before the routed GEMMs "
                          "(early), before the combine (late), or by group size (auto)")
+    ap.add_argument("--split-route", default="auto", choices=["auto", "on", "off"],
+                    help="gate GEMM split over K with a separate top-K pass (on), in one "
+                         "fused pass (off), or split for batches of at most 2048 tokens (auto)")
     ap.add_argument("--parallel", default="dp", choices=["dp", "ep", "ep-p2p"],
                     help="dp: every rank holds all experts, its own batch; ep: the routed "
                          "experts split over the ranks, token rows exchanged by NCCL "
@@ -687,7 +690,7 @@ def main():
                        fp8=cfg.fp8, fused_gather=(args.mode == "fused"),
                        fused_scatter=(args.mode == "scatter"),
                        overlap_shared=not args.no_overlap, shared_join=args.shared_join,
-                       device=dev)
+                       split_route=args.split_route, device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
     torch.cuda.empty_cache()
@@ -803,6 +806,8 @@ def main():
                             "regrouped by expert on the receiving rank" if ep_mode else
                             "fused gather" if lay.fused_gather else
                             "fused scatter" if lay.fused_scatter else "five-call"),
+                   "route": ("gate GEMM split over K, then a warp-per-token top-K pass"
+                             if lay.route_split else "gate GEMM and top-K in one fused pass"),
                    "shared_expert": (f"side stream, overlapped, joins {lay.shared_join}"
                                      if lay.overlap_shared else "after the routed experts"),
                    "parallelism": (f"ep{world}" if ep_mode else

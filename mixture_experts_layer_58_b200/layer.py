@@ -83,11 +83,12 @@ class MoELayer:
         # by its gate and writes it to its (token, slot) row; the combine then
         # adds K adjacent rows per token
         self.fused_scatter = bool(fused_scatter) and not self.fp8
-        # bf16: run the shared expert on a side stream next to the routed path;
+        # run the shared expert on a side stream next to the routed path (FP8:
+        # with its own quantisation of u, so it does not wait for the dispatch);
         # shared_join: where the current stream waits for it -- "early" (before
         # the routed GEMMs), "late" (before the combine) or "auto" (early when
         # the routed groups average >= 256 rows, else late)
-        self.overlap_shared = bool(overlap_shared) and not self.fp8
+        self.overlap_shared = bool(overlap_shared)
         if shared_join not in ("auto", "early", "late"):
             raise ValueError("shared_join must be 'auto', 'early' or 'late'")
         self.shared_join = shared_join
@@ -221,10 +222,11 @@ class MoELayer:
             return
         if self.fp8:
             # each token quantised once (1x128 tiles) inside the dispatch, its
-            # codes written to its K rows and to u8 for the shared expert
+            # codes written to its K rows and, for an in-line shared expert, to u8
+            own_u8 = self.ws13 is not None and not self.overlap_shared
             L.moe_permute_fp8(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
-                              self.x8, self.x_s, self.u8 if self.ws13 is not None else None,
-                              self.u_s if self.ws13 is not None else None, self.offsets,
+                              self.x8, self.x_s, self.u8 if own_u8 else None,
+                              self.u_s if own_u8 else None, self.offsets,
                               self.pos, self.src, self.perm_ws, self.perm_ws_bytes)
             return
         L.moe_permute(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
@@ -274,9 +276,14 @@ class MoELayer:
             return
         T = u.shape[0]
         if self.fp8:
+            if self.overlap_shared:
+                # on the side stream: u's codes of its own (the same 1x128
+                # rule as the dispatch's), not waiting for the dispatch
+                L.moe_quant_act_fp8(u, T, self.d, self.u8, self.u_s)
             L.moe_grouped_ffn(self.u8, self.u_s, self.shared_offsets, 1, T, self.d,
                               self.shared_inter, self.ws13, self.ws13_s, self.ws2, self.ws2_s,
-                              L.MOE_FP8_E4M3, self.shared_out, self.ffn_ws, self.ffn_ws_bytes)
+                              L.MOE_FP8_E4M3, self.shared_out, self.shared_ws,
+                              self.shared_ws_bytes)
             return
         L.moe_grouped_ffn(u, None, self.shared_offsets, 1, T, self.d, self.shared_inter, self.ws13,
                           None, self.ws2, None, L.MOE_BF16, self.shared_out, self.shared_ws,
@@ -296,7 +303,7 @@ class MoELayer:
         """h' for the bf16 batch u [T, d] (device), written to `out` ([T, d]
         bf16, device) or to the layer's own output buffer, which is returned.
         train=True (bf16, copy-based dispatch) keeps what backward() needs.
-        The bf16 shared expert depends on u alone: it runs on a side stream
+        The shared expert depends on u alone: it runs on a side stream
         while the current stream routes and dispatches (and, for decode-sized
         groups, runs the routed experts); the current stream waits for it
         before the routed GEMMs (large groups) or before the combine.
@@ -500,6 +507,8 @@ class MoELayer:
         n = (2 if self.route_split else 1) + perm + ffn + 1
         if self.ws13 is not None:
             n += ffn
+            if self.fp8 and self.overlap_shared:
+                n += 1                      # the shared expert's own quantisation of u
         if self.gate_kind == "sigmoid":
             n += 1
         return n

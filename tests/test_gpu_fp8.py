@@ -262,3 +262,19 @@ def test_fp8_v3p_sampled_tokens():
     ref = of.layer_output_fp8(u_s, gidx[tokens], g, qexp, qsh)
     check_close(f64(out)[tokens], ref, max_tol=FP8_MAX_TOL, mean_tol=FP8_MEAN_TOL,
                 what="FP8 V3 prefill (sampled tokens)")
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_fp8_shared_expert_overlapped_matches_in_line(name):
+    """FP8: the shared expert on its side stream, with its own quantisation of
+    u (default), and in line on the codes the dispatch wrote give the same
+    layer output bit for bit: both quantise u by the same 1x128 rule."""
+    cfg = synth.CONFIGS[name]
+    inp, lay, out, gidx = _fp8_layer_check(cfg)
+    assert lay.overlap_shared
+    overlapped = out.clone()
+    lay.overlap_shared = False
+    out2 = lay.forward(inp.u_dev)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    assert torch.equal(out2, overlapped)
