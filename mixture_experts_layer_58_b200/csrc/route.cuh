@@ -209,19 +209,23 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
     }
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     if constexpr (PARTIAL) {
-      // this split's logits of the thread's token, fp32, to the workspace
-      if (have && t < T) {
+      // this split's logits of the thread's token, fp32, to the workspace.
+      // tcgen05.ld is a warp-wide instruction: every lane of the warp runs
+      // it (under the warp-uniform `have`); only the stores check t < T.
+      if (have) {
         float* prow = partial + (static_cast<size_t>(blockIdx.y) * T + t) * n_pad;
         for (int c = 0; c < n_pad; c += 32) {
           uint32_t zr[32];
           tmem_ld_32cols(taddr + c, zr);
           tmem_ld_wait();
+          if (t < T) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            if (c + i < n_pad)
-              *reinterpret_cast<float4*>(prow + c + i) =
-                  make_float4(__uint_as_float(zr[i]), __uint_as_float(zr[i + 1]),
-                              __uint_as_float(zr[i + 2]), __uint_as_float(zr[i + 3]));
+            for (int i = 0; i < 32; i += 4)
+              if (c + i < n_pad)
+                *reinterpret_cast<float4*>(prow + c + i) =
+                    make_float4(__uint_as_float(zr[i]), __uint_as_float(zr[i + 1]),
+                                __uint_as_float(zr[i + 2]), __uint_as_float(zr[i + 3]));
+          }
         }
       }
     } else if (have) {
