@@ -267,7 +267,7 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
 // expert index on equal keys), the winner leaving the candidates -- the same
 // selection and order as route_insert. Gates, idx and the histogram as the
 // fused kernel. Keys that are not finite numbers are never selected.
-constexpr int kSelectWarps = 8;
+constexpr int kSelectWarps = 4;
 template <int TOPK, int KIND>
 __global__ void __launch_bounds__(32 * kSelectWarps)
 route_select_kernel(const float* __restrict__ partial, int splits, const float* __restrict__ bias,
@@ -281,6 +281,30 @@ route_select_kernel(const float* __restrict__ partial, int splits, const float* 
   const int t = blockIdx.x * kSelectWarps + (threadIdx.x >> 5);
   constexpr int kPer = kRouteMaxExperts / 32;
   if (t < T) {
+    // z_j = sum over the splits in ascending order; the loads of four splits
+    // are issued before their adds so that 4 x kPer of them are in flight
+    float zs[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) zs[i] = 0.0f;
+    const float* base = partial + static_cast<size_t>(t) * n_pad + lane;
+    const size_t stride = static_cast<size_t>(T) * n_pad;
+    int y = 0;
+    for (; y + 4 <= splits; y += 4) {
+      float v[4][kPer];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < kPer; ++i)
+          v[q][i] = (lane + 32 * i < n_routed) ? __ldg(base + (y + q) * stride + 32 * i) : 0.0f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) zs[i] += v[q][i];
+    }
+    for (; y < splits; ++y)
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if (lane + 32 * i < n_routed) zs[i] += __ldg(base + y * stride + 32 * i);
     float key[kPer], sval[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
@@ -288,9 +312,7 @@ route_select_kernel(const float* __restrict__ partial, int splits, const float* 
       key[i] = -INFINITY;
       sval[i] = 0.0f;
       if (j < n_routed) {
-        float z = 0.0f;
-        for (int y = 0; y < splits; ++y)
-          z += __ldg(partial + (static_cast<size_t>(y) * T + t) * n_pad + j);
+        const float z = zs[i];
         float sv, kv;
         if constexpr (KIND == 0) {
           sv = 1.0f / (1.0f + expf(-z));
