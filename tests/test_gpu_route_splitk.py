@@ -24,7 +24,9 @@ def _built(cuda_ok):
 
 def _route_both(cfg, T, bias=None):
     """(split-K result, one-pass result, oracle routing) on the workload's first T tokens."""
+    cfg = cfg.replace(T=max(cfg.T, T))          # the draw must hold T rows
     u = synth.tokens(cfg, T)
+    assert u.shape == (T, cfg.d)
     e = synth.centroids(cfg)
     b = synth.bias(cfg) if bias is None else bias
     use_b = b if cfg.gate_kind == "sigmoid" else None
