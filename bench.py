@@ -586,12 +586,14 @@ def main():
     ap.add_argument("--config", default="v3p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--mode", default="five-call",
-                    choices=["five-call", "fused", "scatter", "train"],
+                    choices=["five-call", "fused", "scatter", "scatter-combine", "train"],
                     help="five-call: route, permute (copy), grouped FFN, combine, bias update; "
                          "fused: the up-projection gathers the token rows itself (bf16; measured "
                          "slower: the TMA gathers are request-rate bound); scatter: the "
                          "down-projection applies the gates and writes slot-ordered rows, the "
-                         "combine adds adjacent rows (bf16); train: forward with saved "
+                         "combine adds adjacent rows (bf16); scatter-combine: the same, with the "
+                         "combine in the down-projection's epilogue too (bf16); train: forward "
+                         "with saved "
                          "pre-activations + backward + bias update (bf16)")
     ap.add_argument("--no-overlap", action="store_true",
                     help="run the shared expert after the routed experts on one stream")
@@ -689,6 +691,7 @@ def main():
                        routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind, gamma=cfg.gamma,
                        fp8=cfg.fp8, fused_gather=(args.mode == "fused"),
                        fused_scatter=(args.mode == "scatter"),
+                       fused_combine=(args.mode == "scatter-combine"),
                        overlap_shared=not args.no_overlap, shared_join=args.shared_join,
                        split_route=args.split_route, device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
@@ -805,6 +808,7 @@ def main():
                             "expert-parallel: NCCL all-to-all dispatch/return, rows "
                             "regrouped by expert on the receiving rank" if ep_mode else
                             "fused gather" if lay.fused_gather else
+                            "fused scatter and combine" if lay.fused_combine else
                             "fused scatter" if lay.fused_scatter else "five-call"),
                    "route": ("gate GEMM split over K, then a warp-per-token top-K pass"
                              if lay.route_split else "gate GEMM and top-K in one fused pass"),

@@ -361,6 +361,34 @@ MOE_API int moe_combine_slots(const void* y_slots, const int32_t* pos, const voi
                               const void* residual, int T, int d, int top_k, void* out,
                               moe_stream_t stream);
 
+/* moe_expert_down_scatter_combine: moe_expert_down_scatter followed, inside
+ * the same kernel, by moe_combine_slots: the store that completes a token's
+ * top_k slot rows over a block of 128 output features (a count per token and
+ * block in the workspace) adds them to residual and shared_out and writes
+ * out, with moe_combine_slots' arithmetic (fp32 in the order residual,
+ * shared, slots 0..top_k-1; one bf16 rounding), so the two give the same
+ * bits. y_slots is still written (the rows are read back from it).
+ *   shared_out, residual  [T, d] bf16 or NULL, 16-B aligned; complete before
+ *              the call is ordered on the stream (they are read during it).
+ *   out        [T, d] bf16 out, 16-B aligned; must not alias y_slots.
+ *   workspace  device scratch, 16-B aligned, at least
+ *              moe_expert_down_scatter_combine_workspace_size(T, d) bytes
+ *              (the counts, zeroed by the call); caller-owned. NULL or too
+ *              small -> MOE_ERR_WORKSPACE.
+ * Every (token, slot) pair must have a row (dst_slot covers all T*top_k
+ * slots, as moe_permute + moe_slot_index give): a token with a slot that no
+ * row maps to never completes, and its out row is not written. top_k <=
+ * 8. Other arguments and errors as moe_expert_down_scatter.
+ */
+MOE_API size_t moe_expert_down_scatter_combine_workspace_size(int T, int d);
+MOE_API int moe_expert_down_scatter_combine(const void* h, const int32_t* group_offsets, int G,
+                                            int rows, int inter, int d, const void* w2,
+                                            const int32_t* dst_slot, const float* topk_gate,
+                                            int T, int top_k, void* y_slots,
+                                            const void* shared_out, const void* residual,
+                                            void* out, void* workspace, size_t ws_bytes,
+                                            moe_stream_t stream);
+
 /* ------------------------------------------------------------------ bias update
  * Auxiliary-loss-free balancing (technical report summary, Method §2): at the
  * end of a step, b_i <- b_i - gamma if expert i is overloaded and

@@ -72,6 +72,9 @@ _SIGS = {
     "moe_expert_down_scatter": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _i, _vp,
                                      _vp]),
     "moe_combine_slots": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_expert_down_scatter_combine": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _i,
+                                             _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_down_scatter_combine_workspace_size": (_sz, [_i, _i]),
     "moe_pack_w13": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_strerror": (ctypes.c_char_p, [_i]),
     "moe_last_cuda_error": (_i, []),
@@ -283,6 +286,19 @@ def moe_expert_down_scatter(h, group_offsets, G, rows, inter, d, w2, dst_slot, t
 def moe_combine_slots(y_slots, pos, shared_out, residual, T, d, top_k, out, stream=None):
     _check(_L().moe_combine_slots(_p(y_slots), _p(pos), _p(shared_out), _p(residual), T, d,
                                   top_k, _p(out), _stream(stream)), "moe_combine_slots")
+
+
+def moe_expert_down_scatter_combine_workspace_size(T, d):
+    return _L().moe_expert_down_scatter_combine_workspace_size(T, d)
+
+
+def moe_expert_down_scatter_combine(h, group_offsets, G, rows, inter, d, w2, dst_slot, topk_gate,
+                                    T, top_k, y_slots, shared_out, residual, out, workspace,
+                                    ws_bytes, stream=None):
+    _check(_L().moe_expert_down_scatter_combine(
+        _p(h), _p(group_offsets), G, rows, inter, d, _p(w2), _p(dst_slot), _p(topk_gate), T,
+        top_k, _p(y_slots), _p(shared_out), _p(residual), _p(out), _p(workspace), ws_bytes,
+        _stream(stream)), "moe_expert_down_scatter_combine")
 
 
 def moe_bias_update(expert_counts, bias, n_routed, T, top_k, gamma, stream=None):

@@ -16,6 +16,7 @@
 // the same time share the weight tile through L2. The tile list is rebuilt
 // on the device from group_offsets: no host round trip for the group sizes.
 #pragma once
+#include "dispatch.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -38,7 +39,64 @@ struct ScatterOut {
   const int32_t* slot;
   const float* scale;
   int n_slots;
+  // Fused combine (cnt != nullptr): cnt [T, n_fb] counts, per token and
+  // 128-feature block, the slot rows stored so far (zeroed before the
+  // launch). The store that completes a block's top_k rows adds them in slot
+  // order to residual and shared (either may be null) in fp32, rounds once
+  // and writes the token's output row: the combine's arithmetic, in the
+  // down-projection's epilogue.
+  int32_t* cnt;
+  const __nv_bfloat16* shared;
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* out;
+  int top_k;
+  int n_fb;
 };
+
+// out[t, c .. c+8) of one token whose top_k slot rows are all stored: the
+// combine's order (residual, shared, then the slots), one bf16 rounding. The
+// slot rows come from other SMs: read through L2 (ld.global.cg).
+__device__ __forceinline__ void combine_slots_8(const ScatterOut& sc, const __nv_bfloat16* y,
+                                                int ldo, int t, int c) {
+  const size_t orow = static_cast<size_t>(t) * ldo + c;
+  uint4 yv[kMaxTopK];
+#pragma unroll
+  for (int k = 0; k < kMaxTopK; ++k)
+    if (k < sc.top_k)
+      yv[k] = __ldcg(reinterpret_cast<const uint4*>(
+          y + (static_cast<size_t>(t) * sc.top_k + k) * ldo + c));
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = 0.0f;
+  if (sc.residual) add_bf16x8(a, __ldcg(reinterpret_cast<const uint4*>(sc.residual + orow)));
+  if (sc.shared) add_bf16x8(a, __ldcg(reinterpret_cast<const uint4*>(sc.shared + orow)));
+#pragma unroll
+  for (int k = 0; k < kMaxTopK; ++k)
+    if (k < sc.top_k) add_bf16x8(a, yv[k]);
+  *reinterpret_cast<uint4*>(sc.out + orow) =
+      make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                 pack_bf16x2(a[6], a[7]));
+}
+
+// Fused combine after one thread stored the features [c0, c0 + 8 * nvec) of
+// slot row drow (-1: nothing stored), counter block fb. Called by every lane
+// of the warp. The store is made visible device-wide before the count, and
+// the completing thread reads the other rows only after its count.
+__device__ __forceinline__ void scatter_combine_thread(const ScatterOut& sc,
+                                                       const __nv_bfloat16* y, int ldo,
+                                                       int drow, int c0, int nvec, int fb) {
+  __threadfence();
+  bool last = false;
+  if (drow >= 0) {
+    const int t = drow / sc.top_k;
+    last = atomicAdd(sc.cnt + static_cast<size_t>(t) * sc.n_fb + fb, 1) == sc.top_k - 1;
+  }
+  if (!last) return;
+  __threadfence();
+  const int t = drow / sc.top_k;
+#pragma unroll 1
+  for (int v = 0; v < nvec; ++v) combine_slots_8(sc, y, ldo, t, c0 + 8 * v);
+}
 
 template <int BN>
 struct GemmCfg {
@@ -346,6 +404,13 @@ grouped_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int v = 0; v < 4; ++v)
               dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
+        }
+        if constexpr (EPI == EPI_SCATTER) {
+          // this thread stored the 256 features of one slot row: counter
+          // block 2 * n_blk of its token stands for both 128-feature halves
+          if (sc.cnt != nullptr)
+            scatter_combine_thread(sc, out, ldo, store ? drow : -1, n_blk * BN, BN / 8,
+                                   2 * n_blk);
         }
       }
       tc_fence_before();

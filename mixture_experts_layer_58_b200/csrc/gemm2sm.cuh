@@ -534,12 +534,15 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
               X[i * 128 + quarter * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
           }
           if (!xfer_sync(&xready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
-          __nv_bfloat16* dst0 = out + n_blk * BN + static_cast<int>(rank) * 128;
+          const int fcol = n_blk * BN + static_cast<int>(rank) * 128;
+          __nv_bfloat16* dst0 = out + fcol;
+          int dr[4];   // slot row this lane stored in step k (-1: none)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int idx = et + 128 * k;
             const int r = idx >> 4, seg = idx & 15;
             const int grow = row0 + j0 + r;
+            dr[k] = -1;
             if (grow < row_end) {
               int drow = grow;
               if constexpr (EPI == EPI_SCATTER) {
@@ -548,6 +551,35 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
               }
               *reinterpret_cast<uint4*>(dst0 + static_cast<size_t>(drow) * ldo + seg * 8) =
                   *reinterpret_cast<const uint4*>(X + r * 128 + seg * 8);
+              dr[k] = drow;
+            }
+          }
+          if constexpr (EPI == EPI_SCATTER) {
+            // Fused combine: the 16 lanes of a half-warp stored one row's 128
+            // features (this CTA's block 2 * n_blk + rank) in each step k;
+            // lane 16h + k counts that row, and the half-warp that completes
+            // a token's block writes its output features.
+            if (sc.cnt != nullptr) {
+              __threadfence();
+              __syncwarp();
+              const int kk = lane & 15;
+              int mine = -1;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if (kk == k) mine = dr[k];
+              bool last = false;
+              if (mine >= 0)
+                last = atomicAdd(sc.cnt + static_cast<size_t>(mine / sc.top_k) * sc.n_fb +
+                                     fcol / 128,
+                                 1) == sc.top_k - 1;
+              const unsigned lm = __ballot_sync(0xffffffffu, last);
+              if (lm != 0) {
+                __threadfence();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  if ((lm >> ((lane & 16) + k)) & 1u)
+                    combine_slots_8(sc, out, ldo, dr[k] / sc.top_k, fcol + (lane & 15) * 8);
+              }
             }
           }
         }

@@ -884,6 +884,51 @@ int moe_expert_down_scatter(const void* h, const int32_t* group_offsets, int G, 
                                                d, as_stream(stream), nullptr, sc);
 }
 
+size_t moe_expert_down_scatter_combine_workspace_size(int T, int d) {
+  if (T <= 0 || d <= 0) return 16;
+  const size_t bytes = static_cast<size_t>(T) * ((d + 127) / 128) * sizeof(int32_t);
+  return (bytes + 255) / 256 * 256;
+}
+
+int moe_expert_down_scatter_combine(const void* h, const int32_t* group_offsets, int G, int rows,
+                                    int inter, int d, const void* w2, const int32_t* dst_slot,
+                                    const float* topk_gate, int T, int top_k, void* y_slots,
+                                    const void* shared_out, const void* residual, void* out,
+                                    void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_ffn_shape(G, rows, d, inter);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0 || T == 0) return MOE_OK;
+  if (!h || !group_offsets || !w2 || !dst_slot || !topk_gate || !y_slots || !out ||
+      !aligned16(h) || !aligned16(w2) || !aligned16(y_slots) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if ((shared_out && !aligned16(shared_out)) || (residual && !aligned16(residual)))
+    return MOE_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) ||
+      ws_bytes < moe_expert_down_scatter_combine_workspace_size(T, d))
+    return MOE_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  const int n_fb = d / 128;
+  int32_t* cnt = static_cast<int32_t*>(workspace);
+  MOE_CUDA(cudaMemsetAsync(cnt, 0, static_cast<size_t>(T) * n_fb * sizeof(int32_t), st));
+  const ScatterOut sc{dst_slot,
+                      topk_gate,
+                      T * top_k,
+                      cnt,
+                      static_cast<const __nv_bfloat16*>(shared_out),
+                      static_cast<const __nv_bfloat16*>(residual),
+                      static_cast<__nv_bfloat16*>(out),
+                      top_k,
+                      n_fb};
+  if (use_pair_tiles(rows, G))
+    return launch_grouped_gemm_pair<EPI_SCATTER>(h, rows, inter, w2, G, d, group_offsets,
+                                                 y_slots, d, st, nullptr, 0, nullptr, sc);
+  return launch_grouped_gemm<256, EPI_SCATTER>(h, rows, inter, w2, G, d, group_offsets, y_slots,
+                                               d, st, nullptr, sc);
+}
+
 int moe_combine_slots(const void* y_slots, const int32_t* pos, const void* shared_out,
                       const void* residual, int T, int d, int top_k, void* out,
                       moe_stream_t stream) {

@@ -63,6 +63,7 @@ class MoELayer:
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
                  fp8: bool = False, fused_gather: bool = False, fused_scatter: bool = False,
+                 fused_combine: bool = False,
                  overlap_shared: bool = True, shared_join: str = "auto",
                  split_route: str = "auto", device="cuda"):
         L.load()
@@ -82,7 +83,11 @@ class MoELayer:
         # fused scatter (bf16): the down-projection multiplies each routed row
         # by its gate and writes it to its (token, slot) row; the combine then
         # adds K adjacent rows per token
-        self.fused_scatter = bool(fused_scatter) and not self.fp8
+        self.fused_scatter = (bool(fused_scatter) or bool(fused_combine)) and not self.fp8
+        # fused combine (bf16, implies the fused scatter): the down-projection's
+        # epilogue also adds each token's K slot rows to the residual and the
+        # shared expert once the last of them is stored; no combine launch
+        self.fused_combine = bool(fused_combine) and not self.fp8
         # run the shared expert on a side stream next to the routed path (FP8:
         # with its own quantisation of u, so it does not wait for the dispatch);
         # shared_join: where the current stream waits for it -- "early" (before
@@ -166,6 +171,10 @@ class MoELayer:
         self.src = torch.empty(rows, dtype=i32, device=dev)
         self.dst_slot = (torch.empty(rows, dtype=i32, device=dev) if self.fused_scatter
                          else None)
+        self.comb_ws_bytes = (L.moe_expert_down_scatter_combine_workspace_size(T, d)
+                              if self.fused_combine else 0)
+        self.comb_ws = (torch.empty(self.comb_ws_bytes, dtype=torch.uint8, device=dev)
+                        if self.fused_combine else None)
         self.x_perm = (None if (self.fp8 or self.fused_gather) else
                        torch.empty((rows, d), dtype=torch.bfloat16, device=dev))
         self.y_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
@@ -248,9 +257,16 @@ class MoELayer:
             L.moe_expert_up_swiglu(self.x_perm, self.offsets, self.n_routed, rows, self.d,
                                    self.inter, self.w13, self.ffn_ws)
 
-    def _routed_down(self, T):
+    def _routed_down(self, T, u=None, residual=True, dst=None):
         rows = T * self.top_k
-        if self.fp8:
+        if self.fused_combine:
+            # the shared expert's output must be complete (the caller joins first)
+            L.moe_expert_down_scatter_combine(
+                self.ffn_ws, self.offsets, self.n_routed, rows, self.inter, self.d, self.w2,
+                self.dst_slot, self.topk_gate, T, self.top_k, self.y_perm, self.shared_out,
+                u if residual else None, self.out if dst is None else dst, self.comb_ws,
+                self.comb_ws_bytes)
+        elif self.fp8:
             h8, hs = self._fp8_h()
             L.moe_expert_down_fp8(h8, hs, self.offsets, self.n_routed, rows, self.inter, self.d,
                                   self.w2, self.w2_s, self.y_perm)
@@ -353,6 +369,16 @@ class MoELayer:
                     self._routed_up_train(T)
                 else:
                     self._routed_up(T, u)
+            if self.fused_combine:
+                # the down-projection's epilogue reads the shared expert's output
+                if side is None:
+                    with ev("shared"):
+                        self.shared_ffn(u)
+                elif not join_early:
+                    torch.cuda.current_stream().wait_event(self._join_event)
+                with ev("down"):
+                    self._routed_down(T, u, residual, dst)
+                return dst
             with ev("down"):
                 if train:
                     self._routed_down_train(T)
@@ -504,7 +530,7 @@ class MoELayer:
         perm = 2 if self.fused_gather else 3
         if self.fused_scatter:
             perm += 1                       # the slot index
-        n = (2 if self.route_split else 1) + perm + ffn + 1
+        n = (2 if self.route_split else 1) + perm + ffn + (0 if self.fused_combine else 1)
         if self.ws13 is not None:
             n += ffn
             if self.fp8 and self.overlap_shared:

@@ -23,7 +23,7 @@ class Inputs:
     accessor for the oracle's copy of any expert's weights."""
 
     def __init__(self, cfg: synth.MoEConfig, T: int | None = None, fused_gather: bool = False,
-                 fused_scatter: bool = False):
+                 fused_scatter: bool = False, fused_combine: bool = False):
         from mixture_experts_layer_58_b200.layer import MoELayer
         self.cfg = cfg
         self.u = synth.tokens(cfg, T)
@@ -39,7 +39,7 @@ class Inputs:
         self.layer = MoELayer(self.e, self.b, W1, W3, W2, self.shared, top_k=cfg.top_k,
                               routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
                               gamma=cfg.gamma, fused_gather=fused_gather,
-                              fused_scatter=fused_scatter)
+                              fused_scatter=fused_scatter, fused_combine=fused_combine)
         del W1, W3, W2
         self.u_dev = self.u.cuda()
         self._cache = {}

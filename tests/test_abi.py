@@ -330,3 +330,55 @@ def test_peer_memory_ep_entry_points_reject_bad_arguments(lib):
     assert lib.moe_ipc_get_handle(None, A, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_ipc_open_handle(None, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_ipc_close_handle(None) == L.MOE_ERR_INVALID_ARG
+
+
+def test_fused_combine_entry_point_rejects_bad_arguments(lib):
+    # moe_expert_down_scatter_combine(h, off, G, rows, inter, d, w2, slot, gate, T, K, y,
+    #                                 shared, residual, out, ws, ws_bytes)
+    need = L.moe_expert_down_scatter_combine_workspace_size(16, 256)
+    assert need == 256 and L.moe_expert_down_scatter_combine_workspace_size(16384, 7168) == \
+        16384 * 56 * 4
+    ok = dict(h=A, off=A, G=4, rows=64, inter=128, d=256, w2=A, slot=A, gate=A, T=16, K=4, y=A,
+              sh=None, res=None, out=A, ws=A, wsb=need)
+
+    def dsc(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.moe_expert_down_scatter_combine(
+            a["h"], a["off"], a["G"], a["rows"], a["inter"], a["d"], a["w2"], a["slot"],
+            a["gate"], a["T"], a["K"], a["y"], a["sh"], a["res"], a["out"], a["ws"], a["wsb"],
+            None)
+    assert dsc(d=100) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert dsc(K=9) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert dsc(T=-1) == L.MOE_ERR_INVALID_ARG
+    assert dsc(out=None) == L.MOE_ERR_INVALID_ARG
+    assert dsc(out=MIS) == L.MOE_ERR_INVALID_ARG
+    assert dsc(sh=MIS) == L.MOE_ERR_INVALID_ARG
+    assert dsc(res=MIS) == L.MOE_ERR_INVALID_ARG
+    assert dsc(ws=None) == L.MOE_ERR_WORKSPACE
+    assert dsc(wsb=need - 1) == L.MOE_ERR_WORKSPACE
+    assert dsc(ws=MIS) == L.MOE_ERR_WORKSPACE
+
+
+def test_split_route_entry_point_rejects_bad_arguments(lib):
+    need = L.moe_route_splitk_workspace_size(128, 7168, 256)
+    # 28 slices of K (4 K blocks of 64 each) x 128 tokens x 256 experts, fp32
+    assert need == 28 * 128 * 256 * 4
+    assert L.moe_route_splitk_workspace_size(16384, 7168, 256) == 16384 * 256 * 4   # one slice
+
+    def rs(**kw):
+        a = dict(u=A, c=A, b=None, T=64, d=256, n=16, k=4, kind=0, s=1.0, idx=A, gate=A, cnt=A,
+                 ws=A, wsb=L.moe_route_splitk_workspace_size(64, 256, 16))
+        a.update(kw)
+        return lib.moe_route_splitk(a["u"], a["c"], a["b"], a["T"], a["d"], a["n"], a["k"],
+                                    a["kind"], a["s"], a["idx"], a["gate"], a["cnt"], a["ws"],
+                                    a["wsb"], None)
+    assert rs(T=-1) == L.MOE_ERR_INVALID_ARG
+    assert rs(kind=7) == L.MOE_ERR_INVALID_ARG
+    assert rs(u=MIS) == L.MOE_ERR_INVALID_ARG
+    assert rs(d=200) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rs(n=300) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rs(k=9) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert rs(ws=None) == L.MOE_ERR_WORKSPACE
+    assert rs(wsb=16) == L.MOE_ERR_WORKSPACE
+    assert rs(ws=MIS) == L.MOE_ERR_WORKSPACE

@@ -97,3 +97,68 @@ def test_fused_scatter_without_residual_matches_oracle():
     g = om.gates_for_indices(inp.u, inp.e, gidx, cfg.routed_scale, cfg.gate_kind)
     ref = om.layer_output(inp.u, gidx, g, inp.expert, inp.shared_list(), residual=False)
     check_close(f64(out), ref)
+
+
+# tiny: 1-CTA tiles (one thread stores a row's 256 features and counts them);
+# mid: CTA-pair tiles (a half-warp stores and counts 128 features); T = 383:
+# ragged token chunks and group tails; no shared expert; no residual
+@pytest.mark.parametrize("name,T,residual,kw", [("tiny", None, True, {}),
+                                                ("tiny", 383, True, {}),
+                                                ("tiny", None, True, {"n_shared": 0}),
+                                                ("mid", None, True, {}),
+                                                ("mid", None, False, {})])
+def test_fused_combine_bit_identical_to_scatter_then_combine(name, T, residual, kw):
+    """The combine in the down-projection's epilogue (the store that completes
+    a token's slot rows over a 128-feature block adds them) gives the same
+    bits as moe_combine_slots after the scattering down-projection, and the
+    oracle's layer output."""
+    cfg = synth.CONFIGS[name].replace(**kw)
+    if T is not None:
+        cfg = cfg.replace(T=512)
+    a = Inputs(cfg, T=T, fused_scatter=True)
+    want = _forward(a, residual).clone()
+    b = Inputs(cfg, T=T, fused_combine=True)
+    assert b.layer.fused_combine
+    got = _forward(b, residual)
+    assert torch.equal(got, want)
+    lay = b.layer
+    gidx = lay.topk_idx.cpu().numpy()
+    g = om.gates_for_indices(b.u, b.e, gidx, cfg.routed_scale, cfg.gate_kind)
+    ref = om.layer_output(b.u, gidx, g, b.expert, b.shared_list(), residual=residual)
+    check_close(f64(got), ref)
+    # a second forward on the same buffers (counts re-zeroed by the call)
+    again = _forward(b, residual)
+    assert torch.equal(again, want)
+
+
+def test_fused_combine_v3p_bit_identical():
+    """V3 prefill (CTA-pair tiles, 256 experts, Zipf-skewed groups): the fused
+    combine against the scatter + combine pair on the same inputs."""
+    cfg = synth.CONFIGS["v3p"]
+    a = Inputs(cfg, fused_scatter=True)
+    want = _forward(a).clone()
+    del a
+    torch.cuda.empty_cache()
+    b = Inputs(cfg, fused_combine=True)
+    got = _forward(b)
+    assert torch.equal(got, want)
+
+
+def test_fused_combine_workspace_contract():
+    cfg = synth.CONFIGS["tiny"]
+    inp = Inputs(cfg, fused_combine=True)
+    _forward(inp)
+    lay = inp.layer
+    T, K, d = cfg.T, cfg.top_k, cfg.d
+    need = L.moe_expert_down_scatter_combine_workspace_size(T, d)
+    assert need >= T * (d // 128) * 4 and need % 256 == 0
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    args = (lay.ffn_ws, lay.offsets, cfg.n_routed, T * K, cfg.inter, d, lay.w2, lay.dst_slot,
+            lay.topk_gate, T, K, lay.y_perm, lay.shared_out, inp.u_dev, lay.out)
+    with pytest.raises(L.MoEError) as ex:
+        L.moe_expert_down_scatter_combine(*args, small, small.numel())
+    assert ex.value.status == L.MOE_ERR_WORKSPACE
+    with pytest.raises(L.MoEError) as ex:
+        L.moe_expert_down_scatter_combine(*args, None, 0)
+    assert ex.value.status == L.MOE_ERR_WORKSPACE
+    assert L.moe_get_device_status() == 0
