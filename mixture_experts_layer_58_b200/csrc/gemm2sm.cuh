@@ -19,8 +19,9 @@
 // TMEM: each CTA receives its 128 weight rows (lanes) x N token columns of the
 // accumulator, double-buffered (2 x 256 columns). The epilogue transposes
 // through shared memory: 32 token columns at a time, each warp's 32 lanes are
-// written into a [32 tokens][features] bf16 tile, then the 4 epilogue warps
-// store whole token rows with 16-byte vectors. With W1/W3 interleaved in
+// written into a [32 tokens][features] bf16 tile, then the group of 4
+// epilogue warps (one per TMEM lane quarter) that owns the chunk stores whole
+// token rows with 16-byte vectors. With W1/W3 interleaved in
 // 16-row chunks, lanes l and l+16 of a warp hold the gate and up products of
 // the same h column, paired with one shuffle.
 //
@@ -30,8 +31,8 @@
 //   empty[s]  both CTAs; the leader's MMA commit arrives on its own and on the
 //             peer's (mapa address) when the stage has been read.
 //   tfull[a]  both CTAs; committed like empty at the end of a tile.
-//   tempty[a] leader only; lane 0 of each of the 8 epilogue warps (both CTAs)
-//             arrives once it has drained its TMEM columns (release.cluster).
+//   tempty[a] leader only; lane 0 of each epilogue warp of both CTAs arrives
+//             once it has drained its TMEM columns (release.cluster).
 // Tiles are (group, 256-token block, 256-weight-row block); token columns past
 // the group's end are computed on whatever rows the loads fetched and never
 // stored.
@@ -42,12 +43,18 @@ namespace moe {
 
 constexpr int kStages2 = 6;
 constexpr int kBM2 = 256;        // rows per CTA-pair tile (128 per CTA)
+// Epilogue warps per CTA, in groups of 4 (one warp per TMEM lane quarter);
+// group e drains the 32-column chunks e, e + groups, ... of each tile through
+// its own double-buffered transpose tile.
+constexpr int kPairEpiWarps = 4;
+constexpr int kPairEpiGroups = kPairEpiWarps / 4;
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 
 struct Gemm2smCfg {
   static constexpr int kABytes = 128 * kBK * 2;   // token rows (up to 128 of this CTA's half)
   static constexpr int kBBytes = 128 * kBK * 2;   // this CTA's 128 weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kXBytes = 2 * 32 * 128 * 2;   // epilogue transpose, double-buffered
+  static constexpr int kXBytes = kPairEpiGroups * 2 * 32 * 128 * 2;   // per group, double-buffered
   static constexpr int kBarBytes = 256;
   static size_t smem_bytes(int G) {
     return 1024 + static_cast<size_t>(kStages2) * kStageBytes + kXBytes + kBarBytes +
@@ -173,14 +180,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 
 // Dynamic tile order. The leader's producer takes the next tile index from a
 // global counter (zeroed before the launch) and publishes it, through a ring
-// of kTileQ slots, to the 10 other roles that walk the same tiles: the peer's
-// producer, the leader's MMA thread and the 4 epilogue warps of each CTA.
+// of kTileQ slots, to the other roles that walk the same tiles: the peer's
+// producer, the leader's MMA thread and the epilogue warps of each CTA.
 // Tiles cost different amounts (a group's last tile is a narrower MMA), so a
 // fixed round-robin split would leave some pairs idle while others still work
 // through full tiles; taking tiles in index order also keeps the pairs that
 // share a weight tile close together in time, while it is still in L2.
 constexpr int kTileQ = 4;
-constexpr int kTileQConsumers = 10;
+constexpr int kTileQConsumers = 2 + 2 * kPairEpiWarps;
 
 __device__ __forceinline__ void st_shared_cluster_s32(uint32_t addr, int v) {
   asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -210,7 +217,7 @@ __device__ __forceinline__ bool tile_q_pop(int i, const int* tq, uint64_t* tq_fu
   return true;
 }
 
-// The 4 epilogue warps of a CTA meet between writing and reading a transpose
+// A group of 4 epilogue warps meets between writing and reading a transpose
 // buffer: lane 0 of each arrives once its warp's writes are done (the
 // mbarrier's release/acquire orders them), and every lane waits, bounded.
 __device__ __forceinline__ bool xfer_sync(uint64_t* bar, uint32_t parity, int lane,
@@ -240,7 +247,7 @@ __device__ __forceinline__ void decode_tile_pair(int t, const int* s_tstart, con
 // src_rows[r] of the tensor behind tmA (the token rows of u, read in place
 // of an expert-contiguous copy), fetched four at a time with tile::gather4.
 template <int EPI, bool GATHER>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                               const __grid_constant__ CUtensorMap tmA32,
                               const __grid_constant__ CUtensorMap tmB,
@@ -261,8 +268,8 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* tfull = empty + kStages2;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint64_t* xready = mma_done + 1;   // [2]: the 4 epilogue warps filled sX half i
-  uint64_t* tq_full = xready + 2;    // [kTileQ]
+  uint64_t* xready = mma_done + 1;   // [2 per group]: the group's 4 warps filled its sX half i
+  uint64_t* tq_full = xready + 2 * kPairEpiGroups;   // [kTileQ]
   uint64_t* tq_empty = tq_full + kTileQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kTileQ);
   int* tq = reinterpret_cast<int*>(tmem_slot + 1);   // [kTileQ] tile indices
@@ -284,11 +291,10 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       for (int a = 0; a < 2; ++a) {
         mbar_init(&tfull[a], 1);
-        mbar_init(&tempty[a], 8);
+        mbar_init(&tempty[a], 2 * kPairEpiWarps);
       }
       mbar_init(mma_done, 1);
-      mbar_init(&xready[0], 4);
-      mbar_init(&xready[1], 4);
+      for (int j = 0; j < 2 * kPairEpiGroups; ++j) mbar_init(&xready[j], 4);
       for (int j = 0; j < kTileQ; ++j) {
         mbar_init(&tq_full[j], 1);
         mbar_init(&tq_empty[j], kTileQConsumers);
@@ -447,11 +453,14 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;
-    const int et = (warp - 2) * 32 + lane;   // 0..127 across the 4 epilogue warps
+    const int eg = (warp - 2) >> 2;                 // epilogue group
+    const int et = ((warp - 2) & 3) * 32 + lane;    // 0..127 across the group's 4 warps
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint64_t* gready = xready + 2 * eg;
+    __nv_bfloat16* gX = sX + eg * (2 * 32 * 128);
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-    int chunk = 0;   // running count of 32-column chunks: selects the sX half
+    int chunk = 0;   // running count of this group's 32-column chunks: selects its sX half
     for (int local = 0;; ++local) {
       int t = total_tiles;
       bool got = true;
@@ -472,12 +481,12 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint32_t taddr = tmem_base + acc * BN + lane_addr;
       bool ok = true;
 #pragma unroll 1
-      for (int j0 = 0; j0 < ncols; j0 += 32, ++chunk) {
+      for (int j0 = 32 * eg; j0 < ncols; j0 += 32 * kPairEpiGroups, ++chunk) {
         ok = false;
         uint32_t v[32];
         tmem_ld_32cols(taddr + j0, v);
         tmem_ld_wait();
-        __nv_bfloat16* X = sX + (chunk & 1) * (32 * 128);
+        __nv_bfloat16* X = gX + (chunk & 1) * (32 * 128);
         if constexpr (EPI == EPI_SWIGLU) {
           // lane l < 16: gate product of h column (l & 15) of this warp's 16;
           // lane l + 16: its up product. Lanes < 16 finish tokens 0..15 of the
@@ -506,7 +515,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const float b = __uint_as_float(lo ? other : own);
             X[(i + (lo ? 0 : 16)) * 64 + hc] = __float2bfloat16_rn(silu_f32(a) * b);
           }
-          if (!xfer_sync(&xready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
+          if (!xfer_sync(&gready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
           __nv_bfloat16* dst0 = out + n_blk * 128 + static_cast<int>(rank) * 64;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
@@ -533,7 +542,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int i = 0; i < 32; ++i)
               X[i * 128 + quarter * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
           }
-          if (!xfer_sync(&xready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
+          if (!xfer_sync(&gready[chunk & 1], (chunk >> 1) & 1, lane, status)) break;
           const int fcol = n_blk * BN + static_cast<int>(rank) * 128;
           __nv_bfloat16* dst0 = out + fcol;
           int dr[4];   // slot row this lane stored in step k (-1: none)

@@ -260,14 +260,14 @@ int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int 
   if (src_rows) {
     auto kern = grouped_gemm_bf16_pair_kernel<EPI, true>;
     if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
-    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
+    kern<<<2 * pairs, kPairThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
                                                  static_cast<__nv_bfloat16*>(out), ldo,
                                                  static_cast<__nv_bfloat16*>(ac), src_rows,
                                                  counter, di->status, sc);
   } else {
     auto kern = grouped_gemm_bf16_pair_kernel<EPI, false>;
     if ((rc = set_smem(kern, smem)) != MOE_OK) return rc;
-    kern<<<2 * pairs, kGemmThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
+    kern<<<2 * pairs, kPairThreads, smem, st>>>(tmA, tmA32, tmB, offsets, G, K, n_per_group, rows,
                                                  static_cast<__nv_bfloat16*>(out), ldo,
                                                  static_cast<__nv_bfloat16*>(ac), nullptr,
                                                  counter, di->status, sc);
