@@ -6,9 +6,11 @@
 // CTAs of a cluster share one M = 256 MMA: CTA r (r = 0 leader, 1 peer) loads
 // weight rows [128r, 128r+128) of the tile's 256 and half of its token rows
 // into its own shared memory, the leader issues the MMA, and the hardware reads
-// both halves from both CTAs. Each SM so loads 32 KB per step for the flops of
-// a 128 x 256 x 64 step (a third less crossbar traffic) and the ring holds 6
-// stages.
+// both halves from both CTAs. Each SM so loads 32 KB per 64 of K for the flops
+// of a 128 x 256 x 64 step (a third less crossbar traffic). A ring stage holds
+// two such K atoms (64 KB per CTA, 3 stages): one barrier round trip between
+// the producer and the MMA thread per 128 of K, which measured far cheaper
+// than one per 64 (the MMA thread waits, fences and commits per stage).
 //
 // Why weights as M: a group's rows come in tiles of 256, and its last tile
 // holds 1..256 of them. With tokens as N that tile's MMA is N = its row count
@@ -41,7 +43,11 @@
 
 namespace moe {
 
-constexpr int kStages2 = 6;
+// A ring stage holds kAtoms2 K-atoms of 64 (one 128-byte swizzle row each):
+// the MMA thread issues 4 * kAtoms2 MMAs per full-barrier wait and per
+// commit, so the barrier round trip, not the MMA, is paid once per 128 of K.
+constexpr int kAtoms2 = 2;
+constexpr int kStages2 = 3;
 constexpr int kBM2 = 256;        // rows per CTA-pair tile (128 per CTA)
 // Epilogue warps per CTA, in groups of 4 (one warp per TMEM lane quarter);
 // group e drains the 32-column chunks e, e + groups, ... of each tile through
@@ -51,8 +57,9 @@ constexpr int kPairEpiGroups = kPairEpiWarps / 4;
 constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 
 struct Gemm2smCfg {
-  static constexpr int kABytes = 128 * kBK * 2;   // token rows (up to 128 of this CTA's half)
-  static constexpr int kBBytes = 128 * kBK * 2;   // this CTA's 128 weight rows
+  static constexpr int kAtomBytes = 128 * kBK * 2;   // 128 rows x one 64-wide K atom
+  static constexpr int kABytes = kAtoms2 * kAtomBytes;   // token rows (up to 128, this CTA's half)
+  static constexpr int kBBytes = kAtoms2 * kAtomBytes;   // this CTA's 128 weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kXBytes = kPairEpiGroups * 2 * 32 * 128 * 2;   // per group, double-buffered
   static constexpr int kBarBytes = 256;
@@ -281,7 +288,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int n_blocks_n = n_per_group / BN;
-  const int num_kb = K / kBK;
+  const int num_kb = K / (kBK * kAtoms2);   // ring stages per tile
 
   if (warp == 0) {
     if (lane == 0) {
@@ -355,7 +362,7 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       // rows rounded up to boxes of 32, not a full 128-row box per K step)
       const int nbox = GATHER ? 4 : ((ncols >> 1) + 31) >> 5;
       const uint32_t stage_tx =
-          2u * static_cast<uint32_t>(C::kBBytes + nbox * 32 * 128);
+          2u * kAtoms2 * static_cast<uint32_t>(C::kAtomBytes + nbox * 32 * 128);
       int src[4] = {0, 0, 0, 0};
       if constexpr (GATHER) {
         // rows past the group's end load any row of the group (masked later)
@@ -377,18 +384,23 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         if (rank == 0 && lane == 0) mbar_arrive_expect_tx(&full[stage], stage_tx);
         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-        if constexpr (GATHER) {
-          tma_gather4_pair(sA + stage * C::kABytes + lane * 4 * 128, &tmA, bar, kb * kBK, src[0],
-                           src[1], src[2], src[3]);
-        } else if (nbox == 4) {
-          tma_load_2d_pair(sA + stage * C::kABytes, &tmA, bar, kb * kBK, a_row);
-        } else {
-          // a ragged tail tile: only the token rows it uses, in boxes of 32
-          for (int j = 0; j < nbox; ++j)
-            tma_load_2d_pair(sA + stage * C::kABytes + j * (32 * 128), &tmA32, bar, kb * kBK,
-                             a_row + 32 * j);
+#pragma unroll
+        for (int at = 0; at < kAtoms2; ++at) {
+          const int x = (kb * kAtoms2 + at) * kBK;
+          uint8_t* a_dst = sA + stage * C::kABytes + at * C::kAtomBytes;
+          if constexpr (GATHER) {
+            tma_gather4_pair(a_dst + lane * 4 * 128, &tmA, bar, x, src[0], src[1], src[2],
+                             src[3]);
+          } else if (nbox == 4) {
+            tma_load_2d_pair(a_dst, &tmA, bar, x, a_row);
+          } else {
+            // a ragged tail tile: only the token rows it uses, in boxes of 32
+            for (int j = 0; j < nbox; ++j)
+              tma_load_2d_pair(a_dst + j * (32 * 128), &tmA32, bar, x, a_row + 32 * j);
+          }
+          if (lane == 0)
+            tma_load_2d_pair(sB + stage * C::kBBytes + at * C::kAtomBytes, &tmB, bar, x, b_row);
         }
-        if (lane == 0) tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, bar, kb * kBK, b_row);
         issued |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages2) {
@@ -429,11 +441,16 @@ grouped_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         tc_fence_after();
         // MMA A operand = the weight rows (sB), B operand = the token rows (sA)
-        const uint64_t wdesc = sw128_kmajor_desc(smem_u32(sB + stage * C::kBBytes));
-        const uint64_t xdesc = sw128_kmajor_desc(smem_u32(sA + stage * C::kABytes));
 #pragma unroll
-        for (int k = 0; k < kBK / kUmmaK; ++k)
-          umma_bf16_pair(d_tmem, wdesc + 2u * k, xdesc + 2u * k, idesc, (kb | k) != 0);
+        for (int at = 0; at < kAtoms2; ++at) {
+          const uint64_t wdesc =
+              sw128_kmajor_desc(smem_u32(sB + stage * C::kBBytes + at * C::kAtomBytes));
+          const uint64_t xdesc =
+              sw128_kmajor_desc(smem_u32(sA + stage * C::kABytes + at * C::kAtomBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k)
+            umma_bf16_pair(d_tmem, wdesc + 2u * k, xdesc + 2u * k, idesc, (kb | at | k) != 0);
+        }
         const uint32_t e = smem_u32(&empty[stage]);
         umma_commit_pair(mapa_shared(e, 0));
         umma_commit_pair(mapa_shared(e, 1));

@@ -237,6 +237,7 @@ int launch_grouped_gemm_pair(const void* A, int rows, int K, const void* B, int 
                              cudaStream_t st, const int32_t* src_rows = nullptr,
                              int a_rows = 0, void* ac = nullptr,
                              ScatterOut sc = ScatterOut{nullptr, nullptr, 0}) {
+  if (K % (kBK * kAtoms2) != 0) return MOE_ERR_UNSUPPORTED_SHAPE;   // whole ring stages
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc != MOE_OK) return rc;
