@@ -35,11 +35,15 @@ struct BwdCfg {
   static constexpr int kBBytes = 4 * kBoxBytes;         // 32 KB: 256 N x 64 K
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarBytes = 256;
-  // wgrad epilogue: per epilogue warp two 32 x 32 bf16 buffers for TMA stores
+  // wgrad: its own ring depth, and per epilogue warp kWgOutBufs 32 x 32 bf16
+  // buffers for TMA stores (a chunk waits only for the store issued
+  // kWgOutBufs chunks before it to have read its buffer)
+  static constexpr int kWgStages = 4;
+  static constexpr int kWgOutBufs = 2;
   static constexpr int kOutBufBytes = 32 * 32 * 2;
-  static constexpr int kOutBytes = 4 * 2 * kOutBufBytes;
+  static constexpr int kOutBytes = 4 * kWgOutBufs * kOutBufBytes;
   static size_t wgrad_smem_bytes(int G) {
-    return 1024 + static_cast<size_t>(kStages) * kStageBytes + kOutBytes + kBarBytes +
+    return 1024 + static_cast<size_t>(kWgStages) * kStageBytes + kOutBytes + kBarBytes +
            2 * static_cast<size_t>(G + 1) * sizeof(int);
   }
   static size_t smem_bytes(int G) {
@@ -313,11 +317,11 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * C::kABytes;
-  uint8_t* sOut = sB + kStages * C::kBBytes;
+  uint8_t* sB = smem + C::kWgStages * C::kABytes;
+  uint8_t* sOut = sB + C::kWgStages * C::kBBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::kOutBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint64_t* empty = full + C::kWgStages;
+  uint64_t* tfull = empty + C::kWgStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
   uint64_t* tq_full = mma_done + 1;
@@ -336,7 +340,7 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < C::kWgStages; ++s) {
         mbar_init(&full[s], 1);
         mbar_init(&empty[s], 1);
       }
@@ -399,13 +403,13 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           tma_load_2d(b + j * C::kBoxBytes, &tmB, &full[stage], n_blk * BN + 64 * j, y);
         issued |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages) {
+        if (++stage == C::kWgStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    for (int s = 0; s < kStages; ++s)
+    for (int s = 0; s < C::kWgStages; ++s)
       if (issued & (1u << s))
         mbar_wait(&full[s], (issued_par >> s) & 1u, status, kStatusTimeoutProducer);
   } else if (warp == 1) {
@@ -464,7 +468,7 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
           umma_commit(&empty[stage]);
         }
         __syncwarp();
-        if (++stage == kStages) {
+        if (++stage == C::kWgStages) {
           stage = 0;
           phase ^= 1u;
         }
@@ -489,7 +493,7 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     // 16-B shared store touches fall in 8 different bank groups.
     const int quarter = warp & 3;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    uint8_t* obuf = sOut + (warp - 2) * 2 * C::kOutBufBytes;
+    uint8_t* obuf = sOut + (warp - 2) * C::kWgOutBufs * C::kOutBufBytes;
     const int sw = (lane >> 1) & 3;
     int chunk = 0;
     for (int local = 0;; ++local) {
@@ -526,9 +530,9 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
             pk[i] = empty_group ? 0u
                                 : pack_bf16x2(__uint_as_float(r[h][2 * i]),
                                               __uint_as_float(r[h][2 * i + 1]));
-          uint8_t* buf = obuf + (chunk & 1) * C::kOutBufBytes;
-          // the store issued from this buffer two chunks ago must have read it
-          if (lane == 0) bulk_wait_group_read<1>();
+          uint8_t* buf = obuf + (chunk % C::kWgOutBufs) * C::kOutBufBytes;
+          // the store issued from this buffer kWgOutBufs chunks ago must have read it
+          if (lane == 0) bulk_wait_group_read<C::kWgOutBufs - 1>();
           __syncwarp();
           uint4* row = reinterpret_cast<uint4*>(buf + lane * 64);
 #pragma unroll
