@@ -530,7 +530,8 @@ def variant_line(name, args, dev, local, stream, pk):
     e_host, b_host = synth.centroids(cfg), synth.bias(cfg)
     lay = MoELayer(e_host, b_host, W1, W3, W2, synth.shared_weights(cfg, "cuda"),
                    top_k=cfg.top_k, routed_scale=cfg.routed_scale, gate_kind=cfg.gate_kind,
-                   gamma=cfg.gamma, fp8=cfg.fp8, split_route=args.split_route, device=dev)
+                   gamma=cfg.gamma, fp8=cfg.fp8, split_route=args.split_route,
+                   shared_grouped=args.shared_grouped, device=dev)
     del W1, W3, W2
     torch.cuda.empty_cache()
     u = synth.tokens(cfg).to(dev)
@@ -600,6 +601,10 @@ def main():
     ap.add_argument("--shared-join", default="auto", choices=["auto", "early", "late"],
                     help="where the overlapped shared expert rejoins: before the routed GEMMs "
                          "(early), before the combine (late), or by group size (auto)")
+    ap.add_argument("--shared-grouped", default="auto", choices=["auto", "on", "off"],
+                    help="the shared expert as the last group of the routed grouped GEMMs (on), "
+                         "in its own launches (off), or grouped when the routed groups average "
+                         ">= 256 rows (auto)")
     ap.add_argument("--split-route", default="auto", choices=["auto", "on", "off"],
                     help="gate GEMM split over K with a separate top-K pass (on), in one "
                          "fused pass (off), or split for batches of at most 2048 tokens (auto)")
@@ -693,7 +698,8 @@ def main():
                        fused_scatter=(args.mode == "scatter"),
                        fused_combine=(args.mode == "scatter-combine"),
                        overlap_shared=not args.no_overlap, shared_join=args.shared_join,
-                       split_route=args.split_route, device=dev)
+                       split_route=args.split_route, shared_grouped=args.shared_grouped,
+                       device=dev)
     W_host = None if cfg.weights_on_gpu else (W1, W3, W2)
     del W1, W3, W2
     torch.cuda.empty_cache()
@@ -812,7 +818,10 @@ def main():
                             "fused scatter" if lay.fused_scatter else "five-call"),
                    "route": ("gate GEMM split over K, then a warp-per-token top-K pass"
                              if lay.route_split else "gate GEMM and top-K in one fused pass"),
-                   "shared_expert": (f"side stream, overlapped, joins {lay.shared_join}"
+                   "shared_expert": ("group N_r of the routed grouped GEMMs (its rows "
+                                     "appended by the dispatch)"
+                                     if getattr(lay, "shared_in_grouped", False) else
+                                     f"side stream, overlapped, joins {lay.shared_join}"
                                      if lay.overlap_shared else "after the routed experts"),
                    "parallelism": (f"ep{world}" if ep_mode else
                                    f"dp{world}" if world > 1 else "single"),

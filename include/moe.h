@@ -153,6 +153,29 @@ MOE_API int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* e
 
 MOE_API size_t moe_permute_workspace_size(int T, int n_routed);
 
+/* moe_permute_shared: moe_permute that also copies u's rows once more, to
+ * rows [T*top_k, T*top_k + T) of x_perm, so that the always-on shared expert
+ * (one expert of the routed experts' inter, technical report summary, Method
+ * §2: every token goes through it) runs as group n_routed of the same grouped
+ * GEMMs as the routed experts: weights [n_routed + 1, ...] with the shared
+ * expert last, and
+ *   x_perm          [T*top_k + T, d] bf16 out, 16-B aligned.
+ *   expert_offsets  [n_routed + 2] int32 out: entries 0..n_routed as
+ *                   moe_permute; entry n_routed + 1 = T*top_k + T. The shared
+ *                   group is [expert_offsets[n_routed], T*top_k + T): it starts
+ *                   where the routed rows end, which is T*top_k unless routed
+ *                   slots were skipped (topk_idx outside [0, n_routed)); the
+ *                   rows in between are not written here, get computed by the
+ *                   shared expert and are read by nothing.
+ * After the down-projection of the n_routed + 1 groups, rows [T*top_k,
+ * T*top_k + T) of its output are the shared expert's output for tokens 0..T-1
+ * (moe_combine's shared_out). Other arguments and errors as moe_permute. */
+MOE_API int moe_permute_shared(const void* u, const int32_t* topk_idx,
+                               const int32_t* expert_counts, int T, int d, int n_routed,
+                               int top_k, void* x_perm, int32_t* expert_offsets, int32_t* pos,
+                               int32_t* src_token, void* workspace, size_t ws_bytes,
+                               moe_stream_t stream);
+
 /* moe_permute_index: the index half of moe_permute (expert_offsets, pos,
  * src_token, same definitions and arguments) without copying any row. For
  * the fused mode, where the up-projection gathers the token rows itself

@@ -50,6 +50,7 @@ _SIGS = {
     "moe_route_splitk_workspace_size": (_sz, [_i, _i, _i]),
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i]),
+    "moe_permute_shared": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
     "moe_permute_index": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_up_swiglu_gather": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
@@ -174,6 +175,13 @@ def moe_permute(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm, exper
     _check(_L().moe_permute(_p(u), _p(topk_idx), _p(expert_counts), T, d, n_routed, top_k,
                             _p(x_perm), _p(expert_offsets), _p(pos), _p(src_token),
                             _p(workspace), ws_bytes, _stream(stream)), "moe_permute")
+
+
+def moe_permute_shared(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm, expert_offsets,
+                       pos, src_token, workspace, ws_bytes, stream=None):
+    _check(_L().moe_permute_shared(_p(u), _p(topk_idx), _p(expert_counts), T, d, n_routed, top_k,
+                                   _p(x_perm), _p(expert_offsets), _p(pos), _p(src_token),
+                                   _p(workspace), ws_bytes, _stream(stream)), "moe_permute_shared")
 
 
 def moe_permute_noalloc(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm,

@@ -125,10 +125,12 @@ permute_index_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict_
 }
 
 // Pass 3: one warp per token reads its row once (16-byte vectors) and writes
-// it to each of its K rows of x_perm.
-__global__ void __launch_bounds__(256)
-permute_copy_kernel(const __nv_bfloat16* __restrict__ u, const int32_t* __restrict__ pos, int T,
-                    int d, int K, __nv_bfloat16* __restrict__ x_perm) {
+// it to each of its K rows of x_perm; TAIL: also to row T*K + t (the rows of
+// the shared expert when it runs as the last group of the routed GEMMs).
+template <bool TAIL>
+__device__ __forceinline__ void permute_copy_rows(const __nv_bfloat16* __restrict__ u,
+                                                  const int32_t* __restrict__ pos, int T, int d,
+                                                  int K, __nv_bfloat16* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const long long total = static_cast<long long>(T) * K;
@@ -159,8 +161,35 @@ permute_copy_kernel(const __nv_bfloat16* __restrict__ u, const int32_t* __restri
           if (v < nvec) drow[v] = x[j];
         }
       }
+      if constexpr (TAIL) {
+        uint4* drow = reinterpret_cast<uint4*>(x_perm + (total + t) * d);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int v = v0 + 32 * j;
+          if (v < nvec) drow[v] = x[j];
+        }
+      }
     }
   }
+}
+
+__global__ void __launch_bounds__(256)
+permute_copy_kernel(const __nv_bfloat16* __restrict__ u, const int32_t* __restrict__ pos, int T,
+                    int d, int K, __nv_bfloat16* __restrict__ x_perm) {
+  permute_copy_rows<false>(u, pos, T, d, K, x_perm);
+}
+
+// The copy with the shared expert's rows appended, and the end of its group:
+// expert_offsets[n_routed + 1] = T*K + T. The shared group starts where the
+// routed rows end (expert_offsets[n_routed], T*K unless routed slots were
+// skipped; rows in between are computed and never read).
+__global__ void __launch_bounds__(256)
+permute_copy_tail_kernel(const __nv_bfloat16* __restrict__ u, const int32_t* __restrict__ pos,
+                         int T, int d, int K, __nv_bfloat16* __restrict__ x_perm,
+                         int32_t* __restrict__ expert_offsets, int n_routed) {
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    expert_offsets[n_routed + 1] = static_cast<int32_t>(static_cast<long long>(T) * K + T);
+  permute_copy_rows<true>(u, pos, T, d, K, x_perm);
 }
 
 // ---------------------------------------------------------------- combine

@@ -557,17 +557,22 @@ size_t moe_permute_workspace_size(int T, int n_routed) {
   return (chunks * n_routed * sizeof(int32_t) + 255) / 256 * 256;
 }
 
-int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* expert_counts, int T, int d,
-                int n_routed, int top_k, void* x_perm, int32_t* expert_offsets, int32_t* pos,
-                int32_t* src_token, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+namespace {
+// moe_permute, and with `tail` the shared expert's rows appended after the
+// routed ones (moe_permute_shared).
+int permute_impl(const void* u, const int32_t* topk_idx, const int32_t* expert_counts, int T,
+                 int d, int n_routed, int top_k, void* x_perm, int32_t* expert_offsets,
+                 int32_t* pos, int32_t* src_token, void* workspace, size_t ws_bytes,
+                 cudaStream_t st, bool tail) {
   if (T < 0 || d <= 0 || n_routed <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
   if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
   if (top_k > kMaxTopK || top_k > n_routed || n_routed > kRouteMaxExperts || d % 256 != 0)
     return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (static_cast<long long>(T) * top_k > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
-  cudaStream_t st = as_stream(stream);
+  if (static_cast<long long>(T) * (top_k + (tail ? 1 : 0)) > INT32_MAX)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) {
-    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (n_routed + 1), st));
+    MOE_CUDA(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (n_routed + (tail ? 2 : 1)),
+                             st));
     return MOE_OK;
   }
   if (!u || !topk_idx || !x_perm || !pos || !src_token || !aligned16(u) || !aligned16(x_perm))
@@ -585,10 +590,31 @@ int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* expert_co
                                                expert_offsets, pos, src_token);
   MOE_CUDA(cudaGetLastError());
   const int blocks = std::max(1, std::min((T + 7) / 8, di->num_sms * 8));
-  permute_copy_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(u), pos, T, d,
-                                              top_k, static_cast<__nv_bfloat16*>(x_perm));
+  if (tail)
+    permute_copy_tail_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(u), pos, T,
+                                                     d, top_k, static_cast<__nv_bfloat16*>(x_perm),
+                                                     expert_offsets, n_routed);
+  else
+    permute_copy_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(u), pos, T, d,
+                                                top_k, static_cast<__nv_bfloat16*>(x_perm));
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
+}
+}  // namespace
+
+int moe_permute(const void* u, const int32_t* topk_idx, const int32_t* expert_counts, int T, int d,
+                int n_routed, int top_k, void* x_perm, int32_t* expert_offsets, int32_t* pos,
+                int32_t* src_token, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  return permute_impl(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm, expert_offsets,
+                      pos, src_token, workspace, ws_bytes, as_stream(stream), false);
+}
+
+int moe_permute_shared(const void* u, const int32_t* topk_idx, const int32_t* expert_counts,
+                       int T, int d, int n_routed, int top_k, void* x_perm,
+                       int32_t* expert_offsets, int32_t* pos, int32_t* src_token,
+                       void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  return permute_impl(u, topk_idx, expert_counts, T, d, n_routed, top_k, x_perm, expert_offsets,
+                      pos, src_token, workspace, ws_bytes, as_stream(stream), true);
 }
 
 int moe_permute_index(const int32_t* topk_idx, const int32_t* expert_counts, int T,

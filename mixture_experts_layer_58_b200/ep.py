@@ -113,6 +113,8 @@ class ExpertParallelMoELayer(MoELayer):
     rank's layer without a process group (the ranks then exchange through the
     caller's own transport between the stage methods)."""
 
+    _merge_shared = False   # the shared expert stays in its own launches
+
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
                  group=None, world: int | None = None, rank: int | None = None,
@@ -311,6 +313,8 @@ class PeerExpertParallelMoELayer(MoELayer):
     caller links them with link_emulated_ranks and drives the stages (begin,
     plan, dispatch, experts, finish) in rank order, which needs no kernel to
     wait on another."""
+
+    _merge_shared = False   # the shared expert stays in its own launches
 
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,

@@ -60,12 +60,16 @@ class MoELayer:
     bias [N_r] fp32 (the layer keeps its own device copy, updated in place).
     """
 
+    # whether the shared expert may run as a group of the routed GEMMs
+    # (subclasses with their own exchange of routed rows keep it apart)
+    _merge_shared = True
+
     def __init__(self, centroids, bias, w1, w3, w2, shared=None, *, top_k: int,
                  routed_scale: float, gate_kind: str = "sigmoid", gamma: float = 0.001,
                  fp8: bool = False, fused_gather: bool = False, fused_scatter: bool = False,
                  fused_combine: bool = False,
                  overlap_shared: bool = True, shared_join: str = "auto",
-                 split_route: str = "auto", device="cuda"):
+                 split_route: str = "auto", shared_grouped: str = "auto", device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -103,18 +107,47 @@ class MoELayer:
         if split_route not in ("auto", "on", "off"):
             raise ValueError("split_route must be 'auto', 'on' or 'off'")
         self.split_route = split_route
+        # shared_grouped: the shared expert as the last group of the routed
+        # grouped GEMMs (bf16 five-call form, one shared expert of the routed
+        # experts' inter): "on", "off" or "auto" (on when the routed groups
+        # average >= 256 rows, where the GEMMs are compute-bound)
+        if shared_grouped not in ("auto", "on", "off"):
+            raise ValueError("shared_grouped must be 'auto', 'on' or 'off'")
+        self.shared_grouped = shared_grouped
         self.centroids = centroids.to(dev, bf).contiguous()
         self.bias = (bias.to(dev, torch.float32).contiguous() if bias is not None
                      else torch.zeros(self.n_routed, dtype=torch.float32, device=dev))
         pack = self.pack_w13_fp8 if self.fp8 else self.pack_w13
-        self.w13 = pack(w1.to(dev, bf).contiguous(), w3.to(dev, bf).contiguous())
-        self.w2 = w2.to(dev, bf).contiguous()
+        # the shared expert can join the routed grouped GEMMs as group N_r when
+        # it has the routed experts' shape: then both live in one weight array
+        # (routed experts first), and self.w13 / self.ws13 are views of it
+        self.mergeable = (self._merge_shared and shared is not None and not self.fp8 and
+                          not self.fused_gather and not self.fused_scatter and
+                          shared[0].shape[0] == self.inter)
+        if self.mergeable:
+            ws1, ws3, ws2 = shared
+            G, I = self.n_routed, self.inter
+            self.w13_all = torch.empty((G + 1, 2 * I, self.d), dtype=bf, device=dev)
+            L.moe_pack_w13(w1.to(dev, bf).contiguous(), w3.to(dev, bf).contiguous(), G, I, self.d,
+                           self.w13_all)
+            L.moe_pack_w13(ws1.to(dev, bf).contiguous()[None], ws3.to(dev, bf).contiguous()[None],
+                           1, I, self.d, self.w13_all[G:])
+            self.w2_all = torch.empty((G + 1, self.d, I), dtype=bf, device=dev)
+            self.w2_all[:G].copy_(w2)
+            self.w2_all[G].copy_(ws2)
+            self.w13, self.ws13 = self.w13_all[:G], self.w13_all[G:]
+            self.w2, self.ws2 = self.w2_all[:G], self.w2_all[G]
+            self.shared_inter = I
+            shared = None                               # weights placed
+        else:
+            self.w13 = pack(w1.to(dev, bf).contiguous(), w3.to(dev, bf).contiguous())
+            self.w2 = w2.to(dev, bf).contiguous()
         if shared is not None:
             ws1, ws3, ws2 = shared
             self.shared_inter = ws1.shape[0]
             self.ws13 = pack(ws1.to(dev, bf).contiguous()[None], ws3.to(dev, bf).contiguous()[None])
             self.ws2 = ws2.to(dev, bf).contiguous()
-        else:
+        elif not self.mergeable:
             self.shared_inter = 0
             self.ws13 = self.ws2 = None
         if self.fp8:
@@ -127,6 +160,8 @@ class MoELayer:
                 self.ws2, self.ws2_s = self.quant_weights(self.ws2[None])
         self._T = -1
         self.route_split = False
+        self.shared_in_grouped = False
+        self._grouped = False
 
     # ------------------------------------------------------------------ setup
     def pack_w13(self, w1, w3):
@@ -163,10 +198,16 @@ class MoELayer:
         dev, K, d = self.device, self.top_k, self.d
         rows = T * K
         i32 = torch.int32
+        # the shared expert as group N_r of the routed GEMMs: T more rows
+        self.shared_in_grouped = self.mergeable and (
+            self.shared_grouped == "on" or
+            (self.shared_grouped == "auto" and rows >= 256 * self.n_routed))
+        rows_all = rows + (T if self.shared_in_grouped else 0)
         self.topk_idx = torch.empty((T, K), dtype=i32, device=dev)
         self.topk_gate = torch.empty((T, K), dtype=torch.float32, device=dev)
         self.counts = torch.empty(self.n_routed, dtype=i32, device=dev)
-        self.offsets = torch.empty(self.n_routed + 1, dtype=i32, device=dev)
+        self.offsets = torch.empty(self.n_routed + (2 if self.shared_in_grouped else 1), dtype=i32,
+                                   device=dev)
         self.pos = torch.empty((T, K), dtype=i32, device=dev)
         self.src = torch.empty(rows, dtype=i32, device=dev)
         self.dst_slot = (torch.empty(rows, dtype=i32, device=dev) if self.fused_scatter
@@ -176,8 +217,8 @@ class MoELayer:
         self.comb_ws = (torch.empty(self.comb_ws_bytes, dtype=torch.uint8, device=dev)
                         if self.fused_combine else None)
         self.x_perm = (None if (self.fp8 or self.fused_gather) else
-                       torch.empty((rows, d), dtype=torch.bfloat16, device=dev))
-        self.y_perm = torch.empty((rows, d), dtype=torch.bfloat16, device=dev)
+                       torch.empty((rows_all, d), dtype=torch.bfloat16, device=dev))
+        self.y_perm = torch.empty((rows_all, d), dtype=torch.bfloat16, device=dev)
         self.route_split = (self.split_route == "on" or
                             (self.split_route == "auto" and T <= 2048))
         self.route_ws_bytes = (L.moe_route_splitk_workspace_size(T, d, self.n_routed)
@@ -187,7 +228,7 @@ class MoELayer:
         self.perm_ws_bytes = L.moe_permute_workspace_size(T, self.n_routed)
         self.perm_ws = torch.empty(self.perm_ws_bytes, dtype=torch.uint8, device=dev)
         dt = L.MOE_FP8_E4M3 if self.fp8 else L.MOE_BF16
-        ffn_ws = max(L.moe_grouped_ffn_workspace_size(rows, self.inter, dt),
+        ffn_ws = max(L.moe_grouped_ffn_workspace_size(rows_all, self.inter, dt),
                      L.moe_grouped_ffn_workspace_size(T, max(self.shared_inter, 128), dt))
         if self.fp8:
             u8 = torch.uint8
@@ -197,8 +238,11 @@ class MoELayer:
             self.x_s = torch.empty((rows, d // 128), dtype=torch.float32, device=dev)
         self.ffn_ws_bytes = ffn_ws
         self.ffn_ws = torch.empty(ffn_ws, dtype=torch.uint8, device=dev)
-        self.shared_out = (torch.empty((T, d), dtype=torch.bfloat16, device=dev)
-                           if self.ws13 is not None else None)
+        if self.shared_in_grouped:
+            self.shared_out = self.y_perm[rows:]        # rows of group N_r
+        else:
+            self.shared_out = (torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+                               if self.ws13 is not None else None)
         # the shared expert runs on a side stream next to the routed path
         # (bf16), so it gets its own workspace
         self.shared_ws_bytes = L.moe_grouped_ffn_workspace_size(T, max(self.shared_inter, 128), dt)
@@ -238,6 +282,12 @@ class MoELayer:
                               self.u_s if own_u8 else None, self.offsets,
                               self.pos, self.src, self.perm_ws, self.perm_ws_bytes)
             return
+        if self._grouped:
+            # u's rows once more after the routed rows: the shared expert's group
+            L.moe_permute_shared(u, self.topk_idx, self.counts, T, self.d, self.n_routed,
+                                 self.top_k, self.x_perm, self.offsets, self.pos, self.src,
+                                 self.perm_ws, self.perm_ws_bytes)
+            return
         L.moe_permute(u, self.topk_idx, self.counts, T, self.d, self.n_routed, self.top_k,
                       self.x_perm, self.offsets, self.pos, self.src, self.perm_ws,
                       self.perm_ws_bytes)
@@ -253,6 +303,10 @@ class MoELayer:
             h8, hs = self._fp8_h()
             L.moe_expert_up_swiglu_fp8(self.x8, self.x_s, self.offsets, self.n_routed, rows,
                                        self.d, self.inter, self.w13, self.w13_s, h8, hs)
+        elif self._grouped:
+            # routed experts and the shared expert (group N_r) in one launch
+            L.moe_expert_up_swiglu(self.x_perm, self.offsets, self.n_routed + 1, rows + T, self.d,
+                                   self.inter, self.w13_all, self.ffn_ws)
         else:
             L.moe_expert_up_swiglu(self.x_perm, self.offsets, self.n_routed, rows, self.d,
                                    self.inter, self.w13, self.ffn_ws)
@@ -275,6 +329,10 @@ class MoELayer:
             L.moe_expert_down_scatter(self.ffn_ws, self.offsets, self.n_routed, rows, self.inter,
                                       self.d, self.w2, self.dst_slot, self.topk_gate, T,
                                       self.top_k, self.y_perm)
+        elif self._grouped:
+            # the shared expert's output lands in rows [T*K, T*K + T) = shared_out
+            L.moe_expert_down(self.ffn_ws, self.offsets, self.n_routed + 1, rows + T, self.inter,
+                              self.d, self.w2_all, self.y_perm)
         else:
             L.moe_expert_down(self.ffn_ws, self.offsets, self.n_routed, rows, self.inter, self.d,
                               self.w2, self.y_perm)
@@ -337,9 +395,11 @@ class MoELayer:
                                  "and the plain combine")
             self._allocate_train(T)
         self._train_state = (u, residual) if train else None
+        # the shared expert as group N_r of the routed GEMMs (not in training)
+        self._grouped = self.shared_in_grouped and not train
         ev = _Timed(timers)
         side = None
-        if T > 0 and self.ws13 is not None and self.overlap_shared:
+        if T > 0 and self.ws13 is not None and self.overlap_shared and not self._grouped:
             side = self._fork()
             u.record_stream(side)
             with torch.cuda.stream(side):
@@ -384,7 +444,7 @@ class MoELayer:
                     self._routed_down_train(T)
                 else:
                     self._routed_down(T)
-            if side is None:
+            if side is None and not self._grouped:
                 with ev("shared"):
                     self.shared_ffn(u)
             elif not join_early:
@@ -531,7 +591,7 @@ class MoELayer:
         if self.fused_scatter:
             perm += 1                       # the slot index
         n = (2 if self.route_split else 1) + perm + ffn + (0 if self.fused_combine else 1)
-        if self.ws13 is not None:
+        if self.ws13 is not None and not getattr(self, "shared_in_grouped", False):
             n += ffn
             if self.fp8 and self.overlap_shared:
                 n += 1                      # the shared expert's own quantisation of u

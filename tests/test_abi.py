@@ -382,3 +382,19 @@ def test_split_route_entry_point_rejects_bad_arguments(lib):
     assert rs(ws=None) == L.MOE_ERR_WORKSPACE
     assert rs(wsb=16) == L.MOE_ERR_WORKSPACE
     assert rs(ws=MIS) == L.MOE_ERR_WORKSPACE
+
+
+def test_permute_shared_rejects_bad_arguments(lib):
+    def ps(**kw):
+        a = dict(u=A, idx=A, cnt=A, T=64, d=256, n=16, k=4, x=A, off=A, pos=A, src=A, ws=A,
+                 wsb=L.moe_permute_workspace_size(64, 16))
+        a.update(kw)
+        return lib.moe_permute_shared(a["u"], a["idx"], a["cnt"], a["T"], a["d"], a["n"], a["k"],
+                                      a["x"], a["off"], a["pos"], a["src"], a["ws"], a["wsb"],
+                                      None)
+    assert ps(T=-1) == L.MOE_ERR_INVALID_ARG
+    assert ps(off=None) == L.MOE_ERR_INVALID_ARG
+    assert ps(d=100) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert ps(k=9) == L.MOE_ERR_UNSUPPORTED_SHAPE
+    assert ps(x=MIS) == L.MOE_ERR_INVALID_ARG
+    assert ps(ws=None) == L.MOE_ERR_WORKSPACE

@@ -328,3 +328,22 @@ def test_shared_expert_in_line_matches_overlapped(name):
     lay.overlap_shared = False
     _full_check(inp)
     assert torch.equal(lay.out, overlapped)
+
+
+@pytest.mark.parametrize("name,T", [("tiny", None), ("tiny", 383)])
+def test_shared_expert_as_a_routed_group_bit_identical(name, T):
+    """The shared expert as group N_r of the routed grouped GEMMs (its rows
+    appended by moe_permute_shared) gives the same layer output bit for bit
+    as its own G = 1 launches, and matches the oracle. Tiny runs the 1-CTA
+    tiles; the V3 prefill test covers the CTA-pair tiles."""
+    cfg = synth.CONFIGS[name] if T is None else synth.CONFIGS[name].replace(T=512)
+    a = Inputs(cfg, T=T)
+    a.layer.shared_grouped = "off"
+    want = _run_forward(a).clone()
+    b = Inputs(cfg, T=T)
+    b.layer.shared_grouped = "on"
+    assert b.layer.mergeable
+    got = _run_forward(b)
+    assert b.layer.shared_in_grouped
+    assert torch.equal(got, want)
+    _full_check(b)

@@ -21,6 +21,10 @@ def _dispatch_invariants(lay, T, K, n_routed):
     off = lay.offsets.cpu().numpy().astype(np.int64)
     pos = lay.pos.cpu().numpy().astype(np.int64)
     src = lay.src.cpu().numpy().astype(np.int64)
+    if off.size == n_routed + 2:
+        # the shared expert as group n_routed: its rows follow the routed ones
+        assert off[-1] == T * K + T
+        off = off[:-1]
     assert np.array_equal(off, np.concatenate([[0], np.cumsum(counts)]))
     assert np.array_equal(np.sort(pos.ravel()), np.arange(T * K))
     t_of = np.repeat(np.arange(T), K)
@@ -83,6 +87,11 @@ def test_v3p_dispatch_all_rows(v3p):
     rows = rng.choice(cfg.T * cfg.top_k, size=2048, replace=False)
     xp = lay.x_perm[torch.from_numpy(rows).cuda()].cpu()
     assert torch.equal(xp, v3p.u[torch.from_numpy(src[rows])])
+    # the benchmark's configuration runs the shared expert as group N_r: its
+    # rows are u's rows, after the routed ones
+    assert lay.shared_in_grouped
+    rk = cfg.T * cfg.top_k
+    assert torch.equal(lay.x_perm[rk:].cpu(), v3p.u)
 
 
 def test_v3p_hottest_expert_rows_incl_ragged_tail(v3p):
@@ -146,3 +155,20 @@ def test_v3p_fused_gather_sampled(cuda_ok):
     _check_sampled_output(inp, lay, tokens)
     del inp
     torch.cuda.empty_cache()
+
+
+def test_v3p_shared_expert_grouped_bit_identical(v3p):
+    """CTA-pair tiles: the benchmark's layer (shared expert as group N_r)
+    against the same layer with the shared expert in its own launches."""
+    lay = v3p.layer
+    assert lay.shared_in_grouped
+    want = lay.out.clone()
+    lay.shared_grouped = "off"
+    lay._T = -1                                   # re-allocate in the separate form
+    got = lay.forward(v3p.u_dev)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    assert not lay.shared_in_grouped
+    assert torch.equal(got, want)
+    lay.shared_grouped = "auto"
+    lay._T = -1
