@@ -444,9 +444,10 @@ class MoELayer:
                     self._routed_down_train(T)
                 else:
                     self._routed_down(T)
-            if side is None and not self._grouped:
-                with ev("shared"):
-                    self.shared_ffn(u)
+            if side is None:
+                if not self._grouped:                   # (grouped: already in y_perm)
+                    with ev("shared"):
+                        self.shared_ffn(u)
             elif not join_early:
                 torch.cuda.current_stream().wait_event(self._join_event)
             with ev("combine"):
