@@ -601,10 +601,9 @@ def main():
     ap.add_argument("--shared-join", default="auto", choices=["auto", "early", "late"],
                     help="where the overlapped shared expert rejoins: before the routed GEMMs "
                          "(early), before the combine (late), or by group size (auto)")
-    ap.add_argument("--shared-grouped", default="auto", choices=["auto", "on", "off"],
-                    help="the shared expert as the last group of the routed grouped GEMMs (on), "
-                         "in its own launches (off), or grouped when the routed groups average "
-                         ">= 256 rows (auto)")
+    ap.add_argument("--shared-grouped", action="store_true",
+                    help="the shared expert as the last group of the routed grouped GEMMs "
+                         "instead of its own launches beside the route and dispatch")
     ap.add_argument("--split-route", default="auto", choices=["auto", "on", "off"],
                     help="gate GEMM split over K with a separate top-K pass (on), in one "
                          "fused pass (off), or split for batches of at most 2048 tokens (auto)")

@@ -69,7 +69,7 @@ class MoELayer:
                  fp8: bool = False, fused_gather: bool = False, fused_scatter: bool = False,
                  fused_combine: bool = False,
                  overlap_shared: bool = True, shared_join: str = "auto",
-                 split_route: str = "auto", shared_grouped: str = "auto", device="cuda"):
+                 split_route: str = "auto", shared_grouped: bool = False, device="cuda"):
         L.load()
         dev = torch.device(device)
         self.device = dev
@@ -109,11 +109,10 @@ class MoELayer:
         self.split_route = split_route
         # shared_grouped: the shared expert as the last group of the routed
         # grouped GEMMs (bf16 five-call form, one shared expert of the routed
-        # experts' inter): "on", "off" or "auto" (on when the routed groups
-        # average >= 256 rows, where the GEMMs are compute-bound)
-        if shared_grouped not in ("auto", "on", "off"):
-            raise ValueError("shared_grouped must be 'auto', 'on' or 'off'")
-        self.shared_grouped = shared_grouped
+        # experts' inter) instead of its own launches beside the route and
+        # dispatch; measured slower at V3 prefill (the overlap is worth more
+        # than the extra launches cost), so off by default
+        self.shared_grouped = bool(shared_grouped)
         self.centroids = centroids.to(dev, bf).contiguous()
         self.bias = (bias.to(dev, torch.float32).contiguous() if bias is not None
                      else torch.zeros(self.n_routed, dtype=torch.float32, device=dev))
@@ -199,9 +198,7 @@ class MoELayer:
         rows = T * K
         i32 = torch.int32
         # the shared expert as group N_r of the routed GEMMs: T more rows
-        self.shared_in_grouped = self.mergeable and (
-            self.shared_grouped == "on" or
-            (self.shared_grouped == "auto" and rows >= 256 * self.n_routed))
+        self.shared_in_grouped = self.mergeable and self.shared_grouped
         rows_all = rows + (T if self.shared_in_grouped else 0)
         self.topk_idx = torch.empty((T, K), dtype=i32, device=dev)
         self.topk_gate = torch.empty((T, K), dtype=torch.float32, device=dev)

@@ -338,10 +338,10 @@ def test_shared_expert_as_a_routed_group_bit_identical(name, T):
     tiles; the V3 prefill test covers the CTA-pair tiles."""
     cfg = synth.CONFIGS[name] if T is None else synth.CONFIGS[name].replace(T=512)
     a = Inputs(cfg, T=T)
-    a.layer.shared_grouped = "off"
+    a.layer.shared_grouped = False
     want = _run_forward(a).clone()
     b = Inputs(cfg, T=T)
-    b.layer.shared_grouped = "on"
+    b.layer.shared_grouped = True
     assert b.layer.mergeable
     got = _run_forward(b)
     assert b.layer.shared_in_grouped

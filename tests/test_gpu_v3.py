@@ -87,11 +87,6 @@ def test_v3p_dispatch_all_rows(v3p):
     rows = rng.choice(cfg.T * cfg.top_k, size=2048, replace=False)
     xp = lay.x_perm[torch.from_numpy(rows).cuda()].cpu()
     assert torch.equal(xp, v3p.u[torch.from_numpy(src[rows])])
-    # the benchmark's configuration runs the shared expert as group N_r: its
-    # rows are u's rows, after the routed ones
-    assert lay.shared_in_grouped
-    rk = cfg.T * cfg.top_k
-    assert torch.equal(lay.x_perm[rk:].cpu(), v3p.u)
 
 
 def test_v3p_hottest_expert_rows_incl_ragged_tail(v3p):
@@ -158,17 +153,21 @@ def test_v3p_fused_gather_sampled(cuda_ok):
 
 
 def test_v3p_shared_expert_grouped_bit_identical(v3p):
-    """CTA-pair tiles: the benchmark's layer (shared expert as group N_r)
-    against the same layer with the shared expert in its own launches."""
-    lay = v3p.layer
-    assert lay.shared_in_grouped
+    """CTA-pair tiles: the shared expert as group N_r of the routed GEMMs (its
+    rows appended by moe_permute_shared) against the benchmark's layer, where
+    it runs in its own launches: the same bits."""
+    cfg, lay = v3p.cfg, v3p.layer
+    assert not lay.shared_in_grouped
     want = lay.out.clone()
-    lay.shared_grouped = "off"
-    lay._T = -1                                   # re-allocate in the separate form
+    lay.shared_grouped = True
+    lay._T = -1                                   # re-allocate with the extra group
     got = lay.forward(v3p.u_dev)
     torch.cuda.synchronize()
     assert L.moe_get_device_status() == 0
-    assert not lay.shared_in_grouped
+    assert lay.shared_in_grouped
     assert torch.equal(got, want)
-    lay.shared_grouped = "auto"
+    rk = cfg.T * cfg.top_k
+    assert torch.equal(lay.x_perm[rk:].cpu(), v3p.u)
+    _dispatch_invariants(lay, cfg.T, cfg.top_k, cfg.n_routed)
+    lay.shared_grouped = False
     lay._T = -1
