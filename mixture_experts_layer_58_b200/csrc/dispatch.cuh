@@ -44,7 +44,7 @@ permute_index_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict_
                      int32_t* __restrict__ src_token) {
   __shared__ int s_scan[256];
   __shared__ int s_next[256];          // next row of each expert
-  __shared__ int s_wcnt[8][256];       // this round: rows per (warp, expert), then their first row
+  __shared__ int s_wcnt[8][256];       // this batch of 256 pairs: rows per (warp, expert), then their first row
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -120,7 +120,7 @@ permute_index_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict_
       }
       pos_c[i] = p;
     }
-    __syncthreads();                              // s_wcnt is cleared next round
+    __syncthreads();                              // s_wcnt is cleared for the next batch
   }
 }
 
