@@ -432,9 +432,16 @@ def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
     from mixture_experts_layer_58_b200 import dp
     T = u.shape[0]
     timers, recv_rows, snap = {}, [], {}
+    use_graph = getattr(args, "graph", False) and world == 1 and not ep_mode
+    if use_graph:
+        # one CUDA graph per step (forward + bias update), reading u in place
+        lay.capture(T, u=u, bias_update=(cfg.gate_kind == "sigmoid"))
 
     def step(i=None):
-        lay.forward(u, timers=timers if i is not None else None)
+        if use_graph:
+            lay.replay(u)
+        else:
+            lay.forward(u, timers=timers if i is not None else None)
         if i == 0:
             snap["idx0"] = lay.topk_idx.clone()
             snap["counts0"] = lay.counts.clone()
@@ -442,7 +449,8 @@ def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
             snap["counts1"] = lay.counts.clone()
         if ep_mode and i is not None and hasattr(lay, "last_plan"):
             recv_rows.append(lay.last_plan.n_recv)
-        bias_step(lay, cfg, T, world, ep_mode)
+        if not use_graph:
+            bias_step(lay, cfg, T, world, ep_mode)
 
     for _ in range(args.warmup):
         step()
@@ -469,6 +477,13 @@ def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
         ms = float(tt.item())
     if L.moe_get_device_status() != 0:
         raise SystemExit("device timeout during the timed region")
+    if use_graph:
+        # stage times from eager steps after the timed region (a graph
+        # records no events between its kernels)
+        for _ in range(max(3, min(args.steps, 5))):
+            lay.forward(u, timers=timers)
+            bias_step(lay, cfg, T, world, ep_mode)
+        torch.cuda.synchronize()
     stage_ms = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in timers.items()}
     return {"ms_step": ms / args.steps, "stage_ms": stage_ms, "clocks": clk.summary(),
             "recv_rows": recv_rows, "bias0": bias0, **snap}
@@ -601,6 +616,8 @@ def main():
     ap.add_argument("--shared-join", default="auto", choices=["auto", "early", "late"],
                     help="where the overlapped shared expert rejoins: before the routed GEMMs "
                          "(early), before the combine (late), or by group size (auto)")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step (forward + bias update) as one CUDA graph (1 GPU)")
     ap.add_argument("--shared-grouped", action="store_true",
                     help="the shared expert as the last group of the routed grouped GEMMs "
                          "instead of its own launches beside the route and dispatch")
@@ -815,6 +832,8 @@ def main():
                             "fused gather" if lay.fused_gather else
                             "fused scatter and combine" if lay.fused_combine else
                             "fused scatter" if lay.fused_scatter else "five-call"),
+                   "launch": ("one CUDA graph per step" if getattr(args, "graph", False)
+                              and world == 1 and not ep_mode else "eager"),
                    "route": ("gate GEMM split over K, then a warp-per-token top-K pass"
                              if lay.route_split else "gate GEMM and top-K in one fused pass"),
                    "shared_expert": ("group N_r of the routed grouped GEMMs (its rows "

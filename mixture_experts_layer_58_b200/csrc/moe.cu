@@ -11,6 +11,7 @@
 #include <cstring>
 #include <atomic>
 #include <mutex>
+#include <unordered_map>
 
 #include "moe.h"
 #include "dispatch.cuh"
@@ -145,8 +146,18 @@ int make_tmap_bf16_store32(CUtensorMap* map, void* base, uint64_t cols, uint64_t
 
 template <typename K>
 int set_smem(K kernel, size_t bytes) {
-  MOE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(bytes)));
+  // The attribute is per-process state of the kernel: set it when a launch
+  // needs more than any launch before (not per launch), so that launches
+  // recorded into a CUDA graph after a first eager call make no such call.
+  static std::mutex mu;
+  static std::unordered_map<const void*, size_t> set;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& cur = set[reinterpret_cast<const void*>(kernel)];
+  if (bytes > cur) {
+    MOE_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(bytes)));
+    cur = bytes;
+  }
   return MOE_OK;
 }
 

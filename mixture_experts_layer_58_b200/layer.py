@@ -398,7 +398,8 @@ class MoELayer:
         side = None
         if T > 0 and self.ws13 is not None and self.overlap_shared and not self._grouped:
             side = self._fork()
-            u.record_stream(side)
+            if not torch.cuda.is_current_stream_capturing():
+                u.record_stream(side)
             with torch.cuda.stream(side):
                 with ev("shared"):
                     if train:
@@ -577,6 +578,56 @@ class MoELayer:
         if self.gate_kind == "sigmoid":
             self.update_bias()
         return out
+
+    # ------------------------------------------------------------------ CUDA graph
+    def capture(self, T: int, residual: bool = True, bias_update: bool = True, u=None):
+        """Record one step for batches of T tokens (the forward and, for the
+        sigmoid gate with bias_update, the end-of-step bias update) into a CUDA
+        graph, so that replay(u) runs all of it with one launch from the host.
+        The recorded launches keep this layer's buffers, workspaces and the
+        library's tile-counter slots: replays must follow one another on one
+        stream and not overlap eager calls of this layer. The shared expert's
+        side stream is part of the graph (forked and joined by events).
+        u: optional [T, d] bf16 device tensor the graph reads its input from
+        (the caller writes each batch into it; replay(u) then copies nothing);
+        by default the layer keeps its own input buffer."""
+        self.allocate(T)
+        dev = self.device
+        if u is not None:
+            assert u.shape == (T, self.d) and u.dtype == torch.bfloat16 and u.is_contiguous()
+            self._gu = u
+        else:
+            self._gu = torch.zeros((T, self.d), dtype=torch.bfloat16, device=dev)
+        self._gout = torch.empty((T, self.d), dtype=torch.bfloat16, device=dev)
+        self._g_bias = bias_update and self.gate_kind == "sigmoid"
+        # one eager pass first: library initialisation and kernel attributes
+        # happen outside the capture
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.forward(self._gu, residual=residual, out=self._gout)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.forward(self._gu, residual=residual, out=self._gout)
+            if self._g_bias:
+                self.update_bias()
+        self._graph = g
+        return self._gout
+
+    def replay(self, u):
+        """One recorded step on the bf16 batch u [T, d] (device): u is copied
+        into the graph's input buffer first. Returns the graph's output buffer
+        (overwritten by the next replay)."""
+        g = getattr(self, "_graph", None)
+        if g is None:
+            raise RuntimeError("capture(T) first")
+        assert u.shape == self._gu.shape and u.dtype == torch.bfloat16
+        if u.data_ptr() != self._gu.data_ptr():
+            self._gu.copy_(u)
+        g.replay()
+        return self._gout
 
     # kernels launched by one step(): route (1, split over K 2; + a memset), permute (3; FP8:
     # + the activation quantisation), routed and shared FFN, combine (1),

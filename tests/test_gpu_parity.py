@@ -347,3 +347,31 @@ def test_shared_expert_as_a_routed_group_bit_identical(name, T):
     assert b.layer.shared_in_grouped
     assert torch.equal(got, want)
     _full_check(b)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid", "v3d"])
+def test_cuda_graph_replay_matches_eager_steps(name):
+    """capture(T) records a step (forward + bias update) as one CUDA graph,
+    side stream included: three replays give the same outputs and biases bit
+    for bit as three eager steps on the same inputs (Tiny: 1-CTA tiles and
+    the shared expert joined late; Mid: pair tiles, joined early; V3 decode:
+    the split-K route)."""
+    cfg = synth.CONFIGS[name]
+    a = Inputs(cfg)
+    want = []
+    for _ in range(3):
+        want.append(a.layer.step(a.u_dev).clone())
+    torch.cuda.synchronize()
+    bias_a = a.layer.bias.clone()
+    del a
+    torch.cuda.empty_cache()
+    b = Inputs(cfg)
+    b.layer.capture(cfg.T)
+    torch.cuda.synchronize()
+    assert torch.equal(b.layer.bias, b.b.to(b.layer.bias.device))   # capture changes nothing
+    for k in range(3):
+        got = b.layer.replay(b.u_dev)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want[k]), f"replay {k}"
+    assert torch.equal(b.layer.bias, bias_a)
+    assert L.moe_get_device_status() == 0
