@@ -421,7 +421,7 @@ def bias_step(lay, cfg, T, world, ep_mode):
         lay.update_bias()
 
 
-def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
+def time_forward(lay, u, cfg, args, world, ep_mode, local, stream, graph=None):
     """W warm-up steps, then K timed steps between barriers and device
     syncs (CUDA events on the launching stream, clocks sampled throughout).
     A step is the forward plus the bias update. Returns the timings and the
@@ -432,10 +432,16 @@ def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
     from mixture_experts_layer_58_b200 import dp
     T = u.shape[0]
     timers, recv_rows, snap = {}, [], {}
-    use_graph = getattr(args, "graph", False) and world == 1 and not ep_mode
+    want_graph = getattr(args, "graph", False) if graph is None else graph
+    use_graph = want_graph and world == 1 and not ep_mode
     if use_graph:
         # one CUDA graph per step (forward + bias update), reading u in place
-        lay.capture(T, u=u, bias_update=(cfg.gate_kind == "sigmoid"))
+        try:
+            lay.capture(T, u=u, bias_update=(cfg.gate_kind == "sigmoid"))
+        except RuntimeError as exc:            # capture refused: time the eager steps
+            print(f"CUDA graph capture failed ({exc}); timing eager steps", file=sys.stderr)
+            use_graph = False
+            torch.cuda.synchronize()
 
     def step(i=None):
         if use_graph:
@@ -486,7 +492,7 @@ def time_forward(lay, u, cfg, args, world, ep_mode, local, stream):
         torch.cuda.synchronize()
     stage_ms = {n: sum(a.elapsed_time(b) for a, b in v) / len(v) for n, v in timers.items()}
     return {"ms_step": ms / args.steps, "stage_ms": stage_ms, "clocks": clk.summary(),
-            "recv_rows": recv_rows, "bias0": bias0, **snap}
+            "recv_rows": recv_rows, "bias0": bias0, "graph": use_graph, **snap}
 
 
 def decode_hbm(cfg, counts, ms_step, pk):
@@ -551,13 +557,18 @@ def variant_line(name, args, dev, local, stream, pk):
     torch.cuda.empty_cache()
     u = synth.tokens(cfg).to(dev)
     lay.allocate(cfg.T)
-    t = time_forward(lay, u, cfg, args, 1, False, local, stream)
+    # decode-sized batches: one CUDA graph per step (the launches are a
+    # visible part of a 3 ms step); prefill: eager (measured equal)
+    decode = cfg.T * cfg.top_k < 256 * cfg.n_routed
+    t = time_forward(lay, u, cfg, args, 1, False, local, stream,
+                     graph=(args.graph or decode))
     T, K = cfg.T, cfg.top_k
     line = {"workload": cfg.name, "T": T, "gate": cfg.gate_kind,
             "dtype": "e4m3 (fp32 promotion)" if cfg.fp8 else "bf16",
             "ms_per_step": t["ms_step"], "value": T / (t["ms_step"] * 1e-3),
             "unit": "tokens/s", "steps": args.steps, "warmup": args.warmup,
             "stage_ms": t["stage_ms"], "clocks": t["clocks"],
+            "launch": "one CUDA graph per step" if t["graph"] else "eager",
             "gpu_launches": args.steps * lay.launches_per_step(),
             "max_expert_load": {"first_timed_step": int(t["counts0"].max()),
                                 "last_timed_step": int(t["counts1"].max())}}
@@ -832,8 +843,7 @@ def main():
                             "fused gather" if lay.fused_gather else
                             "fused scatter and combine" if lay.fused_combine else
                             "fused scatter" if lay.fused_scatter else "five-call"),
-                   "launch": ("one CUDA graph per step" if getattr(args, "graph", False)
-                              and world == 1 and not ep_mode else "eager"),
+                   "launch": "one CUDA graph per step" if t["graph"] else "eager",
                    "route": ("gate GEMM split over K, then a warp-per-token top-K pass"
                              if lay.route_split else "gate GEMM and top-K in one fused pass"),
                    "shared_expert": ("group N_r of the routed grouped GEMMs (its rows "
