@@ -364,6 +364,31 @@ inline int route_splits(int T, int d) {
   return (num_kb + per - 1) / per;
 }
 
+// CTA-pair route (one cluster per 256 tokens): tmE2 boxes half of the
+// centroid rows (n_pad2 / 2, n_pad2 a multiple of 32).
+template <int TOPK>
+int launch_route_pair(int kind, const CUtensorMap& tmU, const CUtensorMap& tmE2, const float* bias,
+                      int T, int d, int n_routed, int n_pad2, uint32_t tcols, float scale,
+                      int32_t* idx, float* gate, int32_t* counts, unsigned int* status,
+                      cudaStream_t st) {
+  const size_t smem = RoutePairSmem::bytes(n_pad2);
+  const int ctas = 2 * ((T + 2 * kBM - 1) / (2 * kBM));
+  int rc;
+  if (kind == MOE_GATE_SIGMOID_BIAS) {
+    auto k = route_pair_kernel<TOPK, 0>;
+    if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
+    k<<<ctas, kGemmThreads, smem, st>>>(tmU, tmE2, bias, T, d, n_routed, n_pad2, tcols, scale, idx,
+                                        gate, counts, status);
+  } else {
+    auto k = route_pair_kernel<TOPK, 1>;
+    if ((rc = set_smem(k, smem)) != MOE_OK) return rc;
+    k<<<ctas, kGemmThreads, smem, st>>>(tmU, tmE2, bias, T, d, n_routed, n_pad2, tcols, scale, idx,
+                                        gate, counts, status);
+  }
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
 template <int TOPK>
 int launch_route_k(int kind, const CUtensorMap& tmU, const CUtensorMap& tmE, const float* bias,
                    int T, int d, int n_routed, int n_pad, uint32_t tcols, float scale,
@@ -496,6 +521,34 @@ int route_impl(const void* u, const void* centroids, const float* bias, int T, i
   if ((rc = make_tmap_bf16(&tmE, centroids, d, n_routed, n_pad)) != MOE_OK) return rc;
   const float* b = (kind == MOE_GATE_SIGMOID_BIAS) ? bias : nullptr;
   const int splits = partial ? route_splits(T, d) : 1;
+  // one pass over K with at least one full pair of 128-token blocks: the
+  // CTA-pair kernel (N = N_r padded to 32, half of it per CTA)
+  const bool pair = partial == nullptr && T >= 2 * kBM;
+  const int n_pad2 = std::max(32, (n_routed + 31) / 32 * 32);
+  uint32_t tcols2 = 32;
+  while (tcols2 < static_cast<uint32_t>(n_pad2)) tcols2 <<= 1;
+  CUtensorMap tmE2;
+  if (pair && (rc = make_tmap_bf16(&tmE2, centroids, d, n_routed, n_pad2 / 2)) != MOE_OK)
+    return rc;
+#define MOE_ROUTE_PAIR_CASE(KK)                                                                \
+  case KK:                                                                                     \
+    return launch_route_pair<KK>(kind, tmU, tmE2, b, T, d, n_routed, n_pad2, tcols2,           \
+                                 routed_scale, topk_idx, topk_gate, expert_counts, di->status, \
+                                 st);
+  if (pair) {
+    switch (top_k) {
+      MOE_ROUTE_PAIR_CASE(1)
+      MOE_ROUTE_PAIR_CASE(2)
+      MOE_ROUTE_PAIR_CASE(3)
+      MOE_ROUTE_PAIR_CASE(4)
+      MOE_ROUTE_PAIR_CASE(5)
+      MOE_ROUTE_PAIR_CASE(6)
+      MOE_ROUTE_PAIR_CASE(7)
+      MOE_ROUTE_PAIR_CASE(8)
+      default: return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
+  }
+#undef MOE_ROUTE_PAIR_CASE
 #define MOE_ROUTE_CASE(KK)                                                                   \
   case KK:                                                                                   \
     return launch_route_k<KK>(kind, tmU, tmE, b, T, d, n_routed, n_pad, tcols, routed_scale, \

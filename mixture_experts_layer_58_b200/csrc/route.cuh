@@ -17,6 +17,7 @@
 // DeepSeekMoE forward listing — top-k of the raw logits, softmax over them.
 #pragma once
 #include "gemm.cuh"
+#include "gemm2sm.cuh"
 
 namespace moe {
 
@@ -258,6 +259,186 @@ route_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// CTA-pair form for large batches: a cluster of 2 CTAs takes 256 tokens, CTA
+// r its 128 token rows (the MMA's M side) and centroid rows [r*N_pad/2,
+// +N_pad/2) (half of its N side); the leader issues tcgen05.mma.cta_group::2
+// M = 256, N = N_pad over a 3-stage ring of two 64-wide K atoms per stage, and
+// each CTA's TMEM receives its 128 tokens x all N_pad logits, so the epilogue
+// is the one-CTA kernel's. Half the centroid bytes per SM and one barrier round
+// trip per eight MMAs. Synchronisation as the pair GEMM (gemm2sm.cuh): full[s]
+// on the leader counts both CTAs' TMA bytes, empty[s] and tfull in both CTAs
+// are committed by the leader; all waits bounded; no TMA multicast.
+constexpr int kRouteAtoms = 2;
+constexpr int kRouteStages2 = 3;
+
+struct RoutePairSmem {
+  static size_t bytes(int n_pad) {
+    return 1024 + static_cast<size_t>(kRouteStages2) * kRouteAtoms *
+                      (128 * kBK * 2 + (n_pad / 2) * kBK * 2) +
+           256 + 2 * kRouteMaxExperts * sizeof(float);
+  }
+};
+
+template <int TOPK, int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+route_pair_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
+                  const float* __restrict__ bias, int T, int d, int n_routed, int n_pad,
+                  uint32_t tmem_cols, float routed_scale, int32_t* __restrict__ topk_idx,
+                  float* __restrict__ topk_gate, int32_t* __restrict__ counts,
+                  unsigned int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const int a_atom = 128 * kBK * 2;              // this CTA's 128 token rows, one K atom
+  const int b_atom = (n_pad / 2) * kBK * 2;      // this CTA's half of the centroids
+  const int a_stage = kRouteAtoms * a_atom;
+  const int b_stage = kRouteAtoms * b_atom;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kRouteStages2 * a_stage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kRouteStages2 * b_stage);
+  uint64_t* empty = full + kRouteStages2;
+  uint64_t* tfull = empty + kRouteStages2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+  float* s_bias = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);
+  int* s_hist = reinterpret_cast<int*>(s_bias + kRouteMaxExperts);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int num_st = d / (kBK * kRouteAtoms);    // d % 256 == 0
+  const int row0 = static_cast<int>(blockIdx.x >> 1) * (2 * kBM) + static_cast<int>(rank) * kBM;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < kRouteStages2; ++s) {
+        mbar_init(&full[s], 1);
+        mbar_init(&empty[s], 1);
+      }
+      mbar_init(tfull, 1);
+      fence_mbar_init();
+      tma_prefetch_desc(&tmU);
+      tma_prefetch_desc(&tmE);
+    }
+    __syncwarp();
+    tmem_alloc_2sm(tmem_slot, tmem_cols);
+    tmem_relinquish_2sm();
+  } else if (warp >= 2) {
+    for (int e = threadIdx.x - 64; e < kRouteMaxExperts; e += 128) {
+      s_bias[e] = (KIND == 0 && bias != nullptr && e < n_routed) ? bias[e] : 0.0f;
+      s_hist[e] = 0;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();   // both CTAs' barriers initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, issued_par = 0;
+    const uint32_t stage_tx = 2u * kRouteAtoms * static_cast<uint32_t>(a_atom + b_atom);
+    for (int st = 0; st < num_st; ++st) {
+      if (!mbar_wait(&empty[stage], phase ^ 1u, status, kStatusTimeoutProducer)) break;
+      if (rank == 0) mbar_arrive_expect_tx(&full[stage], stage_tx);
+      const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+#pragma unroll
+      for (int at = 0; at < kRouteAtoms; ++at) {
+        const int x = (st * kRouteAtoms + at) * kBK;
+        tma_load_2d_pair(sA + stage * a_stage + at * a_atom, &tmU, bar, x, row0);
+        tma_load_2d_pair(sB + stage * b_stage + at * b_atom, &tmE, bar, x,
+                         static_cast<int>(rank) * (n_pad / 2));
+      }
+      issued |= 1u << stage;
+      issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+      if (++stage == kRouteStages2) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    // the leader's full barriers count both CTAs' bytes: once they have
+    // completed no TMA write into either CTA's shared memory is in flight
+    if (rank == 0)
+      for (int s = 0; s < kRouteStages2; ++s)
+        if (issued & (1u << s))
+          mbar_wait(&full[s], (issued_par >> s) & 1u, status, kStatusTimeoutProducer);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    const uint32_t idesc = idesc_bf16_f32(2 * kBM, n_pad);
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int st = 0; st < num_st; ++st) {
+      if (!mbar_wait(&full[stage], phase, status, kStatusTimeoutMma)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int at = 0; at < kRouteAtoms; ++at) {
+        const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * a_stage + at * a_atom));
+        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * b_stage + at * b_atom));
+#pragma unroll
+        for (int k = 0; k < kBK / kUmmaK; ++k)
+          umma_bf16_pair(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc, (st | at | k) != 0);
+      }
+      const uint32_t e = smem_u32(&empty[stage]);
+      umma_commit_pair(mapa_shared(e, 0));
+      umma_commit_pair(mapa_shared(e, 1));
+      if (++stage == kRouteStages2) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    // tfull of both CTAs fires when every MMA above has completed (also on the
+    // error path, so TMEM is never released under a running MMA)
+    const uint32_t f = smem_u32(tfull);
+    umma_commit_pair(mapa_shared(f, 0));
+    umma_commit_pair(mapa_shared(f, 1));
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int t = row0 + quarter * 32 + lane;
+    const bool have = mbar_wait(tfull, 0, status, kStatusTimeoutEpilogue);
+    tc_fence_after();
+    float kv[TOPK], sv[TOPK];
+    int ki[TOPK];
+#pragma unroll
+    for (int p = 0; p < TOPK; ++p) {
+      kv[p] = -INFINITY;
+      sv[p] = 0.0f;
+      ki[p] = -1;
+    }
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    if (have) {
+      for (int c = 0; c < n_pad; c += 32) {
+        uint32_t zr[32];
+        tmem_ld_32cols(taddr + c, zr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int j = c + i;
+          if (j < n_routed)
+            route_insert<TOPK, KIND>(__uint_as_float(zr[i]), j, s_bias[j], kv, sv, ki);
+        }
+      }
+    }
+    tc_fence_before();
+    if (have && t < T)
+      route_emit<TOPK, KIND>(sv, ki, routed_scale, t, topk_idx, topk_gate, s_hist);
+    named_bar_sync(1, 128);
+    for (int e = threadIdx.x - 64; e < n_routed; e += 128) {
+      const int c = s_hist[e];
+      if (c) atomicAdd(&counts[e], c);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();   // neither CTA leaves while the pair may still signal it
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_2sm(tmem_base, tmem_cols);
   }
 }
 

@@ -1,5 +1,6 @@
 """The split-K gate GEMM (moe_route_splitk) against the fp64 oracle and
-against the one-pass moe_route on the same inputs: selection bit-exact away
+against the one-pass moe_route (one CTA per 128 tokens below 256 tokens,
+CTA pairs from 256) on the same inputs: selection bit-exact away
 from near-ties, gates and loads as the oracle's, ragged and degenerate
 shapes, the workspace contract. Needs a B200."""
 import numpy as np
@@ -61,6 +62,10 @@ CASES = [
     ("tiny", 64, {"n_routed": 20, "top_k": 2}),          # 20 experts: padded MMA columns
     ("tiny", 64, {"gate_kind": "softmax", "bias_lo": 0.0, "bias_hi": 0.0}),
     ("tiny", 64, {"n_routed": 8, "top_k": 8}),           # every expert selected
+    # T >= 256: moe_route takes the CTA-pair kernel (N = N_r padded to 32)
+    ("tiny", 300, {"n_routed": 20, "top_k": 2}),
+    ("tiny", 300, {"n_routed": 8, "top_k": 8}),
+    ("tiny", 513, {"gate_kind": "softmax", "bias_lo": 0.0, "bias_hi": 0.0}),
     ("mid", 1000, {}),
     ("v3d", 128, {}),                                    # V3 decode: d 7168, 256 experts, top-8
     ("v3d", 2048, {}),
