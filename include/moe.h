@@ -98,7 +98,9 @@ typedef void* moe_stream_t; /* cudaStream_t */
  *   expert_counts [n_routed] int32 out, OVERWRITTEN (not accumulated):
  *              number of (token, slot) pairs routed to each expert.
  * Logits are accumulated in fp32 on the tensor cores from the bf16 inputs;
- * sigmoid, keys and gates are fp32.
+ * sigmoid, keys and gates are fp32. Batches of 256 tokens or more run on CTA
+ * pairs (256 tokens per cluster), smaller ones one CTA per 128 tokens; the
+ * results follow from the logits the same way.
  */
 MOE_API int moe_route(const void* u, const void* centroids, const float* bias, int T, int d,
                       int n_routed, int top_k, moe_gate_kind kind, float routed_scale,
