@@ -101,6 +101,7 @@ class MoELayer:
         if shared_join not in ("auto", "early", "late"):
             raise ValueError("shared_join must be 'auto', 'early' or 'late'")
         self.shared_join = shared_join
+        self.shared_after_route = False
         # split_route: the gate GEMM split over K (moe_route_splitk) -- "on",
         # "off" or "auto" (on for batches of at most 2048 tokens, where
         # moe_route's 128-token CTAs would leave most SMs idle)
@@ -396,19 +397,31 @@ class MoELayer:
         self._grouped = self.shared_in_grouped and not train
         ev = _Timed(timers)
         side = None
-        if T > 0 and self.ws13 is not None and self.overlap_shared and not self._grouped:
-            side = self._fork()
+
+        def fork_shared():
+            s = self._fork()
             if not torch.cuda.is_current_stream_capturing():
-                u.record_stream(side)
-            with torch.cuda.stream(side):
+                u.record_stream(s)
+            with torch.cuda.stream(s):
                 with ev("shared"):
                     if train:
                         self._shared_ffn_train(u)
                     else:
                         self.shared_ffn(u)
-            self._join_event.record(side)
+            self._join_event.record(s)
+            return s
+
+        overlap = T > 0 and self.ws13 is not None and self.overlap_shared and not self._grouped
+        # The route kernel needs about as much shared memory per SM as a GEMM
+        # CTA, so it cannot share SMs with the shared expert's persistent GEMM;
+        # the dispatch's kernels can. shared_after_route: start the shared
+        # expert once the route is done, beside the dispatch only.
+        if overlap and not self.shared_after_route:
+            side = fork_shared()
         with ev("route"):
             self.route(u)
+        if overlap and self.shared_after_route:
+            side = fork_shared()
         # Where the shared expert rejoins: the routed GEMMs of large groups
         # (CTA-pair form) are compute-bound like the shared expert itself, so
         # the shared expert overlaps only the HBM-bound route and dispatch and
