@@ -40,8 +40,10 @@ struct BwdCfg {
   // kWgOutBufs chunks before it to have read its buffer)
   static constexpr int kWgStages = 4;
   static constexpr int kWgOutBufs = 2;
+  static constexpr int kWgEpiWarps = 4;   // in groups of 4 (one per TMEM lane quarter)
+  static constexpr int kWgThreads = 64 + 32 * kWgEpiWarps;
   static constexpr int kOutBufBytes = 32 * 32 * 2;
-  static constexpr int kOutBytes = 4 * kWgOutBufs * kOutBufBytes;
+  static constexpr int kOutBytes = kWgEpiWarps * kWgOutBufs * kOutBufBytes;
   static size_t wgrad_smem_bytes(int G) {
     return 1024 + static_cast<size_t>(kWgStages) * kStageBytes + kOutBytes + kBarBytes +
            2 * static_cast<size_t>(G + 1) * sizeof(int);
@@ -306,7 +308,7 @@ grouped_dgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
 // wgrad: dW[g][m][n] = sum over the rows r of group g of A[r, m] B[r, n];
 // A [rows, M], B [rows, N], dW [G, M, N] bf16. Tiles (g, 128-row m block,
 // 256-column n block), m blocks fastest; a group without rows writes zeros.
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(BwdCfg::kWgThreads, 1)
 grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmD,
@@ -346,12 +348,12 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       for (int a = 0; a < 2; ++a) {
         mbar_init(&tfull[a], 1);
-        mbar_init(&tempty[a], 128);
+        mbar_init(&tempty[a], 32 * C::kWgEpiWarps);
       }
       mbar_init(mma_done, 1);
       for (int j = 0; j < kCtaTileQ; ++j) {
         mbar_init(&tq_full[j], 1);
-        mbar_init(&tq_empty[j], 5);   // MMA role + 4 epilogue warps
+        mbar_init(&tq_empty[j], 1 + C::kWgEpiWarps);   // MMA role + the epilogue warps
       }
       fence_mbar_init();
       tma_prefetch_desc(&tmA);
@@ -492,6 +494,8 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
     // row r sits at chunk q ^ ((r >> 1) & 3), so the 8 rows one phase of a
     // 16-B shared store touches fall in 8 different bank groups.
     const int quarter = warp & 3;
+    const int eg = (warp - 2) >> 2;   // group eg drains columns [eg * BN / groups, +BN / groups)
+    constexpr int kGroups = C::kWgEpiWarps / 4;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     uint8_t* obuf = sOut + (warp - 2) * C::kWgOutBufs * C::kOutBufBytes;
     const int sw = (lane >> 1) & 3;
@@ -517,7 +521,7 @@ grouped_wgrad_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
       const int y = g * M + m_blk * kBM + quarter * 32;
       const int ncols = min(BN, N - n_blk * BN);   // 128 or 256
 #pragma unroll 1
-      for (int c = 0; c < ncols; c += 64) {
+      for (int c = eg * (BN / kGroups); c < min(ncols, (eg + 1) * (BN / kGroups)); c += 64) {
         uint32_t r[2][32];
         tmem_ld_32cols(taddr + c, r[0]);
         tmem_ld_32cols(taddr + c + 32, r[1]);

@@ -332,7 +332,7 @@ int launch_wgrad(const void* A, const void* B, int rows, int M, int N, int G,
   const long long tiles = static_cast<long long>(G) * (M / kBM) *
                           ((N + BwdCfg::kBN - 1) / BwdCfg::kBN);
   const int grid = static_cast<int>(std::max(1LL, std::min<long long>(di->num_sms, tiles)));
-  grouped_wgrad_bf16_kernel<<<grid, kGemmThreads, smem, st>>>(tmA, tmB, tmD, offsets, G, M, N,
+  grouped_wgrad_bf16_kernel<<<grid, BwdCfg::kWgThreads, smem, st>>>(tmA, tmB, tmD, offsets, G, M, N,
                                                                rows, counter, di->status);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
