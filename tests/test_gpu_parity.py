@@ -269,6 +269,43 @@ def test_grouped_ffn_tile_paths_by_group_size(extra):
                     mean_tol=3e-3, what=f"group {i} ({b - a} rows)")
 
 
+def test_grouped_ffn_most_groups_pair_tiles():
+    """The largest group count (1024) on CTA-pair tiles: the group table in
+    shared memory at its biggest; sizes from 0 to 700 rows, with empty groups,
+    single-row groups and ragged tails. Every group against fp32 torch matmuls
+    of the same bf16 operands."""
+    G, d, inter = 1024, 256, 128
+    rng = np.random.default_rng(13)
+    sizes = rng.choice([0, 1, 33, 256, 257, 300, 511, 700], size=G,
+                       p=[0.05, 0.1, 0.1, 0.2, 0.1, 0.2, 0.15, 0.1])
+    rows = int(sizes.sum())
+    assert rows >= 256 * G                     # groups average >= 256 rows: pair tiles
+    g = torch.Generator(device="cuda").manual_seed(14)
+    x = torch.randn(rows, d, generator=g, device="cuda").bfloat16()
+    w1 = (0.05 * torch.randn(G, inter, d, generator=g, device="cuda")).bfloat16()
+    w3 = (0.05 * torch.randn(G, inter, d, generator=g, device="cuda")).bfloat16()
+    w2 = (0.05 * torch.randn(G, d, inter, generator=g, device="cuda")).bfloat16()
+    w13 = torch.empty(G, 2 * inter, d, dtype=torch.bfloat16, device="cuda")
+    L.moe_pack_w13(w1, w3, G, inter, d, w13)
+    off = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32, device="cuda")
+    y = torch.full((rows, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    wsb = L.moe_grouped_ffn_workspace_size(rows, inter)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    L.moe_grouped_ffn(x, None, off, G, rows, d, inter, w13, None, w2, None, L.MOE_BF16, y, ws, wsb)
+    torch.cuda.synchronize()
+    assert L.moe_get_device_status() == 0
+    o = off.cpu().tolist()
+    for i in range(G):
+        a, b = o[i], o[i + 1]
+        if a == b:
+            continue
+        xa = x[a:b].float()
+        h = (torch.nn.functional.silu(xa @ w1[i].float().T) * (xa @ w3[i].float().T)).bfloat16()
+        ref = h.float() @ w2[i].float().T
+        check_close(y[a:b].float().cpu().numpy(), ref.cpu().numpy(), max_tol=1e-2,
+                    mean_tol=3e-3, what=f"group {i} ({b - a} rows)")
+
+
 @pytest.mark.parametrize("name,T", [("tiny", None), ("tiny", 383), ("mid", None)])
 def test_fused_gather_layer_matches_oracle(name, T):
     """The fused mode: dispatch computes only row indices and the up-projection
